@@ -1,0 +1,165 @@
+"""Float64 CPU oracle for the delta-rule sequence mixer (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY: only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference arm of ``bench.py`` may import this package.  The
+product library never loads it, and it never loads the product library.
+
+* ``deltanet``     - the per-token delta rule (optionally gated), ``oracle.c``.
+* ``linear_attn``  - ELU+1 causal linear attention, ``oracle.c``.
+* ``chunk_form``   - the chunkwise WY form in numpy (see ``chunk_form.py``).
+
+Inputs may be numpy arrays or CPU torch tensors; bfloat16 tensors are passed as
+their bit patterns and widened exactly inside the C code.  Results are float64
+numpy arrays.  Parity: pinned (``tests/test_oracle_pins.py``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import time
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` next to it (plain gcc)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm", "-lpthread"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        vp, fp, dp, L, I = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                            ctypes.c_long, ctypes.c_int)
+        lib.oracle_deltanet.argtypes = [vp, vp, vp, I, fp, fp, dp, dp, dp, L, L, L, L, L, I]
+        lib.oracle_deltanet.restype = I
+        lib.oracle_linear_attn.argtypes = [vp, vp, vp, I, dp, dp, dp, dp, dp, L, L, L, L, L, I]
+        lib.oracle_linear_attn.restype = I
+        _lib = lib
+    return _lib
+
+
+def _as_stored(x):
+    """Return (contiguous numpy array of the stored bits, dtype code)."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), BF16
+            if x.dtype == torch.float32:
+                return x.numpy(), F32
+            raise TypeError(f"oracle inputs must be float32 or bfloat16, got {x.dtype}")
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.uint16:
+        return x, BF16
+    raise TypeError(f"oracle inputs must be float32 or bfloat16 bits, got {x.dtype}")
+
+
+def _f32(x):
+    if x is None:
+        return None
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().float().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _f64(x):
+    if x is None:
+        return None
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().double().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def deltanet(q, k, v, beta, alpha=None, S0=None, nthreads: int = 0):
+    """Delta rule over (B,H,T,D) sequences; returns ``(o, S_out)`` in float64.
+
+    Follows the direct per-token loop of "GPT-2 から Kimi K3 まで" (news.ainew.jp),
+    section "DeltaNet (Parallelizing linear transformers with delta rule)", with
+    the gate of the Gated DeltaNet paragraph of "How a Baseten Engineer Traced 7
+    Years of Attention Mechanism Evolution" (decay first, then the delta write).
+    """
+    qa, dt = _as_stored(q)
+    ka, dtk = _as_stored(k)
+    va, dtv = _as_stored(v)
+    if not (dt == dtk == dtv):
+        raise TypeError("q, k, v must share one dtype")
+    B, H, T, Dk = qa.shape
+    Dv = va.shape[-1]
+    if ka.shape != (B, H, T, Dk) or va.shape != (B, H, T, Dv):
+        raise ValueError("shape mismatch")
+    b = _f32(beta).reshape(B, H, T)
+    a = None if alpha is None else _f32(alpha).reshape(B, H, T)
+    s0 = None if S0 is None else _f64(S0).reshape(B, H, Dk, Dv)
+    o = np.zeros((B, H, T, Dv), np.float64)
+    S = np.zeros((B, H, Dk, Dv), np.float64)
+    rc = _load().oracle_deltanet(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(b), _ptr(a), _ptr(s0),
+                                 _ptr(o), _ptr(S), B, H, T, Dk, Dv, nthreads)
+    if rc != 0:
+        raise RuntimeError(f"oracle_deltanet failed ({rc})")
+    return o, S
+
+
+def linear_attn(q, k, v, S0=None, z0=None, nthreads: int = 0):
+    """ELU+1 causal linear attention; returns ``(o, S_out, z_out)`` in float64.
+
+    Follows the cached forward of "GPT-2 から Kimi K3 まで" (news.ainew.jp),
+    section "Linear attention", one token at a time.
+    """
+    qa, dt = _as_stored(q)
+    ka, _ = _as_stored(k)
+    va, _ = _as_stored(v)
+    B, H, T, Dk = qa.shape
+    Dv = va.shape[-1]
+    s0 = None if S0 is None else _f64(S0).reshape(B, H, Dk, Dv)
+    z0_ = None if z0 is None else _f64(z0).reshape(B, H, Dk)
+    o = np.zeros((B, H, T, Dv), np.float64)
+    S = np.zeros((B, H, Dk, Dv), np.float64)
+    z = np.zeros((B, H, Dk), np.float64)
+    rc = _load().oracle_linear_attn(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(s0), _ptr(z0_),
+                                    _ptr(o), _ptr(S), _ptr(z), B, H, T, Dk, Dv, nthreads)
+    if rc != 0:
+        raise RuntimeError(f"oracle_linear_attn failed ({rc})")
+    return o, S, z
+
+
+def timed(fn, *args, **kw):
+    """Run ``fn`` once and return (result, wall seconds)."""
+    t0 = time.perf_counter()
+    r = fn(*args, **kw)
+    return r, time.perf_counter() - t0

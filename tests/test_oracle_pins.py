@@ -1,0 +1,286 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+None of these re-types the oracle's loop: each checks a property the pages
+state, a closed form, an independent expansion, or a hand-worked fixture.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, rng):
+    return rng.standard_normal(shape).astype(np.float32)
+
+
+def _unit_rows(x):
+    return (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(np.float32)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _seq(a, D=None):
+    """(T, D) list -> (1, 1, T, D) float32 array."""
+    a = np.asarray(a, np.float32)
+    return a.reshape((1, 1) + a.shape)
+
+
+# -- hand-worked fixtures -------------------------------------------------------
+
+def test_golden_delta_rule(oracle_mod):
+    g = _golden("delta_rule_worked.json")
+    o, S = oracle_mod.deltanet(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]),
+                               np.asarray(g["beta"], np.float32).reshape(1, 1, -1))
+    np.testing.assert_allclose(o[0, 0], g["o"], atol=2e-6)
+    np.testing.assert_allclose(S[0, 0], g["S"], atol=2e-6)
+
+
+def test_golden_gated_scalar(oracle_mod):
+    g = _golden("gated_scalar_worked.json")
+    o, S = oracle_mod.deltanet(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]),
+                               np.asarray(g["beta"], np.float32).reshape(1, 1, -1),
+                               alpha=np.asarray(g["alpha"], np.float32).reshape(1, 1, -1))
+    np.testing.assert_allclose(o[0, 0], g["o"], atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], g["S"], atol=1e-12)
+
+
+def test_golden_linear_attn(oracle_mod):
+    g = _golden("linear_attn_worked.json")
+    o, S, z = oracle_mod.linear_attn(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]))
+    np.testing.assert_allclose(o[0, 0], g["o"], rtol=1e-6)
+    np.testing.assert_allclose(S[0, 0], g["S"], rtol=1e-6)
+    np.testing.assert_allclose(z[0, 0], g["z"], rtol=1e-6)
+
+
+# -- properties the pages state ---------------------------------------------------
+
+def test_zero_write_strength_keeps_state(oracle_mod):
+    """beta = 0: nothing is written, so S stays S0 and o_t = q_t S0."""
+    rng = np.random.default_rng(1)
+    B, H, T, Dk, Dv = 2, 3, 17, 8, 5
+    q, k, v = _rand((B, H, T, Dk), rng), _unit_rows(_rand((B, H, T, Dk), rng)), _rand((B, H, T, Dv), rng)
+    S0 = rng.standard_normal((B, H, Dk, Dv))
+    o, S = oracle_mod.deltanet(q, k, v, np.zeros((B, H, T), np.float32), S0=S0)
+    np.testing.assert_allclose(S, S0, rtol=0, atol=0)
+    np.testing.assert_allclose(o, np.einsum("bhti,bhij->bhtj", q.astype(np.float64), S0), atol=1e-12)
+
+
+def test_zero_delta_when_value_already_stored(oracle_mod):
+    """v_t equal to what k_t reads from the state: the delta is zero, S is unchanged."""
+    rng = np.random.default_rng(2)
+    B, H, T, Dk, Dv = 1, 2, 23, 6, 7
+    q, k = _rand((B, H, T, Dk), rng), _unit_rows(_rand((B, H, T, Dk), rng))
+    beta = rng.uniform(0.1, 1.0, (B, H, T)).astype(np.float32)
+    S0 = rng.standard_normal((B, H, Dk, Dv)).astype(np.float32).astype(np.float64)
+    v32 = np.einsum("bhti,bhij->bhtj", k.astype(np.float64), S0).astype(np.float32)
+    o, S = oracle_mod.deltanet(q, k, v32, beta, S0=S0)
+    # the only residual is v32's float32 rounding of k S0
+    resid = np.abs(v32.astype(np.float64) - np.einsum("bhti,bhij->bhtj", k.astype(np.float64), S0)).max()
+    assert np.abs(S - S0).max() <= 4 * T * resid + 1e-12
+    np.testing.assert_allclose(o, np.einsum("bhti,bhij->bhtj", q.astype(np.float64), S0),
+                               atol=4 * T * resid * np.sqrt(Dk) + 1e-12)
+
+
+def test_unit_key_full_strength_overwrites(oracle_mod):
+    """beta = 1 and |k| = 1: after the write, k_t reads back exactly v_t (q_t = k_t)."""
+    rng = np.random.default_rng(3)
+    B, H, T, Dk, Dv = 2, 2, 40, 16, 9
+    k = _unit_rows(_rand((B, H, T, Dk), rng))
+    v = _rand((B, H, T, Dv), rng)
+    S0 = rng.standard_normal((B, H, Dk, Dv))
+    o, _ = oracle_mod.deltanet(k, k, v, np.ones((B, H, T), np.float32), S0=S0)
+    # |k|^2 differs from 1 only by float32 rounding of the normalised key
+    n2 = (k.astype(np.float64) ** 2).sum(-1, keepdims=True)
+    assert np.abs(n2 - 1).max() < 1e-6
+    np.testing.assert_allclose(o, v, atol=2e-5)
+
+
+def test_orthonormal_keys_closed_form(oracle_mod):
+    """Orthonormal keys (T <= Dk), S0 = 0: no read interference, so the deltas are
+    beta_t v_t and O = tril(Q K^T) diag(beta) V, S_T = K^T diag(beta) V."""
+    rng = np.random.default_rng(4)
+    Dk, Dv, T = 12, 6, 10
+    Kf = np.linalg.qr(rng.standard_normal((Dk, Dk)))[0][:T]  # orthonormal rows
+    k = Kf.astype(np.float32)
+    k64 = k.astype(np.float64)
+    q, v = _rand((T, Dk), rng), _rand((T, Dv), rng)
+    beta = rng.uniform(0, 1, T).astype(np.float32)
+    o, S = oracle_mod.deltanet(_seq(q), _seq(k), _seq(v), beta.reshape(1, 1, T))
+    # float32 rounding leaves k_s . k_t ~ 1e-7 off zero; the closed form holds to that order
+    G = k64 @ k64.T
+    off = np.abs(G - np.diag(np.diag(G))).max()
+    bv = beta[:, None].astype(np.float64) * v
+    S_ref = (k64 * 1.0).T @ (bv * 1.0)
+    O_ref = np.tril(q.astype(np.float64) @ k64.T) @ bv
+    np.testing.assert_allclose(S[0, 0], S_ref, atol=50 * off + 1e-6)
+    np.testing.assert_allclose(o[0, 0], O_ref, atol=50 * off * np.abs(q).max() * Dk + 1e-6)
+
+
+def test_householder_transition(oracle_mod):
+    """One token: S_1 = (I - beta k^T k) S0 + beta k^T v (generalised Householder form)."""
+    rng = np.random.default_rng(5)
+    Dk, Dv = 9, 4
+    k = _unit_rows(_rand((1, Dk), rng))
+    v, q = _rand((1, Dv), rng), _rand((1, Dk), rng)
+    S0 = rng.standard_normal((Dk, Dv))
+    beta = np.float32(0.37)
+    _, S = oracle_mod.deltanet(_seq(q), _seq(k), _seq(v), np.full((1, 1, 1), beta),
+                               S0=S0.reshape(1, 1, Dk, Dv))
+    k64, b = k.astype(np.float64), float(beta)
+    Hh = np.eye(Dk) - b * k64.T @ k64
+    np.testing.assert_allclose(S[0, 0], Hh @ S0 + b * k64.T @ v.astype(np.float64), atol=1e-12)
+
+
+def test_unrolled_transition_product(oracle_mod):
+    """Brute force on tiny inputs: S_T = sum_t (M_T ... M_{t+1}) N_t + (M_T ... M_1) S0 with
+    M_t = alpha_t (I - beta_t k_t^T k_t), N_t = beta_t k_t^T v_t; o_t = q_t S_t."""
+    rng = np.random.default_rng(6)
+    T, Dk, Dv = 7, 5, 3
+    q, k, v = _rand((T, Dk), rng), _unit_rows(_rand((T, Dk), rng)), _rand((T, Dv), rng)
+    beta = rng.uniform(0, 1, T).astype(np.float32)
+    alpha = rng.uniform(0.2, 1, T).astype(np.float32)
+    S0 = rng.standard_normal((Dk, Dv))
+    o, S = oracle_mod.deltanet(_seq(q), _seq(k), _seq(v), beta.reshape(1, 1, T),
+                               alpha=alpha.reshape(1, 1, T), S0=S0.reshape(1, 1, Dk, Dv))
+    K, V, Q = k.astype(np.float64), v.astype(np.float64), q.astype(np.float64)
+    Ms = [float(alpha[t]) * (np.eye(Dk) - float(beta[t]) * np.outer(K[t], K[t])) for t in range(T)]
+    Ns = [float(beta[t]) * np.outer(K[t], V[t]) for t in range(T)]
+    for t in range(T):
+        # expansion: S_t = (M_t...M_0) S0 + sum_{s<=t} (M_t...M_{s+1}) N_s
+        prod = np.eye(Dk)
+        acc = np.zeros((Dk, Dv))
+        for s in range(t, -1, -1):
+            acc += prod @ Ns[s]
+            prod = prod @ Ms[s]
+        St = prod @ S0 + acc
+        np.testing.assert_allclose(o[0, 0, t], Q[t] @ St, atol=1e-11)
+    np.testing.assert_allclose(S[0, 0], St, atol=1e-11)
+
+
+def test_gate_one_is_plain_deltanet(oracle_mod):
+    rng = np.random.default_rng(7)
+    B, H, T, D = 1, 2, 33, 8
+    q, k, v = _rand((B, H, T, D), rng), _unit_rows(_rand((B, H, T, D), rng)), _rand((B, H, T, D), rng)
+    beta = rng.uniform(0, 1, (B, H, T)).astype(np.float32)
+    o1, S1 = oracle_mod.deltanet(q, k, v, beta)
+    o2, S2 = oracle_mod.deltanet(q, k, v, beta, alpha=np.ones((B, H, T), np.float32))
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
+
+
+def test_gate_zero_wipes_then_writes(oracle_mod):
+    """alpha_t = 0: the state is wiped before the write, so S_t = beta_t k_t^T v_t."""
+    rng = np.random.default_rng(8)
+    T, Dk, Dv = 12, 6, 5
+    q, k, v = _rand((T, Dk), rng), _unit_rows(_rand((T, Dk), rng)), _rand((T, Dv), rng)
+    beta = rng.uniform(0, 1, T).astype(np.float32)
+    alpha = rng.uniform(0.3, 1, T).astype(np.float32)
+    alpha[-1] = 0.0
+    S0 = rng.standard_normal((1, 1, Dk, Dv))
+    _, S = oracle_mod.deltanet(_seq(q), _seq(k), _seq(v), beta.reshape(1, 1, T),
+                               alpha=alpha.reshape(1, 1, T), S0=S0)
+    np.testing.assert_allclose(S[0, 0], float(beta[-1]) * np.outer(k[-1], v[-1]).astype(np.float64),
+                               atol=1e-12)
+
+
+def test_resume_equals_one_shot(oracle_mod):
+    """Carrying S across two calls equals one call over the concatenated sequence
+    (the cache contract of the pages' forward(x, cache))."""
+    rng = np.random.default_rng(9)
+    B, H, T1, T2, D = 2, 2, 19, 13, 8
+    T = T1 + T2
+    q, k, v = _rand((B, H, T, D), rng), _unit_rows(_rand((B, H, T, D), rng)), _rand((B, H, T, D), rng)
+    beta = rng.uniform(0, 1, (B, H, T)).astype(np.float32)
+    alpha = rng.uniform(0.5, 1, (B, H, T)).astype(np.float32)
+    o, S = oracle_mod.deltanet(q, k, v, beta, alpha=alpha)
+    s1, s2 = slice(0, T1), slice(T1, T)
+    oa, Sa = oracle_mod.deltanet(q[:, :, s1].copy(), k[:, :, s1].copy(), v[:, :, s1].copy(),
+                                 beta[:, :, s1].copy(), alpha=alpha[:, :, s1].copy())
+    ob, Sb = oracle_mod.deltanet(q[:, :, s2].copy(), k[:, :, s2].copy(), v[:, :, s2].copy(),
+                                 beta[:, :, s2].copy(), alpha=alpha[:, :, s2].copy(), S0=Sa)
+    np.testing.assert_allclose(np.concatenate([oa, ob], 2), o, atol=1e-12)
+    np.testing.assert_allclose(Sb, S, atol=1e-12)
+    # linear attention carries (S, z) the same way
+    lo, lS, lz = oracle_mod.linear_attn(q, k, v)
+    la, lSa, lza = oracle_mod.linear_attn(q[:, :, s1].copy(), k[:, :, s1].copy(), v[:, :, s1].copy())
+    lb, lSb, lzb = oracle_mod.linear_attn(q[:, :, s2].copy(), k[:, :, s2].copy(), v[:, :, s2].copy(),
+                                          S0=lSa, z0=lza)
+    np.testing.assert_allclose(np.concatenate([la, lb], 2), lo, rtol=1e-12)
+    np.testing.assert_allclose(lSb, lS, rtol=1e-12)
+    np.testing.assert_allclose(lzb, lz, rtol=1e-12)
+
+
+def test_linear_attn_matmul_closed_form(oracle_mod):
+    """Causal ELU+1 linear attention equals its matmul (C = N) form:
+    O = tril(Q' K'^T) V / tril(Q' K'^T) 1, S_T = K'^T V, z_T = K'^T 1, with the feature
+    map taken from torch's ELU."""
+    rng = np.random.default_rng(10)
+    B, H, T, Dk, Dv = 2, 2, 37, 8, 6
+    q, k, v = _rand((B, H, T, Dk), rng), _rand((B, H, T, Dk), rng), _rand((B, H, T, Dv), rng)
+    o, S, z = oracle_mod.linear_attn(q, k, v)
+    elu1 = lambda x: torch.nn.functional.elu(torch.from_numpy(x).double()) + 1
+    Qp, Kp, V = elu1(q), elu1(k), torch.from_numpy(v).double()
+    P = torch.tril(Qp @ Kp.transpose(-1, -2))
+    O_ref = (P @ V) / P.sum(-1, keepdim=True)
+    np.testing.assert_allclose(o, O_ref.numpy(), rtol=1e-11)
+    np.testing.assert_allclose(S, (Kp.transpose(-1, -2) @ V).numpy(), rtol=1e-11)
+    np.testing.assert_allclose(z, Kp.sum(-2).numpy(), rtol=1e-11)
+
+
+def test_bf16_inputs_widen_exactly(oracle_mod):
+    """bfloat16 inputs give the same result as their exact float32 values."""
+    g = torch.Generator().manual_seed(11)
+    B, H, T, D = 1, 2, 29, 16
+    q, k, v = (torch.randn(B, H, T, D, generator=g).bfloat16() for _ in range(3))
+    beta = torch.rand(B, H, T, generator=g)
+    o1, S1 = oracle_mod.deltanet(q, k, v, beta)
+    o2, S2 = oracle_mod.deltanet(q.float(), k.float(), v.float(), beta)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
+    l1 = oracle_mod.linear_attn(q, k, v)
+    l2 = oracle_mod.linear_attn(q.float(), k.float(), v.float())
+    for a, b in zip(l1, l2):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_empty_sequence(oracle_mod):
+    """T = 0: no outputs, S_out = S0."""
+    rng = np.random.default_rng(12)
+    S0 = rng.standard_normal((1, 2, 4, 3))
+    z = np.zeros((1, 2, 0, 4), np.float32)
+    o, S = oracle_mod.deltanet(z, z, np.zeros((1, 2, 0, 3), np.float32),
+                               np.zeros((1, 2, 0), np.float32), S0=S0)
+    assert o.shape == (1, 2, 0, 3)
+    np.testing.assert_array_equal(S, S0)
+
+
+def test_planted_mistakes_fail_pins(oracle_mod):
+    """A wrong oracle must fail the pins above: plant a read from the undecayed state
+    and an output taken before the write, in a numpy copy of the recurrence, and check
+    the golden fixtures reject both."""
+    g = _golden("gated_scalar_worked.json")
+
+    def wrong(read_undecayed, out_before_write):
+        S, out = 0.0, []
+        for t in range(3):
+            a, b, v = g["alpha"][t], g["beta"][t], g["v"][t][0]
+            Sd = a * S
+            r = S if read_undecayed else Sd
+            if out_before_write:
+                out.append(Sd)
+            S = Sd + b * (v - r)
+            if not out_before_write:
+                out.append(S)
+        return out
+
+    ref = [x[0] for x in g["o"]]
+    assert wrong(False, False) == pytest.approx(ref)
+    assert wrong(True, False) != pytest.approx(ref)
+    assert wrong(False, True) != pytest.approx(ref)
