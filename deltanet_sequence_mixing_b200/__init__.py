@@ -1,0 +1,174 @@
+"""B200 (sm_100a) delta-rule sequence mixing: Python binding of the C ABI.
+
+The functions below carry the names of the C entry points in
+``include/deltanet.h`` and only marshal arguments: torch supplies device
+memory and the current stream, and every step of the computation runs in the
+library's CUDA kernels.  There is no CPU fallback.
+
+    o, S = deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C=64)
+    o    = deltanet_decode_step(q, k, v, beta, S, alpha=None)   # S updated in place
+    o, S, z = linear_attn_fwd(q, k, v, S0=None, z0=None, C=64)
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import DeltaNetError, check, lib, status_string  # noqa: F401
+
+__all__ = [
+    "deltanet_chunk_fwd", "deltanet_decode_step", "linear_attn_fwd", "workspace_for",
+    "deltanet_get_device_status", "deltanet_selftest_wait_timeout", "DeltaNetError",
+]
+
+_DT = {torch.float32: _lib.DN_F32, torch.bfloat16: _lib.DN_BF16}
+_workspaces: dict = {}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+def workspace_for(device, nbytes: int = 256) -> torch.Tensor:
+    """A cleared device workspace of at least ``nbytes``, cached per device."""
+    device = torch.device(device)
+    ws = _workspaces.get(device)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        check("deltanet_workspace_init",
+              lib().deltanet_workspace_init(_ptr(ws), ws.numel(), _stream(device)))
+        _workspaces[device] = ws
+    return ws
+
+
+def _ws_bytes(B, H, T, Dk, Dv, C, dt):
+    n = lib().deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt)
+    if n == 0:
+        raise DeltaNetError("deltanet_workspace_bytes", _lib.DN_ERR_UNSUPPORTED)
+    return n
+
+
+def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, S_out=None,
+                       workspace=None):
+    """Chunkwise DeltaNet forward.  q, k: (B,H,T,Dk); v: (B,H,T,Dv) (bf16 or f32);
+    beta, alpha: (B,H,T) f32; S0: (B,H,Dk,Dv) f32.  Returns (o, S_out)."""
+    _need(q, "q")
+    dev, dtype = q.device, q.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if alpha is not None:
+        _need(alpha, "alpha", torch.float32, dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, T, Dv, dtype=dtype, device=dev)
+    if S_out is None:
+        S_out = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    _need(o, "o", dtype, dev)
+    _need(S_out, "S_out", torch.float32, dev)
+    dt = _DT[dtype]
+    nb = _ws_bytes(B, H, T, Dk, Dv, C, dt)
+    ws = workspace if workspace is not None else workspace_for(dev, nb)
+    check("deltanet_chunk_fwd", lib().deltanet_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
+        B, H, T, Dk, Dv, C, dt, _ptr(ws), ws.numel(), _stream(dev)))
+    return o, S_out
+
+
+def linear_attn_fwd(q, k, v, S0=None, z0=None, C: int = 64, o=None, S_out=None, z_out=None,
+                    workspace=None):
+    """Chunkwise ELU+1 causal linear attention.  Returns (o, S_out, z_out)."""
+    _need(q, "q")
+    dev, dtype = q.device, q.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, dtype, dev)
+    for t, n in ((S0, "S0"), (z0, "z0")):
+        if t is not None:
+            _need(t, n, torch.float32, dev)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, T, Dv, dtype=dtype, device=dev)
+    if S_out is None:
+        S_out = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    if z_out is None:
+        z_out = torch.empty(B, H, Dk, dtype=torch.float32, device=dev)
+    dt = _DT[dtype]
+    nb = _ws_bytes(B, H, T, Dk, Dv, C, dt)
+    ws = workspace if workspace is not None else workspace_for(dev, nb)
+    check("linear_attn_fwd", lib().linear_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(S0), _ptr(z0), _ptr(o), _ptr(S_out), _ptr(z_out),
+        B, H, T, Dk, Dv, C, dt, _ptr(ws), ws.numel(), _stream(dev)))
+    return o, S_out, z_out
+
+
+def deltanet_decode_step(q, k, v, beta, S, alpha=None, o=None):
+    """One decode step.  q, k: (B,H,Dk); v: (B,H,Dv); beta, alpha: (B,H) f32;
+    S: (B,H,Dk,Dv) f32, updated in place.  Returns o (B,H,Dv)."""
+    _need(q, "q")
+    dev, dtype = q.device, q.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if alpha is not None:
+        _need(alpha, "alpha", torch.float32, dev)
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, Dv, dtype=dtype, device=dev)
+    check("deltanet_decode_step", lib().deltanet_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S), _ptr(o),
+        B, H, Dk, Dv, _DT[dtype], _stream(dev)))
+    return o
+
+
+def deltanet_get_device_status(device=None, workspace=None) -> int:
+    """Synchronise and return the sticky device status of ``workspace`` (or of the
+    cached workspace of ``device``)."""
+    device = torch.device(device if device is not None else "cuda")
+    ws = workspace if workspace is not None else workspace_for(device)
+    return lib().deltanet_get_device_status(_ptr(ws), _stream(device))
+
+
+def deltanet_selftest_wait_timeout(wait_ns: int, workspace, device=None) -> int:
+    """Launch the bounded-wait self test on ``workspace``; returns the launch status."""
+    device = torch.device(device if device is not None else workspace.device)
+    return lib().deltanet_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(wait_ns),
+                                                _stream(device))
+
+
+def reset_device_status(device=None, workspace=None) -> None:
+    device = torch.device(device if device is not None else "cuda")
+    ws = workspace if workspace is not None else workspace_for(device)
+    check("deltanet_workspace_init",
+          lib().deltanet_workspace_init(_ptr(ws), ws.numel(), _stream(device)))

@@ -1,0 +1,309 @@
+// CUDA-core chunked kernel: the chunkwise delta rule (plain and gated) and the
+// chunkwise ELU+1 linear attention, all arithmetic in float32.
+//
+// This is the float32 path of deltanet_chunk_fwd / linear_attn_fwd.  One CTA
+// owns one (b, h) sequence and a 64-column slice of Dv (the delta rule is
+// separable over the columns of v: column j of the deltas depends only on
+// column j of v and of S), keeps its Dk x 64 slice of the state in shared
+// memory, and walks the chunks in order.
+//
+// Per chunk of n <= C rows (ragged tail zero-filled with beta = 0, which is an
+// exact no-op), following the derived WY form of the Householder
+// reparameterisation ("GPT-2 から Kimi K3 まで", news.ainew.jp, section "DeltaNet
+// (Parallelizing linear transformers with delta rule)"):
+//   Gamma[r][s] = alpha_{s+1} ... alpha_r (s <= r),  gamma_r = alpha_0 ... alpha_r
+//   A = strict_lower(diag(beta) (K K^T * Gamma)),    T = (I + A)^-1
+//   X = V - diag(gamma) K S,   U = T diag(beta) X
+//   O = diag(gamma) Q S + (tril(Q K^T) * Gamma) U
+//   S = gamma_{n-1} S + (diag(Gamma[n-1][.]) K)^T U
+// and, for linear attention, the additive chunk loop of the same section on the
+// ELU+1 feature maps of section "Linear attention", with the normaliser z
+// carried like S:  O = (Q'S + tril(Q'K'^T) V) / (Q'z + tril(Q'K'^T) 1).
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+
+namespace dn {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename TI>
+__device__ __forceinline__ float load_in(const TI* p, size_t i);
+template <>
+__device__ __forceinline__ float load_in<float>(const float* p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float load_in<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+template <typename TI>
+__device__ __forceinline__ void store_out(TI* p, size_t i, float x);
+template <>
+__device__ __forceinline__ void store_out<float>(float* p, size_t i, float x) { p[i] = x; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, size_t i, float x) {
+  p[i] = __float2bfloat16_rn(x);
+}
+
+// ELU(x) + 1: x + 1 for x > 0, and e^x (= (e^x - 1) + 1) otherwise.
+__device__ __forceinline__ float elu_plus_one(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+template <int DK, int DVS, int C, bool GATED>
+struct SimtSmem {
+  static constexpr int KP = DK + 1, VP = DVS + 1, CP = C + 1;
+  static constexpr int kFloats = 2 * C * KP      // Q, K
+                                 + 2 * C * VP    // V (then X), U
+                                 + DK * VP       // S slice
+                                 + 2 * C * CP    // T, A / P
+                                 + (GATED ? C * CP : 0)  // Gamma
+                                 + 3 * C + DK + C;       // beta, gamma, alpha, z, den
+  static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <typename TI, bool LINEAR, bool GATED, int DK, int DVS, int C>
+__global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem p) {
+  using L = SimtSmem<DK, DVS, C, GATED>;
+  constexpr int KP = L::KP, VP = L::VP, CP = L::CP;
+  extern __shared__ float sm[];
+  float* Qs = sm;
+  float* Ks = Qs + C * KP;
+  float* Vs = Ks + C * KP;
+  float* Us = Vs + C * VP;
+  float* Ss = Us + C * VP;
+  float* Ts = Ss + DK * VP;
+  float* Ps = Ts + C * CP;
+  float* Gm = Ps + C * CP;  // only meaningful when GATED
+  float* bs = Gm + (GATED ? C * CP : 0);
+  float* gs = bs + C;
+  float* as = gs + C;
+  float* zs = as + C;
+  float* dens = zs + DK;
+
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x;
+  const int j0 = blockIdx.y * DVS;
+  const int T = p.T, Dv = p.Dv;
+  const TI* q = static_cast<const TI*>(p.q);
+  const TI* k = static_cast<const TI*>(p.k);
+  const TI* v = static_cast<const TI*>(p.v);
+  TI* o = static_cast<TI*>(p.o);
+  const size_t qk_base = (size_t)bh * T * DK;
+  const size_t v_base = (size_t)bh * T * Dv;
+  const size_t s_base = (size_t)bh * DK * Dv;
+
+  for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+    const int i = idx / DVS, j = idx % DVS;
+    Ss[i * VP + j] = p.S0 ? p.S0[s_base + (size_t)i * Dv + j0 + j] : 0.f;
+  }
+  if (LINEAR)
+    for (int i = tid; i < DK; i += kThreads) zs[i] = p.z0 ? p.z0[(size_t)bh * DK + i] : 0.f;
+
+  for (int c0 = 0; c0 < T; c0 += C) {
+    const int n = min(C, T - c0);
+    __syncthreads();  // previous chunk finished with every buffer
+    // ---- stage the chunk (rows >= n are zero; beta 0, alpha 1) ----
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      float qv = 0.f, kv = 0.f;
+      if (r < n) {
+        qv = load_in(q, qk_base + (size_t)(c0 + r) * DK + i);
+        kv = load_in(k, qk_base + (size_t)(c0 + r) * DK + i);
+        if (LINEAR) {
+          qv = elu_plus_one(qv);
+          kv = elu_plus_one(kv);
+        }
+      }
+      Qs[r * KP + i] = qv;
+      Ks[r * KP + i] = kv;
+    }
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      Vs[r * VP + j] = r < n ? load_in(v, v_base + (size_t)(c0 + r) * Dv + j0 + j) : 0.f;
+    }
+    if (!LINEAR)
+      for (int r = tid; r < C; r += kThreads) {
+        bs[r] = r < n ? p.beta[(size_t)bh * T + c0 + r] : 0.f;
+        as[r] = (GATED && r < n) ? p.alpha[(size_t)bh * T + c0 + r] : 1.f;
+      }
+    __syncthreads();
+
+    if (LINEAR) {
+      // P = tril(Q' K'^T)
+      for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, s = idx % C;
+        float acc = 0.f;
+        if (s <= r)
+          for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ks[s * KP + i];
+        Ps[r * CP + s] = acc;
+      }
+      __syncthreads();
+      for (int r = tid; r < C; r += kThreads) {
+        float acc = 0.f;
+        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * zs[i];
+        for (int s = 0; s <= r; ++s) acc += Ps[r * CP + s];
+        dens[r] = acc;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        const int r = idx / DVS, j = idx % DVS;
+        if (r >= n) continue;
+        float acc = 0.f;
+        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ss[i * VP + j];
+        for (int s = 0; s <= r; ++s) acc += Ps[r * CP + s] * Vs[s * VP + j];
+        store_out(o, v_base + (size_t)(c0 + r) * Dv + j0 + j, acc / dens[r]);
+      }
+      __syncthreads();
+      for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+        const int i = idx / DVS, j = idx % DVS;
+        float acc = Ss[i * VP + j];
+        for (int s = 0; s < n; ++s) acc += Ks[s * KP + i] * Vs[s * VP + j];
+        Ss[i * VP + j] = acc;
+      }
+      for (int i = tid; i < DK; i += kThreads) {
+        float acc = zs[i];
+        for (int s = 0; s < n; ++s) acc += Ks[s * KP + i];
+        zs[i] = acc;
+      }
+      continue;
+    }
+
+    // ---- decay tables: Gamma[r][s] = alpha_{s+1} ... alpha_r, gamma_r ----
+    if (GATED) {
+      for (int r = tid; r < C; r += kThreads) {
+        float prod = 1.f;
+        Gm[r * CP + r] = 1.f;
+        for (int s = r - 1; s >= 0; --s) {
+          prod *= as[s + 1];
+          Gm[r * CP + s] = prod;
+        }
+        for (int s = r + 1; s < C; ++s) Gm[r * CP + s] = 0.f;
+        gs[r] = prod * as[0];
+      }
+      __syncthreads();
+    }
+    // ---- A = strict_lower(diag(beta) (K K^T * Gamma)) ----
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s < r) {
+        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
+        acc *= bs[r];
+        if (GATED) acc *= Gm[r * CP + s];
+      }
+      Ps[r * CP + s] = acc;
+    }
+    __syncthreads();
+    // ---- T = (I + A)^-1 by forward substitution, one column per thread ----
+    for (int j = tid; j < C; j += kThreads) {
+      for (int i = 0; i < C; ++i) {
+        float t;
+        if (i < j) {
+          t = 0.f;
+        } else if (i == j) {
+          t = 1.f;
+        } else {
+          float acc = 0.f;
+          for (int m = j; m < i; ++m) acc += Ps[i * CP + m] * Ts[m * CP + j];
+          t = -acc;
+        }
+        Ts[i * CP + j] = t;
+      }
+    }
+    // ---- X = V - diag(gamma) K S (in place in Vs) ----
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ss[i * VP + j];
+      if (GATED) acc *= gs[r];
+      Vs[r * VP + j] -= acc;
+    }
+    __syncthreads();
+    // ---- U = T diag(beta) X;  P = tril(Q K^T) * Gamma ----
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int s = 0; s <= r; ++s) acc += Ts[r * CP + s] * bs[s] * Vs[s * VP + j];
+      Us[r * VP + j] = acc;
+    }
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s <= r) {
+        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ks[s * KP + i];
+        if (GATED) acc *= Gm[r * CP + s];
+      }
+      Ps[r * CP + s] = acc;
+    }
+    __syncthreads();
+    // ---- O = diag(gamma) Q S + P U ----
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      if (r >= n) continue;
+      float inter = 0.f;
+      for (int i = 0; i < DK; ++i) inter += Qs[r * KP + i] * Ss[i * VP + j];
+      if (GATED) inter *= gs[r];
+      float intra = 0.f;
+      for (int s = 0; s <= r; ++s) intra += Ps[r * CP + s] * Us[s * VP + j];
+      store_out(o, v_base + (size_t)(c0 + r) * Dv + j0 + j, inter + intra);
+    }
+    __syncthreads();
+    // ---- S = gamma_{n-1} S + (diag(Gamma[n-1][.]) K)^T U ----
+    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+      const int i = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int s = 0; s < n; ++s) {
+        float kk = Ks[s * KP + i];
+        if (GATED) kk *= Gm[(n - 1) * CP + s];
+        acc += kk * Us[s * VP + j];
+      }
+      const float carry = GATED ? gs[n - 1] : 1.f;
+      Ss[i * VP + j] = carry * Ss[i * VP + j] + acc;
+    }
+  }
+  __syncthreads();
+  if (p.S_out)
+    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+      const int i = idx / DVS, j = idx % DVS;
+      p.S_out[s_base + (size_t)i * Dv + j0 + j] = Ss[i * VP + j];
+    }
+  if (LINEAR && p.z_out && blockIdx.y == 0)
+    for (int i = tid; i < DK; i += kThreads) p.z_out[(size_t)bh * DK + i] = zs[i];
+}
+
+template <typename TI, bool LINEAR, bool GATED, int DK>
+cudaError_t launch_one(const ChunkProblem& p, cudaStream_t st) {
+  constexpr int DVS = 64, C = 64;
+  using L = SimtSmem<DK, DVS, C, GATED>;
+  auto kern = chunk_simt_kernel<TI, LINEAR, GATED, DK, DVS, C>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)L::kBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(p.B * p.H), (unsigned)(p.Dv / DVS));
+  kern<<<grid, kThreads, L::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t dispatch_mode(const ChunkProblem& p, cudaStream_t st) {
+  const bool lin = p.mode == Mode::Linear;
+  const bool gated = !lin && p.alpha != nullptr;
+  if (p.Dk == 64) {
+    if (lin) return launch_one<TI, true, false, 64>(p, st);
+    return gated ? launch_one<TI, false, true, 64>(p, st) : launch_one<TI, false, false, 64>(p, st);
+  }
+  if (lin) return launch_one<TI, true, false, 128>(p, st);
+  return gated ? launch_one<TI, false, true, 128>(p, st) : launch_one<TI, false, false, 128>(p, st);
+}
+
+}  // namespace
+
+bool chunk_simt_supported(int Dk, int Dv, int C) {
+  return (Dk == 64 || Dk == 128) && (Dv == 64 || Dv == 128) && C == 64;
+}
+
+cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t st) {
+  if (!chunk_simt_supported(p.Dk, p.Dv, p.C)) return cudaErrorNotSupported;
+  return p.bf16 ? dispatch_mode<__nv_bfloat16>(p, st) : dispatch_mode<float>(p, st);
+}
+
+}  // namespace dn

@@ -1,0 +1,592 @@
+// tcgen05 chunked DeltaNet forward (bf16 operands, float32 accumulation and
+// state), the bf16 path of deltanet_chunk_fwd.
+//
+// The method: the delta rule o_t = q_t S_t, S_t = alpha_t S_{t-1} + k_t^T u_t,
+// u_t = beta_t (v_t - alpha_t k_t S_{t-1}) ("GPT-2 から Kimi K3 まで",
+// news.ainew.jp, section "DeltaNet (Parallelizing linear transformers with
+// delta rule)", per-token loop; gate from the Gated DeltaNet paragraph of "How a
+// Baseten Engineer Traced 7 Years of Attention Mechanism Evolution"), evaluated
+// chunk by chunk (C = 64) with the Householder / WY reparameterisation so that
+// all deltas of a chunk come out of dense products.  For a chunk entered with
+// state S (g_r = sum_{j<=r} log alpha_j, Gamma_rs = exp(g_r - g_s) for s <= r):
+//   G  = [K;Q] K^T                    (KK^T and QK^T in one M = 128 MMA)
+//   A  = strict_lower(diag(beta) KK^T * Gamma),  T = (I + A)^-1   (fp32, CUDA cores)
+//   Tb = T diag(beta),  Tbg = Tb diag(gamma)
+//   W  = Tbg K,  Uh = Tb V            (S-independent)
+//   [QS; WS] = [Q;W] S                (one M = 128 MMA against the bf16 state)
+//   U  = Uh - WS                      (the chunk's deltas)
+//   O  = diag(gamma) QS + (tril(QK^T) * Gamma) U
+//   S <- gamma_last S + K^T (diag(Gamma_last,.) U)
+//
+// Hardware mapping (sm_100a): one CTA per (b, h, 64-column slice of Dv).
+// Warps 0-3 own TMEM lanes 0-127 and do the epilogues; warp 4 streams q, k, v
+// chunks with TMA (128-byte swizzle, 3-D maps so a ragged tail reads zeros)
+// into a two-stage ring; thread 0 issues the tcgen05 MMAs.  All operands live in
+// shared memory in the 128-byte-swizzled canonical layout, accumulators in
+// TMEM, the running state in float32 registers (one state row per thread).
+// Every wait is bounded; a wait that runs out sets the workspace status word
+// and the CTA winds down cleanly (outstanding copies drained, TMEM freed).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dn {
+namespace {
+
+constexpr int kC = 64;              // chunk rows
+constexpr int kDVS = 64;            // state columns per CTA
+constexpr uint32_t kTile = 8192;    // 64 rows x 128 bytes
+constexpr int kCompute = 128;       // warps 0-3
+constexpr int kThreads = kCompute + 32;
+constexpr int kApad = 68;           // float row stride of the A / T scratch
+
+// TMEM column map (512 columns allocated).
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_UH = 192, TM_QW = 256, TM_PU = 320, TM_DS = 384;
+
+template <int DK>
+struct TcLayout {
+  static constexpr int KB = DK / 64;                       // 64-column blocks of Dk
+  static constexpr uint32_t KB_STRIDE = 3 * kTile;         // [K | Q | W] per block
+  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
+  static constexpr uint32_t V_OFF = KB * KB_STRIDE;
+  static constexpr uint32_t STAGE = KB * KB_STRIDE + kTile;
+  static constexpr uint32_t PT_OFF = 2 * STAGE;            // [P | Tb | Tbg]
+  static constexpr uint32_t S_OFF = PT_OFF + 3 * kTile;    // bf16 state, DK rows x 128 B
+  static constexpr uint32_t U_OFF = S_OFF + DK * 128;
+  static constexpr uint32_t UT_OFF = U_OFF + kTile;        // decay-weighted U (gated)
+  static constexpr uint32_t AM_OFF = UT_OFF + kTile;       // fp32 A (64 x kApad)
+  static constexpr uint32_t TM_OFF = AM_OFF + 64 * kApad * 4;
+  static constexpr uint32_t VEC_OFF = TM_OFF + 64 * kApad * 4;  // beta[64], g[64]
+  static constexpr uint32_t BAR_OFF = VEC_OFF + 2 * 64 * 4;
+  static constexpr uint32_t BYTES = BAR_OFF + 64;
+  static constexpr uint32_t ALLOC = BYTES + 1024;          // 1024-byte alignment slack
+  static_assert(BYTES + 1024 <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ bool bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.and.pred po, 1, 128, pi;"
+      " selp.u32 %0, 1, 0, po; }"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_compute() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Write 8 consecutive floats as one 16-byte bf16 chunk.
+__device__ __forceinline__ void st_chunk(uint8_t* dst, const float* x) {
+  uint4 u;
+  u.x = pack_bf16(x[0], x[1]);
+  u.y = pack_bf16(x[2], x[3]);
+  u.z = pack_bf16(x[4], x[5]);
+  u.w = pack_bf16(x[6], x[7]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return sw128_desc(addr, 16, 1024); }
+__device__ __forceinline__ uint64_t mndesc(uint32_t addr, uint32_t lbo) {
+  return sw128_desc(addr, lbo, 1024);
+}
+
+template <int DK, bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const ChunkProblem p) {
+  using L = TcLayout<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int j0 = blockIdx.y * kDVS;
+  const int T = p.T, Dv = p.Dv;
+  const int nchunks = (T + kC - 1) / kC;
+
+  const uint32_t bar_full0 = sb + L::BAR_OFF, bar_empty0 = sb + L::BAR_OFF + 16;
+  const uint32_t bar_mma = sb + L::BAR_OFF + 32, bar_fin = sb + L::BAR_OFF + 40;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR_OFF + 48);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF + 52);
+  float* betas = reinterpret_cast<float*>(sm + L::VEC_OFF);
+  float* gs = betas + 64;
+  float* Am = reinterpret_cast<float*>(sm + L::AM_OFF);
+  float* Tm = reinterpret_cast<float*>(sm + L::TM_OFF);
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_full0 + 8 * s, 1);
+      mbar_init(bar_empty0 + 8 * s, 1);
+    }
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1, use = c >> 1;
+        if (use > 0 && !mbar_wait(bar_empty0 + 8 * s, (use - 1) & 1, wc)) break;
+        const uint32_t st = sb + s * L::STAGE;
+        const uint32_t full = bar_full0 + 8 * s;
+        mbar_expect_tx(full, (2 * L::KB + 1) * kTile);
+#pragma unroll
+        for (int kb = 0; kb < L::KB; ++kb) {
+          tma_load_3d(st + kb * L::KB_STRIDE + L::K_OFF, &tmK, full, kb * 64, c * kC, bh);
+          tma_load_3d(st + kb * L::KB_STRIDE + L::Q_OFF, &tmQ, full, kb * 64, c * kC, bh);
+        }
+        tma_load_3d(st + L::V_OFF, &tmV, full, j0, c * kC, bh);
+        issued = c + 1;
+      }
+      // Never leave with copies in flight: wait for the last loads to land.
+      int zero = 0;
+      const WaitCtl drain{&zero, p.status, kWaitLimitNs};
+      for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
+        (void)mbar_wait(bar_full0 + 8 * (c & 1), (c >> 1) & 1, drain);
+    }
+  } else {
+    // ------------------------------------------------------------- compute --
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const size_t s_base = (size_t)bh * DK * Dv;
+    const int row = tid & 63;  // chunk row handled in row-parallel epilogues
+    float sreg[kDVS];
+    if (tid < DK) {
+      const float* src = p.S0 ? p.S0 + s_base + (size_t)tid * Dv + j0 : nullptr;
+#pragma unroll
+      for (int j = 0; j < kDVS; j += 4) {
+        float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
+      }
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) st_chunk(sm + L::S_OFF + sw128_off(tid, c16), sreg + 8 * c16);
+    }
+    fence_proxy_async_smem();
+    bar_compute();
+
+    uint32_t mma_count = 0;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int s = c & 1, use = c >> 1;
+      const int c0 = c * kC, n = min(kC, T - c0);
+      const uint32_t st = sb + s * L::STAGE;
+      uint8_t* stp = sm + s * L::STAGE;
+
+      // write strengths and log-decay prefix g of this chunk (rows >= n: beta 0, alpha 1)
+      if (tid < 64) {
+        const size_t tb = (size_t)bh * T + c0;
+        betas[tid] = tid < n ? p.beta[tb + tid] : 0.f;
+        if (GATED) {
+          float la = tid < n ? fmaxf(__logf(p.alpha[tb + tid]), -87.f) : 0.f;
+          float x = la;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+          }
+          if (warp == 1) {  // add the total of rows 0..31
+            float l0 = lane < n ? fmaxf(__logf(p.alpha[tb + lane]), -87.f) : 0.f;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            x += l0;
+          }
+          gs[tid] = x;
+        }
+      }
+      ok = bar_and(mbar_wait(bar_full0 + 8 * s, use & 1, wc));
+      if (!ok) break;
+
+      // ---- MMA 1: G = [K;Q] K^T  (lanes 0-63: K K^T, lanes 64-127: Q K^T) ----
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::K_OFF + (ks & 3) * 32;
+          mma_bf16_ss(tmem + TM_G, kdesc(a), kdesc(a), id, ks > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
+      ++mma_count;
+      if (!ok) break;
+      tc_fence_after();
+
+      // ---- E1: A rows (threads 0-63) and P rows (threads 64-127) ----
+      {
+        uint32_t g[64];
+        tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
+        tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+        tmem_wait_ld();
+        const float gr = GATED ? gs[row] : 0.f;
+        if (tid < 64) {
+          const float br = betas[row];
+          float* arow = Am + row * kApad;
+#pragma unroll
+          for (int s4 = 0; s4 < 64; s4 += 4) {
+            float a4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int sc = s4 + e;
+              float val = br * __uint_as_float(g[sc]);
+              if (GATED) val *= __expf(gr - gs[sc]);
+              a4[e] = sc < row ? val : 0.f;
+            }
+            *reinterpret_cast<float4*>(arow + s4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+          }
+        } else {
+          uint8_t* ptile = sm + L::PT_OFF;
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int sc = c16 * 8 + e;
+              float val = __uint_as_float(g[sc]);
+              if (GATED) val *= __expf(gr - gs[sc]);
+              x[e] = sc <= row ? val : 0.f;
+            }
+            st_chunk(ptile + sw128_off(row, c16), x);
+          }
+        }
+      }
+      bar_compute();
+
+      // ---- T = (I + A)^-1: two 32x32 diagonal inverses, then the off-diagonal block ----
+      if (tid < 64) {
+        const int o = (tid >> 5) * 32, j = tid & 31;
+        float col[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) col[k] = (k == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 1; i < 32; ++i) {
+          const float* ar = Am + (o + i) * kApad + o;
+          float acc = 0.f;
+#pragma unroll
+          for (int m4 = 0; m4 < i; m4 += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(ar + m4);
+            acc = fmaf(a.x, col[m4], acc);
+            acc = fmaf(a.y, col[m4 + 1], acc);
+            acc = fmaf(a.z, col[m4 + 2], acc);
+            acc = fmaf(a.w, col[m4 + 3], acc);
+          }
+          if (i > j) col[i] = -acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) Tm[(o + i) * kApad + o + j] = col[i];
+      }
+      bar_compute();
+      {  // Y = A21 T11 into the (unused) upper-right block of Tm
+        const int cy = tid & 31, r0 = (tid >> 5) * 8;
+        float acc[8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const float tk = Tm[k * kApad + cy];
+#pragma unroll
+          for (int rr = 0; rr < 8; ++rr) acc[rr] = fmaf(Am[(32 + r0 + rr) * kApad + k], tk, acc[rr]);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) Tm[(r0 + rr) * kApad + 32 + cy] = acc[rr];
+      }
+      bar_compute();
+      {  // T21 = -T22 Y
+        const int cy = tid & 31, r0 = (tid >> 5) * 8;
+        float acc[8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+          const float yk = Tm[k * kApad + 32 + cy];
+#pragma unroll
+          for (int rr = 0; rr < 8; ++rr) {
+            const float t22 = (k <= r0 + rr) ? Tm[(32 + r0 + rr) * kApad + 32 + k] : 0.f;
+            acc[rr] = fmaf(t22, yk, acc[rr]);
+          }
+        }
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) Tm[(32 + r0 + rr) * kApad + cy] = -acc[rr];
+      }
+      bar_compute();
+      {  // Tb = T diag(beta), Tbg = Tb diag(gamma): row `row`, columns [32h, 32h + 32)
+        const int h = tid >> 6;
+        uint8_t* tb_tile = sm + L::PT_OFF + kTile;
+        uint8_t* tbg_tile = sm + L::PT_OFF + 2 * kTile;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c16 = h * 4 + cc;
+          float x[8], y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int sc = c16 * 8 + e;
+            const float t = sc <= row ? Tm[row * kApad + sc] : 0.f;
+            x[e] = t * betas[sc];
+            if (GATED) y[e] = x[e] * __expf(gs[sc]);
+          }
+          st_chunk(tb_tile + sw128_off(row, c16), x);
+          if (GATED) st_chunk(tbg_tile + sw128_off(row, c16), y);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar_compute();
+
+      // ---- MMA 2: W = Tbg K (lanes 64-127), Uh = Tb V (lanes 64-127) ----
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t pt = sb + L::PT_OFF;
+        const uint32_t aw = GATED ? pt + kTile : pt;
+        constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
+        constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ss(tmem + TM_W, kdesc(aw + ks * 32),
+                      mndesc(st + L::K_OFF + ks * 2048, L::KB_STRIDE), idw, ks > 0);
+          mma_bf16_ss(tmem + TM_UH, kdesc(pt + ks * 32), mndesc(st + L::V_OFF + ks * 2048, kTile),
+                      idu, ks > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
+      ++mma_count;
+      if (!ok) break;
+      tc_fence_after();
+
+      // ---- E2: W rows -> bf16 into the stage (next to Q) ----
+      if (tid >= 64) {
+#pragma unroll
+        for (int q = 0; q < DK / 32; ++q) {
+          uint32_t w[32];
+          tmem_ld32(tmem + lane_base + TM_W + q * 32, w);
+          tmem_wait_ld();
+          uint8_t* wt = stp + (q >> 1) * L::KB_STRIDE + L::W_OFF;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(w[cc * 8 + e]);
+            st_chunk(wt + sw128_off(row, (q & 1) * 4 + cc), x);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar_compute();
+
+      // ---- MMA 3: [QS; WS] = [Q; W] S ----
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+          mma_bf16_ss(tmem + TM_QW, kdesc(a), mndesc(sb + L::S_OFF + ks * 2048, kTile), id, ks > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
+      ++mma_count;
+      if (!ok) break;
+      tc_fence_after();
+
+      // ---- E3: U = Uh - WS (rows on lanes 64-127) ----
+      if (tid >= 64) {
+        const float wl = GATED ? __expf(gs[n - 1] - gs[row]) : 1.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t ws[32], uh[32];
+          tmem_ld32(tmem + lane_base + TM_QW + q * 32, ws);
+          tmem_ld32(tmem + lane_base + TM_UH + q * 32, uh);
+          tmem_wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float x[8], y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              x[e] = __uint_as_float(uh[cc * 8 + e]) - __uint_as_float(ws[cc * 8 + e]);
+              y[e] = x[e] * wl;
+            }
+            st_chunk(sm + L::U_OFF + sw128_off(row, q * 4 + cc), x);
+            if (GATED) st_chunk(sm + L::UT_OFF + sw128_off(row, q * 4 + cc), y);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar_compute();
+
+      // ---- MMA 4: PU = [P; Tb] U (lanes 0-63), dS = K^T U~ (lanes 0-DK) ----
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t pt = sb + L::PT_OFF;
+        const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
+        constexpr uint32_t idp = idesc_bf16(128, 64, false, true);
+        constexpr uint32_t ids = idesc_bf16(128, 64, true, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ss(tmem + TM_PU, kdesc(pt + ks * 32), mndesc(sb + L::U_OFF + ks * 2048, kTile),
+                      idp, ks > 0);
+          mma_bf16_ss(tmem + TM_DS, mndesc(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                      mndesc(ut + ks * 2048, kTile), ids, ks > 0);
+        }
+        mma_commit(bar_mma);
+        mma_commit(bar_empty0 + 8 * s);  // the stage may be refilled once these are done
+      }
+      ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
+      ++mma_count;
+      if (!ok) break;
+      tc_fence_after();
+
+      // ---- E4: outputs (rows on lanes 0-63) and the state update ----
+      if (tid < 64) {
+        const float gam = GATED ? __expf(gs[row]) : 1.f;
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + row) * Dv + j0;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t qs[32], pu[32];
+          tmem_ld32(tmem + lane_base + TM_QW + q * 32, qs);
+          tmem_ld32(tmem + lane_base + TM_PU + q * 32, pu);
+          tmem_wait_ld();
+          if (row < n) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              float x[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                x[e] = fmaf(gam, __uint_as_float(qs[cc * 8 + e]), __uint_as_float(pu[cc * 8 + e]));
+              st_chunk(reinterpret_cast<uint8_t*>(orow + q * 32 + cc * 8), x);
+            }
+          }
+        }
+      }
+      if (tid < DK) {
+        const float carry = GATED ? __expf(gs[n - 1]) : 1.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t ds[32];
+          tmem_ld32(tmem + lane_base + TM_DS + q * 32, ds);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sreg[q * 32 + e] = fmaf(carry, sreg[q * 32 + e], __uint_as_float(ds[e]));
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) st_chunk(sm + L::S_OFF + sw128_off(tid, c16), sreg + 8 * c16);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar_compute();
+    }
+
+    if (p.S_out && tid < DK) {
+      float* dst = p.S_out + s_base + (size_t)tid * Dv + j0;
+#pragma unroll
+      for (int j = 0; j < kDVS; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
+    }
+    // Make sure no MMA is still running before TMEM is released.
+    if (tid == 0) {
+      tc_fence_after();
+      mma_commit(bar_fin);
+      int zero = 0;
+      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
+      (void)mbar_wait(bar_fin, 0, fin);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host ---
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over a (BH, T, D) bf16 tensor with a 64 x 64 box, 128-byte swizzle;
+// rows past T read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int D, int T, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, bool GATED>
+cudaError_t launch_t(const ChunkProblem& p, cudaStream_t st) {
+  using L = TcLayout<DK>;
+  CUtensorMap mq, mk, mv;
+  const int BH = p.B * p.H;
+  if (!make_map(&mq, p.q, DK, p.T, BH) || !make_map(&mk, p.k, DK, p.T, BH) ||
+      !make_map(&mv, p.v, p.Dv, p.T, BH))
+    return cudaErrorInvalidValue;
+  auto kern = chunk_tc_kernel<DK, GATED>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
+  kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_tc_supported(const ChunkProblem& p) {
+  return p.bf16 && p.mode == Mode::Delta && p.T > 0 && p.C == 64 &&
+         (p.Dk == 64 || p.Dk == 128) && (p.Dv == 64 || p.Dv == 128);
+}
+
+cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t st) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_t<128, true>(p, st) : launch_t<128, false>(p, st);
+  return gated ? launch_t<64, true>(p, st) : launch_t<64, false>(p, st);
+}
+
+}  // namespace dn

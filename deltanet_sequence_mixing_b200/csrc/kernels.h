@@ -1,0 +1,61 @@
+// Internal launcher declarations shared by the ABI layer and the kernel files.
+// Not part of the public interface (that is include/deltanet.h).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dn {
+
+// Bits of the device status word kept in the first bytes of the workspace.
+// Kernels only ever set bits; the host clears the word.
+constexpr unsigned int kStatusTimeoutBit = 1u;  // a bounded wait ran out
+
+enum class Mode : int { Delta = 0, Linear = 1 };
+
+// Problem description passed from the ABI layer to the launchers.  All pointers
+// are device pointers that the ABI layer has validated.
+struct ChunkProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;   // Delta only
+  const float* alpha;  // Delta only, nullable
+  const float* S0;     // nullable
+  const float* z0;     // Linear only, nullable
+  void* o;
+  float* S_out;        // nullable
+  float* z_out;        // Linear only, nullable
+  int B, H, T, Dk, Dv, C;
+  int bf16;            // 1: q/k/v/o are bfloat16, 0: float32
+  Mode mode;
+  unsigned int* status;  // device status word (workspace)
+};
+
+// CUDA-core (float32 arithmetic) chunked kernel: both modes, both input types.
+// Returns cudaErrorNotSupported for shapes it does not instantiate.
+cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t st);
+bool chunk_simt_supported(int Dk, int Dv, int C);
+
+// tcgen05 (bf16 operands, float32 accumulate) chunked kernels.
+cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t st);
+bool chunk_tc_supported(const ChunkProblem& p);
+
+// Decode step (in-place state update).
+struct DecodeProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  const float* alpha;  // nullable
+  float* S;
+  void* o;
+  int B, H, Dk, Dv;
+  int bf16;
+};
+cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t st);
+
+// Bounded-wait self test.
+cudaError_t launch_wait_selftest(unsigned int* status, long long wait_ns, cudaStream_t st);
+
+}  // namespace dn

@@ -1,0 +1,178 @@
+/*
+ * deltanet.h - C ABI of the B200 (sm_100a) delta-rule sequence-mixing library.
+ *
+ * The library computes the innermost layer of a DeltaNet / linear-attention
+ * block: the sequence mixing over a per-head Dk x Dv state S, with the q/k/v
+ * projections, feature maps of the DeltaNet layer (silu + L2 normalise) and
+ * the output projection left to the caller.  Row-vector convention:
+ * o_t = q_t S_t, S is Dk x Dv.
+ *
+ * Sources (web pages on the subject):
+ *   [P1] "How a Baseten Engineer Traced 7 Years of Attention Mechanism
+ *        Evolution -- From GPT-2 to Kimi K3, in Runable PyTorch" (wpnews.pro)
+ *   [P3] "GPT-2 から Kimi K3 まで、AI モデルの進化を解説" (news.ainew.jp)
+ *
+ * Conventions common to every call
+ *   - All tensors are row-major and contiguous.  q, k: (B,H,T,Dk);
+ *     v, o: (B,H,T,Dv); beta, alpha: (B,H,T) float32; S0, S_out, S:
+ *     (B,H,Dk,Dv) float32 (Dv contiguous); z0, z_out: (B,H,Dk) float32.
+ *   - q, k, v and o share one element type, dn_dtype.  State, normaliser,
+ *     beta and alpha are always float32.
+ *   - Every pointer except `workspace` of the host-side queries is a DEVICE
+ *     pointer on the current CUDA device.  The caller owns and allocates every
+ *     buffer, including the workspace; the library allocates nothing per call.
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  DN_OK means "validated and launched".
+ *   - Argument validation happens on the host, before any CUDA call; a
+ *     rejected call launches nothing and touches no buffer.
+ *   - No query scaling (no 1/sqrt(d)), no normalisation of k: the pages' read
+ *     "o = q @ S" has no denominator ([P3] "DeltaNet (Fast weight
+ *     programmers)").  NaN/Inf inputs propagate as through the recurrence.
+ *   - Device-side waits are bounded: a wait that runs out sets a sticky
+ *     status word in the workspace (read it with deltanet_get_device_status)
+ *     and the kernel returns without trapping.
+ */
+#ifndef DELTANET_H_
+#define DELTANET_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    DN_OK = 0,
+    DN_ERR_INVALID_ARG = -1,    /* null pointer, negative size, bad aliasing     */
+    DN_ERR_UNSUPPORTED = -2,    /* shape / chunk size / dtype not implemented    */
+    DN_ERR_ALIGNMENT = -3,      /* q, k, v, o not 16-byte aligned (TMA rule)     */
+    DN_ERR_CUDA = -4,           /* a CUDA runtime / driver call failed           */
+    DN_ERR_DEVICE_TIMEOUT = -5, /* a bounded device wait ran out (status word)   */
+    DN_ERR_WORKSPACE = -6       /* workspace missing or smaller than required    */
+} dn_status;
+
+/* Element type of q, k, v and o. */
+typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
+
+/*
+ * Bytes of device workspace the chunked calls need for this problem (at least
+ * 256: the sticky device status word and its padding).  The workspace must be
+ * cleared once with deltanet_workspace_init before its first use; it may then
+ * be reused by any number of calls on the same stream.  Returns 0 for sizes
+ * the library rejects.
+ */
+size_t deltanet_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt);
+
+/* Clear the device status word of `workspace` (asynchronous memset). */
+int deltanet_workspace_init(void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
+ * Chunkwise-parallel DeltaNet forward (prefill / training forward).
+ *
+ * Computes, for every (b,h) sequence and t = 0..T-1, the delta rule of [P3]
+ * "DeltaNet (Parallelizing linear transformers with delta rule)" (the direct
+ * per-token loop), gated as in [P1]'s Gated DeltaNet paragraph ("decay first,
+ * then precise write"):
+ *     S'   = alpha_t S_{t-1}                 (alpha_t = 1 when alpha == NULL)
+ *     u_t  = beta_t (v_t - k_t S')
+ *     S_t  = S' + k_t^T u_t
+ *     o_t  = q_t S_t                         (state after the write)
+ * It evaluates this in chunks of C tokens with the Householder / WY
+ * reparameterisation ([P3] same section; [P1] "split the sequence into chunks
+ * of size C ... a Householder transformation reparameterizes the delta
+ * updates"): per chunk, T = (I + strict_lower(diag(beta) (K K^T * Gamma)))^-1,
+ * U = T diag(beta) (V - diag(gamma) K S), O = diag(gamma) Q S +
+ * (tril(Q K^T) * Gamma) U, S <- gamma_C S + (diag(gamma_C/gamma) K)^T U.
+ *
+ *   q, k       (B,H,T,Dk), v (B,H,T,Dv), element type dt, 16-byte aligned.
+ *   beta       (B,H,T) float32 write strengths.
+ *   alpha      (B,H,T) float32 decays in [0,1], or NULL for plain DeltaNet.
+ *   S0         (B,H,Dk,Dv) float32 initial state, or NULL for zero.
+ *   o          (B,H,T,Dv) output, element type dt, 16-byte aligned; must not
+ *              overlap any input.
+ *   S_out      (B,H,Dk,Dv) float32 final state, or NULL.  May equal S0
+ *              (in-place carry); any other overlap is rejected.
+ *   Dk, Dv     64 or 128.   C: 64 (bf16 and f32) or 128 (bf16).
+ *   T >= 0; T need not be a multiple of C (the ragged tail is handled
+ *   exactly).  T == 0 copies S0 (or zeros) to S_out; q, k, v, beta, alpha
+ *   and o may then be NULL.
+ *   workspace  device buffer of deltanet_workspace_bytes(...) bytes.
+ * bf16 runs on tcgen05 tensor cores with float32 state and accumulation;
+ * f32 runs on CUDA cores in float32 throughout.
+ */
+int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
+                       const float *beta, const float *alpha, const float *S0,
+                       void *o, float *S_out,
+                       int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                       void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
+ * One recurrent decode step for a batch of B x H states, updated in place.
+ *
+ * The case t = 1 of the recurrence above ([P3] "DeltaNet (Fast weight
+ * programmers)" with a cached state; [P1] Gated DeltaNet):
+ *     r = k S, p = q S (one pass over S)
+ *     u = beta (v - alpha r);   o = alpha p + (q . k) u
+ *     S <- alpha S + k^T u
+ * Each state is read once and written once.
+ *   q, k (B,H,Dk); v, o (B,H,Dv): element type dt, 16-byte aligned.
+ *   beta (B,H) float32; alpha (B,H) float32 or NULL.
+ *   S    (B,H,Dk,Dv) float32, updated in place; 16-byte aligned.
+ *   Dk, Dv in {64, 128}.  No workspace.
+ */
+int deltanet_decode_step(const void *q, const void *k, const void *v,
+                         const float *beta, const float *alpha, float *S, void *o,
+                         int B, int H, int Dk, int Dv, dn_dtype dt, void *cuda_stream);
+
+/*
+ * Causal linear attention with the ELU+1 feature map (the additive special
+ * case: the delta rule with its read term dropped).
+ *
+ * [P3] "Linear attention" (cached forward) and [P1] (Q' = ELU(Q)+1,
+ * K' = ELU(K)+1): with q' = ELU(q)+1, k' = ELU(k)+1 applied inside,
+ *     S_t = S_{t-1} + k'_t^T v_t,   z_t = z_{t-1} + k'_t,
+ *     o_t = (q'_t S_t) / (q'_t . z_t)
+ * evaluated with the chunked loop of [P3] "DeltaNet (Parallelizing linear
+ * transformers with delta rule)": per chunk O = (Q'S + tril(Q'K'^T) V) /
+ * (Q'z + tril(Q'K'^T) 1), S += K'^T V, z += K'^T 1.
+ *   q, k raw (feature map applied inside); v unmapped.
+ *   S0, z0 nullable (zero); S_out, z_out nullable.  S_out may equal S0 and
+ *   z_out may equal z0.  Other arguments as deltanet_chunk_fwd (no beta, alpha).
+ */
+int linear_attn_fwd(const void *q, const void *k, const void *v,
+                    const float *S0, const float *z0,
+                    void *o, float *S_out, float *z_out,
+                    int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                    void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
+ * Synchronise `cuda_stream` and read the sticky device status word of
+ * `workspace`: DN_OK, or DN_ERR_DEVICE_TIMEOUT if any earlier kernel given
+ * this workspace ran out of a bounded wait (results of that call are then
+ * undefined).  Clear it with deltanet_workspace_init.
+ */
+int deltanet_get_device_status(const void *workspace, void *cuda_stream);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing arrives on, for at most `wait_ns` nanoseconds (<= 2e9),
+ * then records DN_ERR_DEVICE_TIMEOUT in the workspace status word and exits.
+ * Used by tests to show that a wait that runs out ends in a status the host
+ * reads, with the context still usable.
+ */
+int deltanet_selftest_wait_timeout(void *workspace, size_t ws_bytes, long long wait_ns,
+                                   void *cuda_stream);
+
+/* Static string for a status code. */
+const char *deltanet_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int deltanet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTANET_H_ */

@@ -1,0 +1,153 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library loads, exports every function that include/deltanet.h declares,
+and rejects bad arguments with the documented status codes before making any
+CUDA call (so these run on a machine without a GPU).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from deltanet_sequence_mixing_b200 import _lib
+from deltanet_sequence_mixing_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            if not m.group(0).lstrip().startswith(("typedef", "#")):
+                names.add(m.group(1))
+    return names
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared_functions()
+    for n in ("deltanet_chunk_fwd", "deltanet_decode_step", "linear_attn_fwd",
+              "deltanet_workspace_bytes", "deltanet_get_device_status", "deltanet_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert names, "no declarations parsed"
+    for n in sorted(names):
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+        assert n in _lib.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_status_strings(L):
+    for code in range(0, -7, -1):
+        s = _lib.status_string(code)
+        assert s and s != "unknown status"
+    assert _lib.status_string(-99) == "unknown status"
+    assert L.deltanet_version() >= 100
+
+
+def test_workspace_bytes(L):
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 64, 1) >= 256
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 96, 128, 64, 1) == 0
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 32, 1) == 0
+    assert L.deltanet_workspace_bytes(-1, 16, 4096, 128, 128, 64, 1) == 0
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 64, 7) == 0
+
+
+# Fake, never dereferenced device addresses: every call below must be rejected
+# on the host before any CUDA call.
+A = 1 << 32
+MB = 1 << 20
+
+
+def _chunk(L, q=A, k=A + 64 * MB, v=A + 128 * MB, beta=A + 192 * MB, alpha=None, S0=None,
+           o=A + 256 * MB, S_out=A + 320 * MB, B=2, H=2, T=100, Dk=64, Dv=64, C=64, dt=1,
+           ws=A + 400 * MB, ws_bytes=256):
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return L.deltanet_chunk_fwd(vp(q), vp(k), vp(v), vp(beta), vp(alpha), vp(S0), vp(o),
+                                vp(S_out), B, H, T, Dk, Dv, C, dt, vp(ws), ws_bytes, None)
+
+
+def test_chunk_rejects_bad_arguments(L):
+    E = _lib
+    assert _chunk(L, q=None) == E.DN_ERR_INVALID_ARG
+    assert _chunk(L, beta=None) == E.DN_ERR_INVALID_ARG
+    assert _chunk(L, o=None) == E.DN_ERR_INVALID_ARG
+    assert _chunk(L, B=-1) == E.DN_ERR_INVALID_ARG
+    assert _chunk(L, T=-5) == E.DN_ERR_INVALID_ARG
+    assert _chunk(L, Dk=96) == E.DN_ERR_UNSUPPORTED
+    assert _chunk(L, Dv=32) == E.DN_ERR_UNSUPPORTED
+    assert _chunk(L, C=32) == E.DN_ERR_UNSUPPORTED
+    assert _chunk(L, dt=5) == E.DN_ERR_UNSUPPORTED
+    assert _chunk(L, ws=None) == E.DN_ERR_WORKSPACE
+    assert _chunk(L, ws_bytes=16) == E.DN_ERR_WORKSPACE
+    assert _chunk(L, q=A + 8) == E.DN_ERR_ALIGNMENT
+    assert _chunk(L, o=A + 256 * MB + 2) == E.DN_ERR_ALIGNMENT
+    assert _chunk(L, S0=A + 500 * MB + 4) == E.DN_ERR_ALIGNMENT
+
+
+def test_chunk_rejects_overlaps(L):
+    E = _lib
+    assert _chunk(L, o=A + 4096) == E.DN_ERR_INVALID_ARG  # o inside q
+    assert _chunk(L, S_out=A + 64 * MB) == E.DN_ERR_INVALID_ARG  # S_out inside k
+    S0 = A + 500 * MB
+    assert _chunk(L, S0=S0, S_out=S0 + 256) == E.DN_ERR_INVALID_ARG  # partial overlap
+    assert _chunk(L, ws=A + 256 * MB) == E.DN_ERR_INVALID_ARG  # workspace inside o
+
+
+def test_decode_rejects_bad_arguments(L):
+    E = _lib
+    vp = ctypes.c_void_p
+
+    def dec(q=A, k=A + MB, v=A + 2 * MB, beta=A + 3 * MB, alpha=None, S=A + 8 * MB,
+            o=A + 4 * MB, B=4, H=2, Dk=128, Dv=128, dt=1):
+        f = lambda x: None if x is None else vp(x)
+        return L.deltanet_decode_step(f(q), f(k), f(v), f(beta), f(alpha), f(S), f(o), B, H, Dk,
+                                      Dv, dt, None)
+
+    assert dec(S=None) == E.DN_ERR_INVALID_ARG
+    assert dec(beta=None) == E.DN_ERR_INVALID_ARG
+    assert dec(Dk=48) == E.DN_ERR_UNSUPPORTED
+    assert dec(S=A + 8 * MB + 4) == E.DN_ERR_ALIGNMENT
+    assert dec(o=A + 8 * MB) == E.DN_ERR_INVALID_ARG  # o inside S
+    assert dec(B=-2) == E.DN_ERR_INVALID_ARG
+
+
+def test_linear_rejects_bad_arguments(L):
+    E = _lib
+    vp = ctypes.c_void_p
+
+    def lin(q=A, k=A + 64 * MB, v=A + 128 * MB, S0=None, z0=None, o=A + 256 * MB,
+            S_out=None, z_out=None, Dk=64, C=64):
+        f = lambda x: None if x is None else vp(x)
+        return L.linear_attn_fwd(f(q), f(k), f(v), f(S0), f(z0), f(o), f(S_out), f(z_out),
+                                 2, 2, 100, Dk, 64, C, 1, vp(A + 400 * MB), 256, None)
+
+    assert lin(v=None) == E.DN_ERR_INVALID_ARG
+    assert lin(Dk=80) == E.DN_ERR_UNSUPPORTED
+    assert lin(C=96) == E.DN_ERR_UNSUPPORTED
+    assert lin(z0=A + 300 * MB, z_out=A + 300 * MB + 4) == E.DN_ERR_ALIGNMENT
+    assert lin(z0=A + 300 * MB, z_out=A + 300 * MB + 16) == E.DN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    import deltanet_sequence_mixing_b200 as dn
+
+    x = torch.zeros(1, 1, 4, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        dn.deltanet_chunk_fwd(x, x, x, torch.zeros(1, 1, 4))
