@@ -220,7 +220,7 @@ def kernel_hash():
 def traffic_from_profile():
     """DRAM bytes per launch of the chunk kernel from the committed ncu summary,
     or None if it was taken on a different kernel source."""
-    p = os.path.join(ROOT, "profiles", "chunk_fwd_prefill_B4H16T4096D128.md")
+    p = os.path.join(ROOT, "profiles", "chunk_tc_kernel_prefill_B4H16T4096D128.md")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -408,6 +408,33 @@ def extras_measure(dn, gen, dev, stream, peaks):
     return out
 
 
+def profile_run(args):
+    """Launch one kernel on its workload (warm-up launches + 1), for ncu."""
+    import deltanet_sequence_mixing_b200 as dn
+    from deltanet_sequence_mixing_b200 import inputs as gen
+
+    dev = torch.device("cuda", 0)
+    n = args.warmup + 1
+    if args.profile in ("chunk", "gated", "linear"):
+        w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR}[args.profile]
+        x = gen.make_workload(w, seed=0, device=dev)
+        for _ in range(n):
+            if args.profile == "linear":
+                dn.linear_attn_fwd(x["q"], x["k"], x["v"], C=w.C)
+            else:
+                dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C)
+    else:
+        B, H, D = gen.DECODE_SEQS, gen.DECODE_HEADS, 128
+        S = torch.randn(B, H, D, D, device=dev) * 0.01
+        st = gen.make_decode_step_inputs(B, H, D, D, torch.bfloat16, seed=0, device=dev)
+        for _ in range(n):
+            dn.deltanet_decode_step(st["q"], st["k"], st["v"], st["beta"], S)
+    torch.cuda.synchronize()
+    status = dn.deltanet_get_device_status(dev)
+    print(json.dumps({"profile": args.profile, "launches": n, "status": status}))
+    return 0 if status == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,11 +444,16 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--profile", choices=["chunk", "linear", "gated", "decode"], default=None,
+                    help="untimed run for a profiler: --warmup launches of one kernel on its "
+                         "workload, then one more (the one to capture)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return profile_run(args)
 
     world, rank, local = dist_setup(args)
     import deltanet_sequence_mixing_b200 as dn
