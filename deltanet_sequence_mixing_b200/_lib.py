@@ -31,6 +31,8 @@ SIGNATURES = {
     "deltanet_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "linear_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "deltanet_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _i, _i, _i, _i, _i, _i, _i, _vp]),
     "deltanet_get_device_status": (_i, [_vp, _vp]),
     "deltanet_selftest_wait_timeout": (_i, [_vp, _sz, _ll, _vp]),
     "deltanet_status_string": (ctypes.c_char_p, [_i]),

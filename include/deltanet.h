@@ -165,6 +165,41 @@ int deltanet_get_device_status(const void *workspace, void *cuda_stream);
 int deltanet_selftest_wait_timeout(void *workspace, size_t ws_bytes, long long wait_ns,
                                    void *cuda_stream);
 
+/*
+ * deltanet_chunk_fwd without a workspace argument, for callers that cannot
+ * allocate device memory where they call the library: code running inside
+ * another framework's allocator or memory-pool hooks (a cudaMalloc there would
+ * re-enter the allocator), plug-ins or embedded runtimes whose device memory is
+ * budgeted up front, and paths that must avoid cudaMalloc because it can
+ * synchronise the device.  The pages have no counterpart to this; it only
+ * changes where the scratch lives.
+ *
+ * Arguments, computation, results and status codes are those of
+ * deltanet_chunk_fwd.  The scratch (the device status word) comes from a
+ * static device array of 4096 bytes inside the library, one per device that
+ * loads it, held until the process exits.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with the caller's current device, which must be
+ *     the device of the pointers and the stream); make that first call before
+ *     any stream capture.
+ *   - Each call clears the status word with an asynchronous memset on
+ *     `cuda_stream`, then launches the kernel there.  A call rejected by
+ *     validation may still have cleared that private word; it touches none of
+ *     the caller's buffers.
+ *   - All calls on a device share the one array: calls that overlap on the GPU
+ *     (for instance on different streams) race on it.  The status word cannot
+ *     be read back through this entry point; use deltanet_chunk_fwd with a
+ *     caller-owned workspace when bounded-wait timeouts must be observed.
+ *   - A problem whose workspace need (deltanet_workspace_bytes) exceeds 4096
+ *     bytes is rejected with DN_ERR_WORKSPACE.
+ */
+int deltanet_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                               const float *beta, const float *alpha, const float *S0,
+                               void *o, float *S_out,
+                               int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                               void *cuda_stream);
+
 /* Static string for a status code. */
 const char *deltanet_status_string(int status);
 
