@@ -89,6 +89,7 @@ int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
   p.status = static_cast<unsigned int*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dn::chunk_ws_supported(p)) return map_cuda(dn::launch_chunk_ws(p, st));
   if (dn::chunk_tc_supported(p)) return map_cuda(dn::launch_chunk_tc(p, st));
   if (dn::chunk_simt_supported(p.Dk, p.Dv, p.C)) return map_cuda(dn::launch_chunk_simt(p, st));
   return DN_ERR_UNSUPPORTED;

@@ -196,4 +196,42 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c16) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c16 ^ (r & 7)) << 4));
 }
 
+// K-major and MN-major descriptors of 128-byte-swizzled bf16 tiles (8-row
+// groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return sw128_desc(addr, 16, 1024); }
+__device__ __forceinline__ uint64_t desc_mn(uint32_t addr, uint32_t lbo) {
+  return sw128_desc(addr, lbo, 1024);
+}
+
+// Named barrier over `count` threads; the AND form returns true only if every
+// participating thread passed true (a uniform decision for the whole group).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.and.pred po, %2, %3, pi;"
+      " selp.u32 %0, 1, 0, po; }"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+// Store 8 floats as one 16-byte chunk of bf16 (shared or global address).
+__device__ __forceinline__ void st_bf16x8(void* dst, const float* x) {
+  uint4 u;
+  u.x = pack2_bf16(x[0], x[1]);
+  u.y = pack2_bf16(x[2], x[3]);
+  u.z = pack2_bf16(x[4], x[5]);
+  u.w = pack2_bf16(x[6], x[7]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
 }  // namespace dn

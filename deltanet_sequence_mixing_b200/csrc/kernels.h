@@ -1,6 +1,7 @@
 // Internal launcher declarations shared by the ABI layer and the kernel files.
 // Not part of the public interface (that is include/deltanet.h).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -54,6 +55,14 @@ struct DecodeProblem {
   int bf16;
 };
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t st);
+
+// Warp-specialised tcgen05 chunked delta rule (bf16, C = 64).
+cudaError_t launch_chunk_ws(const ChunkProblem& p, cudaStream_t st);
+bool chunk_ws_supported(const ChunkProblem& p);
+
+// 3-D TMA map over a (BH, T, D) bf16 tensor: 64 x 64 boxes, 128-byte swizzle,
+// rows past T read as zeros.
+bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, int D, int T, int BH);
 
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(unsigned int* status, long long wait_ns, cudaStream_t st);
