@@ -467,7 +467,7 @@ def main():
     sets = [gen.make_workload(w, seed=rank * 2 + i, device=dev) for i in range(2)]
     o = [torch.empty_like(s["v"]) for s in sets]
     S = [torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev) for _ in sets]
-    ws = dn.workspace_for(dev)
+    ws = dn.workspace_for(dev, dn.lib().deltanet_workspace_bytes(w.B, w.H, w.T, w.Dk, w.Dv, w.C, 1))
 
     def step(i):
         j = i & 1

@@ -89,7 +89,11 @@ int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
   p.status = static_cast<unsigned int*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dn::chunk_ws_supported(p)) return map_cuda(dn::launch_chunk_ws(p, st));
+  if (dn::chunk_main_supported(p)) {
+    const dn::WyWorkspace w =
+        dn::chunk_main_carve(static_cast<uint8_t*>(ws) + kStatusBytes, p.B, p.H, p.T);
+    return map_cuda(dn::launch_chunk_main(p, w, st));
+  }
   if (dn::chunk_tc_supported(p)) return map_cuda(dn::launch_chunk_tc(p, st));
   if (dn::chunk_simt_supported(p.Dk, p.Dv, p.C)) return map_cuda(dn::launch_chunk_simt(p, st));
   return DN_ERR_UNSUPPORTED;
@@ -102,6 +106,8 @@ extern "C" {
 size_t deltanet_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
   if (B < 0 || H < 0 || T < 0 || !valid_dim(Dk) || !valid_dim(Dv)) return 0;
   if ((C != 64 && C != 128) || (dt != DN_F32 && dt != DN_BF16)) return 0;
+  // bf16 chunk size 64: room for the per-chunk WY factors of the pre-pass
+  if (dt == DN_BF16 && C == 64 && T > 0) return kStatusBytes + dn::chunk_main_workspace(B, H, T);
   return kStatusBytes;
 }
 

@@ -1,0 +1,489 @@
+// tcgen05 chunked DeltaNet forward (bf16 operands, float32 accumulation and
+// state): the bf16 path of deltanet_chunk_fwd, run after the chunk-parallel
+// WY pre-pass (tsolve.cu) has written Tb = (I + A)^-1 diag(beta), Tbg =
+// Tb diag(gamma) and the decay prefix g of every chunk into the workspace.
+//
+// Per chunk of C = 64 rows entered with state S ("GPT-2 から Kimi K3 まで",
+// news.ainew.jp, section "DeltaNet (Parallelizing linear transformers with delta
+// rule)"; gate from the Gated DeltaNet paragraph of "How a Baseten Engineer
+// Traced 7 Years of Attention Mechanism Evolution"):
+//   P  = tril(Q K^T) * Gamma,  W = Tbg K,  Uh = Tb V          (state-independent)
+//   [gamma Q S ; W S] = [diag(gamma) Q ; W] S                  (one M = 128 MMA)
+//   U  = Uh - W S                                              (the chunk's deltas)
+//   O  = gamma Q S + P U        (accumulated onto the same TMEM tile)
+//   S <- gamma_last S + K^T (diag(Gamma_last,.) U)             (float32 registers)
+//
+// One CTA per (b, h, 64-column slice of Dv), 9 warps:
+//   warp 8     producer: TMA of K, Q, V, Tb, Tbg (+ beta and g rows) into a
+//              two-stage ring, L2 prefetch two chunks ahead
+//   warps 4-7  prep, one chunk ahead of the chain: the three S-independent
+//              MMAs, then P and W to bf16 shared memory (in parallel halves),
+//              diag(gamma) applied to Q in place
+//   warps 0-3  chain: [Q;W]S, U, PU + K^T U, the state update; warps 0-1 then
+//              drain the output tile while warps 2-3 start the next chunk
+// Accumulators live in TMEM (512 columns), every operand in the 128-byte-
+// swizzled canonical layout, the running state in float32 registers.  All
+// waits are bounded; a wait that runs out sets the workspace status word and
+// the CTA winds down (copies drained, TMEM freed) without trapping.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dn {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kDVS = 64;
+constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
+constexpr int kWG = 128;
+constexpr int kThreads = 2 * kWG + 32;
+constexpr int kBarChain = 1, kBarPrep = 2, kBarChainHi = 3, kBarChainLo = 4;
+
+// TMEM columns: G (P scores), W, Uh[2], QW[2] (lanes 0-63: O, lanes 64-127: WS), dS
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_UH = 192, TM_QW = 320, TM_DS = 448;
+
+template <int DK>
+struct MainLayout {
+  static constexpr int KB = DK / 64;
+  static constexpr uint32_t KB_STRIDE = 3 * kTile;  // [K | Q | W] per 64 columns of Dk
+  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
+  static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | Tbg | beta, g
+  static constexpr uint32_t TB_OFF = V_OFF + kTile;
+  static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
+  static constexpr uint32_t VEC_OFF = TBG_OFF + kTile;
+  static constexpr uint32_t STAGE = VEC_OFF + 1024;
+  static constexpr uint32_t P_OFF = 2 * STAGE;        // P[0] | P[1] | U | UT
+  static constexpr uint32_t U_OFF = P_OFF + 2 * kTile;
+  static constexpr uint32_t UT_OFF = U_OFF + kTile;
+  static constexpr uint32_t S_OFF = UT_OFF + kTile;   // bf16 state, DK rows x 128 B
+  static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // chain copy of g per parity: [2][64]
+  static constexpr uint32_t BAR_OFF = CV_OFF + 2 * 64 * 4;
+  static constexpr uint32_t BYTES = BAR_OFF + 128;
+  static constexpr uint32_t ALLOC = BYTES + 1024;
+  static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+// mbarrier slots; each completes once per chunk (or once per use of a parity),
+// so every waiter is at most one phase behind and parity waits are unambiguous.
+constexpr uint32_t B_FULL = 0, B_EMPTY = 16, B_READY = 32, B_FREE = 48, B_PMMA = 64, B_CMMA3 = 72,
+                   B_CMMA4 = 80, B_FINP = 88, B_FINC = 96, B_TMEM = 104, B_ABORT = 108;
+
+__device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+template <int DK, bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
+                      const __grid_constant__ CUtensorMap tmTbg, const ChunkProblem p,
+                      const float* __restrict__ gw) {
+  using L = MainLayout<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int j0 = blockIdx.y * kDVS;
+  const int T = p.T, Dv = p.Dv;
+  const int nchunks = (T + kC - 1) / kC;
+  const uint32_t bar = sb + L::BAR_OFF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR_OFF + B_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF + B_ABORT);
+  float* cvec = reinterpret_cast<float*>(sm + L::CV_OFF);
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's vector rows
+      mbar_init(bar + B_EMPTY + 8 * i, 1);
+      mbar_init(bar + B_READY + 8 * i, 1);
+      mbar_init(bar + B_FREE + 8 * i, 1);
+    }
+    mbar_init(bar + B_PMMA, 1);
+    mbar_init(bar + B_CMMA3, 1);
+    mbar_init(bar + B_CMMA4, 1);
+    mbar_init(bar + B_FINP, 1);
+    mbar_init(bar + B_FINC, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t tile_bytes = (2 * L::KB + (GATED ? 3 : 2)) * kTile;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmTb);
+      if (GATED) prefetch_tmap(&tmTbg);
+    }
+    int issued = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1, use = c >> 1;
+      const int c0 = c * kC, n = min(kC, T - c0);
+      bool ok = true;
+      if (lane == 0 && use > 0) ok = mbar_wait(bar + B_EMPTY + 8 * s, (use - 1) & 1, wc);
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      const uint32_t st = sb + s * L::STAGE;
+      const uint32_t full = bar + B_FULL + 8 * s;
+      if (lane == 0) {
+        mbar_expect_tx(full, tile_bytes);
+#pragma unroll
+        for (int kb = 0; kb < L::KB; ++kb) {
+          tma_load_3d(st + kb * L::KB_STRIDE + L::K_OFF, &tmK, full, kb * 64, c0, bh);
+          tma_load_3d(st + kb * L::KB_STRIDE + L::Q_OFF, &tmQ, full, kb * 64, c0, bh);
+        }
+        tma_load_3d(st + L::V_OFF, &tmV, full, j0, c0, bh);
+        tma_load_3d(st + L::TB_OFF, &tmTb, full, 0, c0, bh);
+        if (GATED) tma_load_3d(st + L::TBG_OFF, &tmTbg, full, 0, c0, bh);
+      }
+      // beta and g rows of the chunk (rows >= n: beta 0, g flat)
+      float* vs = reinterpret_cast<float*>(sm + s * L::STAGE + L::VEC_OFF);
+      const size_t tb = (size_t)bh * T + c0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = lane + 32 * h;
+        vs[r] = r < n ? p.beta[tb + r] : 0.f;
+        if (GATED) vs[64 + r] = gw[((size_t)bh * nchunks + c) * kC + r];
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(full);
+        if (c + 2 < nchunks) {  // warm L2 for the chunk after next
+          const int cn = c0 + 2 * kC;
+#pragma unroll
+          for (int kb = 0; kb < L::KB; ++kb) {
+            prefetch_l2_3d(&tmK, kb * 64, cn, bh);
+            prefetch_l2_3d(&tmQ, kb * 64, cn, bh);
+          }
+          prefetch_l2_3d(&tmV, j0, cn, bh);
+          prefetch_l2_3d(&tmTb, 0, cn, bh);
+          if (GATED) prefetch_l2_3d(&tmTbg, 0, cn, bh);
+        }
+      }
+      issued = c + 1;
+    }
+    if (lane == 0) {  // never leave with copies in flight
+      int zero = 0;
+      const WaitCtl drain{&zero, p.status, kWaitLimitNs};
+      for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
+        (void)mbar_wait(bar + B_FULL + 8 * (c & 1), (c >> 1) & 1, drain);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- prep --
+    const int pt = tid - kWG;
+    const int row = pt & 63;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int b = c & 1, use = c >> 1;
+      const uint32_t st = sb + b * L::STAGE;
+      uint8_t* stp = sm + b * L::STAGE;
+      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
+      if (c >= 2) {  // the chain is done with this parity's P, Uh and g copy
+        ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FREE + 8 * b, (use - 1) & 1, wc));
+        if (!ok) break;
+      }
+      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FULL + 8 * b, use & 1, wc));
+      if (!ok) break;
+
+      // ---- P scores = Q K^T (lanes 0-63), W (lanes 64-127), Uh (lanes 64-127) ----
+      if (pt == 0) {
+        tc_fence_after();
+        constexpr uint32_t idg = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
+        constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
+          mma_bf16_ss(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), idg, ks > 0);
+        }
+        const uint32_t aw = st + (GATED ? L::TB_OFF : L::V_OFF);  // rows 64-127: Tbg (Tb)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ss(tmem + TM_W, desc_k(aw + ks * 32),
+                      desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), idw, ks > 0);
+          mma_bf16_ss(tmem + TM_UH + 64 * b, desc_k(st + L::V_OFF + ks * 32),
+                      desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
+        }
+        mma_commit(bar + B_PMMA);
+      }
+      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_PMMA, c & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      if (pt < 64) {
+        // P row: tril(QK^T) * Gamma -> bf16 P[b]
+        uint32_t g[64];
+        tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
+        tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+        tmem_wait_ld();
+        const float gr = GATED ? vs[64 + row] : 0.f;
+        uint8_t* ptile = sm + L::P_OFF + b * kTile;
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int sc = c16 * 8 + e;
+            float val = __uint_as_float(g[sc]);
+            if (GATED) val *= __expf(gr - vs[64 + sc]);
+            x[e] = sc <= row ? val : 0.f;
+          }
+          st_bf16x8(ptile + sw128_off(row, c16), x);
+        }
+        if (GATED) cvec[b * 64 + row] = vs[64 + row];
+      } else {
+        // W row -> bf16 into the stage, right after Q
+#pragma unroll
+        for (int q = 0; q < DK / 32; ++q) {
+          uint32_t w[32];
+          tmem_ld32(tmem + lane_base + TM_W + q * 32, w);
+          tmem_wait_ld();
+          uint8_t* wt = stp + (q >> 1) * L::KB_STRIDE + L::W_OFF;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
+        }
+      }
+      if (GATED) {  // Q <- diag(gamma) Q in place (the scores above used the plain Q)
+        const float gam = __expf(vs[64 + row]);
+        const int h = pt >> 6;
+#pragma unroll
+        for (int i = 0; i < DK / 16; ++i) {
+          const int c16 = h * (DK / 16) + i;  // this thread's half of the row's 16-byte chunks
+          uint8_t* ptr = stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16 & 7);
+          uint4 u = *reinterpret_cast<uint4*>(ptr);
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
+            wv[e] = pack2_bf16(f.x * gam, f.y * gam);
+          }
+          *reinterpret_cast<uint4*>(ptr) = u;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarPrep, kWG);
+      if (pt == 0) mbar_arrive(bar + B_READY + 8 * b);
+    }
+    if (pt == 0) {
+      tc_fence_after();
+      mma_commit(bar + B_FINP);
+      int zero = 0;
+      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
+      (void)mbar_wait(bar + B_FINP, 0, fin);
+    }
+  } else {
+    // --------------------------------------------------------------- chain --
+    const int ct = tid;
+    const int row = ct & 63;
+    const size_t s_base = (size_t)bh * DK * Dv;
+    float sreg[kDVS];
+    if (ct < DK) {
+      const float* src = p.S0 ? p.S0 + s_base + (size_t)ct * Dv + j0 : nullptr;
+#pragma unroll
+      for (int j = 0; j < kDVS; j += 4) {
+        const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
+      }
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(kBarChain, kWG);
+
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int b = c & 1, use = c >> 1;
+      const int c0 = c * kC, n = min(kC, T - c0);
+      const uint32_t st = sb + b * L::STAGE;
+      const uint32_t qw = tmem + TM_QW + 64 * b;
+      bool ok2 = true;
+      if (ct >= 64) {
+        // warps 2-3: [Q;W] S, then U, then issue PU and K^T U
+        ok2 = named_bar_and(kBarChainHi, 64, mbar_wait(bar + B_READY + 8 * b, use & 1, wc));
+        if (ok2) {
+          if (ct == 64) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+            for (int ks = 0; ks < DK / 16; ++ks) {
+              const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+              mma_bf16_ss(qw, desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile), id, ks > 0);
+            }
+            mma_commit(bar + B_CMMA3);
+          }
+          ok2 = named_bar_and(kBarChainHi, 64, mbar_wait(bar + B_CMMA3, c & 1, wc));
+        }
+        if (ok2) {
+          tc_fence_after();
+          const float wl = GATED ? __expf(cvec[b * 64 + n - 1] - cvec[b * 64 + row]) : 1.f;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t ws[32], uh[32];
+            tmem_ld32(qw + lane_base + q * 32, ws);
+            tmem_ld32(tmem + lane_base + TM_UH + 64 * b + q * 32, uh);
+            tmem_wait_ld();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              float x[8], y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                x[e] = __uint_as_float(uh[cc * 8 + e]) - __uint_as_float(ws[cc * 8 + e]);
+                y[e] = x[e] * wl;
+              }
+              st_bf16x8(sm + L::U_OFF + sw128_off(row, q * 4 + cc), x);
+              if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(row, q * 4 + cc), y);
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          named_bar_sync(kBarChainHi, 64);
+          if (ct == 64) {
+            tc_fence_after();
+            const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
+            const uint32_t pa = sb + L::P_OFF + b * kTile;
+            constexpr uint32_t idp = idesc_bf16(128, 64, false, true);
+            constexpr uint32_t ids = idesc_bf16(128, 64, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              mma_bf16_ss(qw, desc_k(pa + ks * 32), desc_mn(sb + L::U_OFF + ks * 2048, kTile), idp, 1);
+              mma_bf16_ss(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                          desc_mn(ut + ks * 2048, kTile), ids, ks > 0);
+            }
+            mma_commit(bar + B_CMMA4);
+            mma_commit(bar + B_EMPTY + 8 * b);  // the stage may be refilled
+          }
+        }
+      }
+      ok = named_bar_and(kBarChain, kWG, ok2 && mbar_wait(bar + B_CMMA4, c & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+
+      // ---- state update (all lanes 0..DK-1), then release the next [Q;W]S ----
+      if (ct < DK) {
+        const float carry = GATED ? __expf(cvec[b * 64 + n - 1]) : 1.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t ds[32];
+          tmem_ld32(tmem + lane_base + TM_DS + q * 32, ds);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sreg[q * 32 + e] = fmaf(carry, sreg[q * 32 + e], __uint_as_float(ds[e]));
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarChain, kWG);
+
+      // ---- outputs O = gamma QS + PU (lanes 0-63), drained by warps 0-1 ----
+      if (ct < 64) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + row) * Dv + j0;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t ov[32];
+          tmem_ld32(qw + lane_base + q * 32, ov);
+          tmem_wait_ld();
+          if (row < n) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              st_bf16x8(orow + q * 32 + cc * 8, reinterpret_cast<const float*>(ov) + cc * 8);
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(kBarChainLo, 64);
+        if (ct == 0) mbar_arrive(bar + B_FREE + 8 * b);
+      }
+    }
+    if (p.S_out && ct < DK) {
+      float* dst = p.S_out + s_base + (size_t)ct * Dv + j0;
+#pragma unroll
+      for (int j = 0; j < kDVS; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
+    }
+    if (ct == 64) {
+      tc_fence_after();
+      mma_commit(bar + B_FINC);
+      int zero = 0;
+      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
+      (void)mbar_wait(bar + B_FINC, 0, fin);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int DK, bool GATED>
+cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  using L = MainLayout<DK>;
+  const int BH = p.B * p.H;
+  const int nchunks = (p.T + kC - 1) / kC;
+  cudaError_t e = launch_tsolve(p, w, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mq, mk, mv, mtb, mtbg;
+  if (!make_tmap_3d_bf16(&mq, p.q, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, p.k, DK, p.T, BH) ||
+      !make_tmap_3d_bf16(&mv, p.v, p.Dv, p.T, BH) ||
+      !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
+      !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))
+    return cudaErrorInvalidValue;
+  auto kern = chunk_main_kernel<DK, GATED>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
+  kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, mtb, mtbg, p, w.g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_main_supported(const ChunkProblem& p) {
+  return p.bf16 && p.mode == Mode::Delta && p.T > 0 && p.C == 64 && (p.Dk == 64 || p.Dk == 128) &&
+         (p.Dv == 64 || p.Dv == 128);
+}
+
+size_t chunk_main_workspace(int B, int H, int T) {
+  const size_t nch = ((size_t)T + kC - 1) / kC;
+  const size_t tiles = (size_t)B * H * nch;
+  return tiles * (2 * (size_t)kC * kC * 2 + (size_t)kC * 4);  // Tb, Tbg (bf16) and g (f32)
+}
+
+WyWorkspace chunk_main_carve(void* base, int B, int H, int T) {
+  const size_t nch = ((size_t)T + kC - 1) / kC;
+  const size_t tiles = (size_t)B * H * nch;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  WyWorkspace w;
+  w.tb = reinterpret_cast<__nv_bfloat16*>(p);
+  w.tbg = reinterpret_cast<__nv_bfloat16*>(p + tiles * kC * kC * 2);
+  w.g = reinterpret_cast<float*>(p + 2 * tiles * kC * kC * 2);
+  return w;
+}
+
+cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
+  return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
+}
+
+}  // namespace dn

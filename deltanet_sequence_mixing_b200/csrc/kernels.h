@@ -2,6 +2,7 @@
 // Not part of the public interface (that is include/deltanet.h).
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -56,13 +57,23 @@ struct DecodeProblem {
 };
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t st);
 
-// Warp-specialised tcgen05 chunked delta rule (bf16, C = 64).
-cudaError_t launch_chunk_ws(const ChunkProblem& p, cudaStream_t st);
-bool chunk_ws_supported(const ChunkProblem& p);
-
 // 3-D TMA map over a (BH, T, D) bf16 tensor: 64 x 64 boxes, 128-byte swizzle,
 // rows past T read as zeros.
 bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, int D, int T, int BH);
+
+// Per-chunk WY factors written by the pre-pass and read by the chunk kernel.
+struct WyWorkspace {
+  __nv_bfloat16* tb;   // [B*H][chunks][64][64]  T diag(beta)
+  __nv_bfloat16* tbg;  // [B*H][chunks][64][64]  T diag(beta) diag(exp(g))   (gated)
+  float* g;            // [B*H][chunks][64]      cumulative log decay        (gated)
+};
+cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
+
+// tcgen05 chunked delta rule after the pre-pass (bf16, C = 64).
+bool chunk_main_supported(const ChunkProblem& p);
+size_t chunk_main_workspace(int B, int H, int T);
+WyWorkspace chunk_main_carve(void* base, int B, int H, int T);
+cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(unsigned int* status, long long wait_ns, cudaStream_t st);

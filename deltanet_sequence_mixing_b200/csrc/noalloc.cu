@@ -16,9 +16,11 @@
 
 namespace {
 
-// The scratch: the device status word and its padding, up to this many bytes.
-// Every device that loads the library holds one copy until the process exits.
-constexpr size_t kNoAllocScratchBytes = 4096;
+// The scratch: the device status word plus, for bf16 problems, the per-chunk
+// WY factors of the pre-pass (16.25 KB per (b, h, 64-token chunk)), up to this
+// many bytes; larger problems are rejected.  Every device that loads the
+// library holds one copy until the process exits.
+constexpr size_t kNoAllocScratchBytes = 1u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -61,8 +63,9 @@ extern "C" int deltanet_chunk_fwd_noalloc(const void* q, const void* k, const vo
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return DN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  // The status word must start at zero for this call.
-  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return DN_ERR_CUDA;
+  // The status word (first 256 bytes) must start at zero for this call; the rest
+  // of the scratch is fully written by the call before it is read.
+  if (cudaMemsetAsync(scratch, 0, 256, st) != cudaSuccess) return DN_ERR_CUDA;
   return deltanet_chunk_fwd(q, k, v, beta, alpha, S0, o, S_out, B, H, T, Dk, Dv, C, dt, scratch,
                             kNoAllocScratchBytes, cuda_stream);
 }

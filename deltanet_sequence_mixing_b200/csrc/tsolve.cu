@@ -1,0 +1,265 @@
+// Chunk-parallel WY pre-pass of the tcgen05 delta-rule forward: for every
+// (b, h, chunk) it forms T = (I + A)^-1 with
+//   A = strict_lower(diag(beta) (K K^T * Gamma)),   Gamma_rs = exp(g_r - g_s),
+// and writes Tb = T diag(beta) (and, gated, Tbg = Tb diag(exp(g))) as bf16
+// 64 x 64 tiles into the workspace, plus the chunk's decay prefix g.  These are
+// the state-independent parts of the Householder / WY reparameterisation
+// ("GPT-2 から Kimi K3 まで", news.ainew.jp, section "DeltaNet (Parallelizing linear
+// transformers with delta rule)"); the chunk kernel then applies them with
+// tensor-core products, keeping only matrix products on its serial state chain.
+//
+// One 128-thread CTA per chunk, several CTAs per SM: the solve is a short chain
+// of dependent steps, so it is latency-bound per chunk and the grid's
+// parallelism over chunks hides that latency.
+//   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
+//   2. G = K K^T with bf16 WMMA (float32 accumulate) straight into the A scratch.
+//   3. A = mask / scale G in place.
+//   4. Four 16x16 diagonal inverses (one column per lane, right-looking
+//      substitution so only one multiply-add per step is on the dependency
+//      chain), then tf32 WMMA merges 16 -> 32 -> 64:
+//      T_ij = -T_ii A_ij T_jj,  T21 = -T22 A21 T11.
+//   5. Tb, Tbg -> global (row-major bf16, 8 KB per tile).
+#include <cuda_bf16.h>
+#include <mma.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dn {
+namespace {
+
+using namespace nvcuda;
+
+constexpr int kC = 64;
+constexpr int kThreads = 128;
+constexpr int kApad = 68;
+constexpr int kKpad = 8;  // bf16 padding of the K rows (keeps WMMA rows 16-byte aligned)
+
+template <typename Frag>
+__device__ __forceinline__ void to_tf32(Frag& f) {
+#pragma unroll
+  for (int t = 0; t < f.num_elements; ++t) f.x[t] = wmma::__float_to_tf32(f.x[t]);
+}
+
+template <int DK, bool GATED>
+__global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
+                                                          const float* __restrict__ beta,
+                                                          const float* __restrict__ alpha,
+                                                          __nv_bfloat16* __restrict__ tb_out,
+                                                          __nv_bfloat16* __restrict__ tbg_out,
+                                                          float* __restrict__ g_out, int T,
+                                                          int nchunks) {
+  constexpr int KS = DK + kKpad;
+  extern __shared__ __align__(128) uint8_t tsolve_smem[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(tsolve_smem);
+  float* Am = reinterpret_cast<float*>(tsolve_smem + kC * KS * 2);
+  float* Tm = Am + kC * kApad;
+  float* vb = Tm + kC * kApad;
+  float* vg = vb + 64;
+  float* veg = vg + 64;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int c0 = chunk * kC, n = min(kC, T - c0);
+
+  // 1. K tile, beta and the log-decay prefix g (rows >= n: k = 0, beta = 0, alpha = 1)
+  {
+    const __nv_bfloat16* src = k + ((size_t)bh * T + c0) * DK;
+    constexpr int kVecPerRow = DK / 8;
+    for (int i = tid; i < kC * kVecPerRow; i += kThreads) {
+      const int r = i / kVecPerRow, v = i % kVecPerRow;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (r < n) u = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * DK) + v);
+      *reinterpret_cast<uint4*>(Ks + r * KS + v * 8) = u;
+    }
+    if (tid < 64) {
+      const size_t tb = (size_t)bh * T + c0;
+      vb[tid] = tid < n ? beta[tb + tid] : 0.f;
+      if (GATED) {
+        float x = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        if (warp == 1) {
+          float l0 = lane < n ? fmaxf(__logf(alpha[tb + lane]), -87.f) : 0.f;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+          x += l0;
+        }
+        vg[tid] = x;
+        veg[tid] = __expf(x);
+        g_out[((size_t)bh * nchunks + chunk) * kC + tid] = x;
+      }
+    }
+    // T's strictly-upper 16x16 blocks are read by the merges and must be zero
+    for (int i = tid; i < 64 * 64; i += kThreads) {
+      const int r = i >> 6, c = i & 63;
+      if ((c >> 4) > (r >> 4)) Tm[r * kApad + c] = 0.f;
+    }
+  }
+  __syncthreads();
+
+  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps)
+  {
+    wmma::fragment<wmma::matrix_a, 16, 16, 16, __nv_bfloat16, wmma::row_major> fa;
+    wmma::fragment<wmma::matrix_b, 16, 16, 16, __nv_bfloat16, wmma::col_major> fb;
+    wmma::fragment<wmma::accumulator, 16, 16, 16, float> acc;
+    for (int t = warp; t < 10; t += 4) {
+      // t -> (ti, tj) with tj <= ti: 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) 4:(2,1) 5:(2,2) 6..9:(3,*)
+      const int ti = t < 1 ? 0 : t < 3 ? 1 : t < 6 ? 2 : 3;
+      const int tj = t - ti * (ti + 1) / 2;
+      wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+      for (int kk = 0; kk < DK; kk += 16) {
+        wmma::load_matrix_sync(fa, Ks + (16 * ti) * KS + kk, KS);
+        wmma::load_matrix_sync(fb, Ks + (16 * tj) * KS + kk, KS);
+        wmma::mma_sync(acc, fa, fb, acc);
+      }
+      wmma::store_matrix_sync(Am + (16 * ti) * kApad + 16 * tj, acc, kApad, wmma::mem_row_major);
+    }
+  }
+  __syncthreads();
+
+  // 3. A = strict_lower(diag(beta) G * Gamma) in place; the upper part is zeroed
+  for (int i = tid; i < 64 * 64; i += kThreads) {
+    const int r = i >> 6, s = i & 63;
+    float a = 0.f;
+    if (s < r) {
+      a = vb[r] * Am[r * kApad + s];
+      if (GATED) a *= __expf(vg[r] - vg[s]);
+    }
+    Am[r * kApad + s] = a;
+  }
+  __syncthreads();
+
+  // 4a. diagonal 16x16 inverses: warp w, lanes 0-15 own column j of block w
+  if (lane < 16) {
+    const int o = 16 * warp, j = lane;
+    float col[16], acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      col[i] = 0.f;
+      acc[i] = 0.f;
+    }
+    // right-looking: once col[m] is final, fold it into every later row
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      col[m] = (m == j) ? 1.f : (m > j ? -acc[m] : 0.f);
+#pragma unroll
+      for (int i = m + 1; i < 16; ++i) acc[i] = fmaf(Am[(o + i) * kApad + o + m], col[m], acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tm[(o + i) * kApad + o + j] = col[i];
+  }
+  __syncthreads();
+  // 4b. T_{r,r-1} = -D_r A_{r,r-1} D_{r-1}, r = 1 (warp 0) and r = 3 (warp 2)
+  if ((warp & 1) == 0) {
+    const int o = 16 * (warp + 1), q0 = o - 16;
+    float* ys = Am + (warp == 0 ? 0 : 16) * kApad + 48;  // scratch in A's zero upper part
+    wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
+    wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
+    wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
+    wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < 16; kk += 8) {
+      wmma::load_matrix_sync(fa, Am + o * kApad + q0 + kk, kApad);
+      wmma::load_matrix_sync(fb, Tm + (q0 + kk) * kApad + q0, kApad);
+      to_tf32(fa);
+      to_tf32(fb);
+      wmma::mma_sync(acc, fa, fb, acc);
+    }
+    wmma::store_matrix_sync(ys, acc, kApad, wmma::mem_row_major);
+    __syncwarp();
+    wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < 16; kk += 8) {
+      wmma::load_matrix_sync(fa, Tm + o * kApad + o + kk, kApad);
+      wmma::load_matrix_sync(fb, ys + kk * kApad, kApad);
+      to_tf32(fa);
+      to_tf32(fb);
+      wmma::mma_sync(acc, fa, fb, acc);
+    }
+#pragma unroll
+    for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
+    wmma::store_matrix_sync(Tm + o * kApad + q0, acc, kApad, wmma::mem_row_major);
+  }
+  __syncthreads();
+  // 4c. Y = A21 T11, then T21 = -T22 Y (one 16x16 tile per warp)
+  {
+    const int ti = warp >> 1, tj = warp & 1;
+    wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
+    wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
+    wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
+    wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < 32; kk += 8) {
+      wmma::load_matrix_sync(fa, Am + (32 + 16 * ti) * kApad + kk, kApad);
+      wmma::load_matrix_sync(fb, Tm + kk * kApad + 16 * tj, kApad);
+      to_tf32(fa);
+      to_tf32(fb);
+      wmma::mma_sync(acc, fa, fb, acc);
+    }
+    wmma::store_matrix_sync(Am + (16 * ti) * kApad + 32 + 16 * tj, acc, kApad, wmma::mem_row_major);
+    __syncthreads();
+    wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < 32; kk += 8) {
+      wmma::load_matrix_sync(fa, Tm + (32 + 16 * ti) * kApad + 32 + kk, kApad);
+      wmma::load_matrix_sync(fb, Am + kk * kApad + 32 + 16 * tj, kApad);
+      to_tf32(fa);
+      to_tf32(fb);
+      wmma::mma_sync(acc, fa, fb, acc);
+    }
+#pragma unroll
+    for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
+    wmma::store_matrix_sync(Tm + (32 + 16 * ti) * kApad + 16 * tj, acc, kApad, wmma::mem_row_major);
+  }
+  __syncthreads();
+
+  // 5. Tb = T diag(beta) and Tbg = Tb diag(e^g), bf16 rows: thread -> (row, 32-column half)
+  {
+    const int row = tid & 63, h = tid >> 6;
+    const size_t tile = ((size_t)bh * nchunks + chunk) * kC * kC;
+    __nv_bfloat16* dst = tb_out + tile + row * kC + 32 * h;
+    __nv_bfloat16* dstg = GATED ? tbg_out + tile + row * kC + 32 * h : nullptr;
+    const float* trow = Tm + row * kApad + 32 * h;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      float x[8], y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int sc = 32 * h + cc * 8 + e;
+        x[e] = sc <= row ? trow[cc * 8 + e] * vb[sc] : 0.f;
+        if (GATED) y[e] = x[e] * veg[sc];
+      }
+      st_bf16x8(dst + cc * 8, x);
+      if (GATED) st_bf16x8(dstg + cc * 8, y);
+    }
+  }
+}
+
+template <int DK, bool GATED>
+cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  const int nchunks = (p.T + kC - 1) / kC;
+  constexpr size_t smem = (size_t)kC * (DK + kKpad) * 2 + 2 * (size_t)kC * kApad * 4 + 3 * 64 * 4;
+  auto kern = tsolve_kernel<DK, GATED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)nchunks, (unsigned)(p.B * p.H));
+  kern<<<grid, kThreads, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(p.k), p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
+  if (p.Dk == 64) return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace dn

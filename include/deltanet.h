@@ -57,8 +57,11 @@ typedef enum {
 typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
 
 /*
- * Bytes of device workspace the chunked calls need for this problem (at least
- * 256: the sticky device status word and its padding).  The workspace must be
+ * Bytes of device workspace the chunked calls need for this problem: 256 for
+ * the sticky device status word and its padding, plus, for bf16 inputs with
+ * C = 64, 16,640 bytes per (b, h, 64-token chunk) for the per-chunk factors
+ * T diag(beta), T diag(beta) diag(gamma) and the decay prefix that the
+ * chunk-parallel pre-pass hands to the chunk kernel.  The workspace must be
  * cleared once with deltanet_workspace_init before its first use; it may then
  * be reused by any number of calls on the same stream.  Returns 0 for sizes
  * the library rejects.
@@ -175,9 +178,11 @@ int deltanet_selftest_wait_timeout(void *workspace, size_t ws_bytes, long long w
  * changes where the scratch lives.
  *
  * Arguments, computation, results and status codes are those of
- * deltanet_chunk_fwd.  The scratch (the device status word) comes from a
- * static device array of 4096 bytes inside the library, one per device that
- * loads it, held until the process exits.  Nothing is allocated: no
+ * deltanet_chunk_fwd.  The scratch (the device status word and, for bf16
+ * inputs, the per-chunk factors of the chunked solve) comes from a static
+ * device array of 1 MiB inside the library, one per device that loads it,
+ * held until the process exits: enough for about 64 (b, h, 64-token chunk)
+ * units of bf16 work.  Nothing is allocated: no
  * cudaMalloc, cudaFree or allocating library routine is called.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with the caller's current device, which must be
@@ -191,8 +196,8 @@ int deltanet_selftest_wait_timeout(void *workspace, size_t ws_bytes, long long w
  *     (for instance on different streams) race on it.  The status word cannot
  *     be read back through this entry point; use deltanet_chunk_fwd with a
  *     caller-owned workspace when bounded-wait timeouts must be observed.
- *   - A problem whose workspace need (deltanet_workspace_bytes) exceeds 4096
- *     bytes is rejected with DN_ERR_WORKSPACE.
+ *   - A problem whose workspace need (deltanet_workspace_bytes) exceeds 1 MiB
+ *     is rejected with DN_ERR_WORKSPACE.
  */
 int deltanet_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                const float *beta, const float *alpha, const float *S0,

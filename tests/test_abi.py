@@ -75,8 +75,10 @@ MB = 1 << 20
 
 def _chunk(L, q=A, k=A + 64 * MB, v=A + 128 * MB, beta=A + 192 * MB, alpha=None, S0=None,
            o=A + 256 * MB, S_out=A + 320 * MB, B=2, H=2, T=100, Dk=64, Dv=64, C=64, dt=1,
-           ws=A + 400 * MB, ws_bytes=256):
+           ws=A + 400 * MB, ws_bytes=None):
     vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    if ws_bytes is None:
+        ws_bytes = max(256, L.deltanet_workspace_bytes(max(B, 0), max(H, 0), max(T, 0), 64, 64, 64, 1))
     return L.deltanet_chunk_fwd(vp(q), vp(k), vp(v), vp(beta), vp(alpha), vp(S0), vp(o),
                                 vp(S_out), B, H, T, Dk, Dv, C, dt, vp(ws), ws_bytes, None)
 
@@ -134,7 +136,7 @@ def test_linear_rejects_bad_arguments(L):
             S_out=None, z_out=None, Dk=64, C=64):
         f = lambda x: None if x is None else vp(x)
         return L.linear_attn_fwd(f(q), f(k), f(v), f(S0), f(z0), f(o), f(S_out), f(z_out),
-                                 2, 2, 100, Dk, 64, C, 1, vp(A + 400 * MB), 256, None)
+                                 2, 2, 100, Dk, 64, C, 1, vp(A + 400 * MB), 1 << 24, None)
 
     assert lin(v=None) == E.DN_ERR_INVALID_ARG
     assert lin(Dk=80) == E.DN_ERR_UNSUPPORTED

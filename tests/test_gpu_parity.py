@@ -223,7 +223,8 @@ def test_bounded_wait_times_out_cleanly(dn):
     """A wait nothing satisfies ends in DN_ERR_DEVICE_TIMEOUT read by the host, and the
     context keeps working afterwards."""
     dev = torch.device("cuda")
-    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(dn.lib().deltanet_workspace_bytes(1, 1, 64, 64, 64, 64, 1), dtype=torch.uint8,
+                     device=dev)
     assert dn.deltanet_selftest_wait_timeout(20_000_000, ws) == 0
     assert dn.deltanet_get_device_status(workspace=ws) == dn._lib.DN_ERR_DEVICE_TIMEOUT
     dn.reset_device_status(workspace=ws)
