@@ -14,13 +14,21 @@
 //   S <- gamma_last S + K^T (diag(Gamma_last,.) U)             (float32 registers)
 //
 // One CTA per (b, h, 64-column slice of Dv), 9 warps:
+//   warp 9     MMA issuer (one thread): every tcgen05.mma of the CTA, in a
+//              fixed order chosen so the shared tensor pipe never holds the
+//              state chain behind state-independent work:
+//                [Q;W]S (c), QK^T (c), K^T U (c), W/Uh (c+1), PU (c)
+//              (gated: QK^T (c+1) right after W/Uh (c+1) instead, so that Q
+//              can be scaled by gamma before [Q;W]S (c+1))
 //   warp 8     producer: TMA of K, Q, V, Tb, Tbg (+ beta and g rows) into a
 //              two-stage ring, L2 prefetch two chunks ahead
-//   warps 4-7  prep, one chunk ahead of the chain: the three S-independent
-//              MMAs, then P and W to bf16 shared memory (in parallel halves),
-//              diag(gamma) applied to Q in place
-//   warps 0-3  chain: [Q;W]S, U, PU + K^T U, the state update; warps 0-1 then
-//              drain the output tile while warps 2-3 start the next chunk
+//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead)
+//   warps 4-5  P rows to bf16; gated: Q <- diag(gamma) Q in place
+//   warps 2-3  U = Uh - WS;   warps 0-3 the state update;
+//   warps 0-1  drain the output tile O = gamma QS + PU
+// Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
+// signal back; the issuer waits on their signals.  Every mbarrier completes
+// once per chunk (or per use of a parity), so parity waits are unambiguous.
 // Accumulators live in TMEM (512 columns), every operand in the 128-byte-
 // swizzled canonical layout, the running state in float32 registers.  All
 // waits are bounded; a wait that runs out sets the workspace status word and
@@ -38,11 +46,13 @@ constexpr int kC = 64;
 constexpr int kDVS = 64;
 constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
 constexpr int kWG = 128;
-constexpr int kThreads = 2 * kWG + 32;
-constexpr int kBarChain = 1, kBarPrep = 2, kBarChainHi = 3, kBarChainLo = 4;
+constexpr int kThreads = 2 * kWG + 64;  // chain 0-3, prep 4-7, producer 8, issuer 9
+constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kBarPrepW = 5;
 
 // TMEM columns: G (P scores), W, Uh[2], QW[2] (lanes 0-63: O, lanes 64-127: WS), dS
-constexpr uint32_t TM_G = 0, TM_W = 64, TM_UH = 192, TM_QW = 320, TM_DS = 448;
+// Uh sits right after W (at TM_W + Dk) so that, ungated, one N = Dk + 64
+// product writes both.
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384;
 
 template <int DK>
 struct MainLayout {
@@ -60,15 +70,16 @@ struct MainLayout {
   static constexpr uint32_t S_OFF = UT_OFF + kTile;   // bf16 state, DK rows x 128 B
   static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // chain copy of g per parity: [2][64]
   static constexpr uint32_t BAR_OFF = CV_OFF + 2 * 64 * 4;
-  static constexpr uint32_t BYTES = BAR_OFF + 128;
+  static constexpr uint32_t BYTES = BAR_OFF + 192;
   static constexpr uint32_t ALLOC = BYTES + 1024;
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
-// mbarrier slots; each completes once per chunk (or once per use of a parity),
-// so every waiter is at most one phase behind and parity waits are unambiguous.
-constexpr uint32_t B_FULL = 0, B_EMPTY = 16, B_READY = 32, B_FREE = 48, B_PMMA = 64, B_CMMA3 = 72,
-                   B_CMMA4 = 80, B_FINP = 88, B_FINC = 96, B_TMEM = 104, B_ABORT = 108;
+// mbarrier slots (8 bytes each)
+// (FULL, EMPTY, OFREE, CMMA5 and PREADY come in pairs, one per chunk parity)
+constexpr uint32_t B_FULL = 0, B_EMPTY = 16, B_OFREE = 32, B_CMMA3 = 48, B_CMMA4 = 56, B_CMMA5 = 64,
+                   B_PMMA1 = 80, B_PMMA2 = 88, B_UREADY = 96, B_SREADY = 104, B_PREADY = 112,
+                   B_WREADY = 128, B_FIN = 136, B_TMEM = 144, B_ABORT = 148;
 
 __device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -84,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmTbg, const ChunkProblem p,
                       const float* __restrict__ gw) {
   using L = MainLayout<DK>;
+  constexpr uint32_t TM_UH = TM_W + DK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -102,14 +114,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's vector rows
       mbar_init(bar + B_EMPTY + 8 * i, 1);
-      mbar_init(bar + B_READY + 8 * i, 1);
-      mbar_init(bar + B_FREE + 8 * i, 1);
+      mbar_init(bar + B_OFREE + 8 * i, 1);
+      mbar_init(bar + B_CMMA5 + 8 * i, 1);
+      mbar_init(bar + B_PREADY + 8 * i, 1);
     }
-    mbar_init(bar + B_PMMA, 1);
     mbar_init(bar + B_CMMA3, 1);
     mbar_init(bar + B_CMMA4, 1);
-    mbar_init(bar + B_FINP, 1);
-    mbar_init(bar + B_FINC, 1);
+    mbar_init(bar + B_PMMA1, 1);
+    mbar_init(bar + B_PMMA2, 1);
+    mbar_init(bar + B_UREADY, 1);
+    mbar_init(bar + B_SREADY, 1);
+    mbar_init(bar + B_WREADY, GATED ? 2 : 1);  // W rows (+ gamma-scaled Q when gated)
+    mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -186,49 +202,163 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
         (void)mbar_wait(bar + B_FULL + 8 * (c & 1), (c >> 1) & 1, drain);
     }
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------------- prep --
-    const int pt = tid - kWG;
-    const int row = pt & 63;
-    bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      const int b = c & 1, use = c >> 1;
-      const uint32_t st = sb + b * L::STAGE;
-      uint8_t* stp = sm + b * L::STAGE;
-      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
-      if (c >= 2) {  // the chain is done with this parity's P, Uh and g copy
-        ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FREE + 8 * b, (use - 1) & 1, wc));
-        if (!ok) break;
-      }
-      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FULL + 8 * b, use & 1, wc));
-      if (!ok) break;
-
-      // ---- P scores = Q K^T (lanes 0-63), W (lanes 64-127), Uh (lanes 64-127) ----
-      if (pt == 0) {
-        tc_fence_after();
-        constexpr uint32_t idg = idesc_bf16(128, 64, false, false);
-        constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
-        constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+  } else if (warp == 9) {
+    // -------------------------------------------------------------- issuer --
+    if (lane == 0) {
+      auto stage = [&](int c) { return sb + (c & 1) * L::STAGE; };
+      // P scores = Q K^T of chunk c (lanes 0-63 of TM_G)
+      auto issue_qkt = [&](int c) {
+        const uint32_t st = stage(c);
+        constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
-          mma_bf16_ss(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), idg, ks > 0);
+          mma_bf16_ss(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
         }
-        const uint32_t aw = st + (GATED ? L::TB_OFF : L::V_OFF);  // rows 64-127: Tbg (Tb)
+      };
+      // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of TM_UH).
+      // Ungated both share the A operand Tb, and K's 64-column blocks and V sit
+      // KB_STRIDE apart, so [W | Uh] = Tb [K | V] is one N = Dk + 64 product.
+      auto issue_wu = [&](int c) {
+        const uint32_t st = stage(c);
+        if (!GATED) {
+          constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ss(tmem + TM_W, desc_k(aw + ks * 32),
-                      desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), idw, ks > 0);
-          mma_bf16_ss(tmem + TM_UH + 64 * b, desc_k(st + L::V_OFF + ks * 32),
-                      desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + TM_W, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
+                        desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), id, ks > 0);
+        } else {
+          constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
+          constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            mma_bf16_ss(tmem + TM_W, desc_k(st + L::TB_OFF + ks * 32),  // rows 64-127: Tbg
+                        desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), idw, ks > 0);
+            mma_bf16_ss(tmem + TM_UH, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
+                        desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
+          }
         }
-        mma_commit(bar + B_PMMA);
+      };
+      // [gamma Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
+      auto issue_qw = [&](int c) {
+        const uint32_t st = stage(c);
+        constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+          mma_bf16_ss(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
+                      id, ks > 0);
+        }
+      };
+      // dS = K^T U~
+      auto issue_ds = [&](int c) {
+        const uint32_t st = stage(c);
+        const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
+        constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                      desc_mn(ut + ks * 2048, kTile), id, ks > 0);
+      };
+      // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
+      auto issue_pu = [&](int c) {
+        const uint32_t pa = sb + L::P_OFF + (c & 1) * kTile;
+        constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32),
+                      desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
+      };
+      bool ok = mbar_wait(bar + B_FULL, 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_wu(0);
+        mma_commit(bar + B_PMMA2);
+        if (GATED) {
+          issue_qkt(0);
+          mma_commit(bar + B_PMMA1);
+        }
       }
-      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_PMMA, c & 1, wc));
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int b = c & 1;
+        const bool nxt = c + 1 < nchunks;
+        ok = mbar_wait(bar + B_WREADY, c & 1, wc) && mbar_wait(bar + B_SREADY, c & 1, wc) &&
+             (c < 2 || mbar_wait(bar + B_OFREE + 8 * b, ((c >> 1) - 1) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        issue_qw(c);
+        mma_commit(bar + B_CMMA3);
+        if (!GATED) {  // this chunk's scores: needed only by PU (c), run during the U epilogue
+          issue_qkt(c);
+          mma_commit(bar + B_PMMA1);
+        }
+        ok = mbar_wait(bar + B_UREADY, c & 1, wc);  // Uh (single buffer) has been consumed
+        if (!ok) break;
+        tc_fence_after();
+        issue_ds(c);
+        mma_commit(bar + B_CMMA4);
+        if (nxt) {
+          ok = mbar_wait(bar + B_FULL + 8 * (b ^ 1), ((c + 1) >> 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_wu(c + 1);
+          mma_commit(bar + B_PMMA2);
+          if (GATED) {
+            issue_qkt(c + 1);
+            mma_commit(bar + B_PMMA1);
+          }
+        }
+        ok = mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pu(c);
+        mma_commit(bar + B_CMMA5 + 8 * b);
+        mma_commit(bar + B_EMPTY + 8 * b);  // stage b: every reader (MMAs and P/Q epilogue) is done
+      }
+      tc_fence_after();  // no MMA may outlive TMEM
+      mma_commit(bar + B_FIN);
+      int zero = 0;
+      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
+      (void)mbar_wait(bar + B_FIN, 0, fin);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------- W rows (6-7) --
+    const int row = (tid - 192) & 63;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      uint8_t* stp = sm + (c & 1) * L::STAGE;
+      ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_PMMA2, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      if (pt < 64) {
-        // P row: tril(QK^T) * Gamma -> bf16 P[b]
+#pragma unroll
+      for (int q = 0; q < DK / 32; ++q) {
+        uint32_t w[32];
+        tmem_ld32(tmem + lane_base + TM_W + q * 32, w);
+        tmem_wait_ld();
+        uint8_t* wt = stp + (q >> 1) * L::KB_STRIDE + L::W_OFF;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarPrepW, 64);
+      if (tid == 192) mbar_arrive(bar + B_WREADY);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------- P rows, gamma Q (4-5) --
+    const int row = tid - 128;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int b = c & 1;
+      uint8_t* stp = sm + b * L::STAGE;
+      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
+      ok = named_bar_and(kBarPrepP, 64,
+                         mbar_wait(bar + B_FULL + 8 * b, (c >> 1) & 1, wc) &&
+                             mbar_wait(bar + B_PMMA1, c & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      {
         uint32_t g[64];
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
@@ -247,26 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           st_bf16x8(ptile + sw128_off(row, c16), x);
         }
-        if (GATED) cvec[b * 64 + row] = vs[64 + row];
-      } else {
-        // W row -> bf16 into the stage, right after Q
-#pragma unroll
-        for (int q = 0; q < DK / 32; ++q) {
-          uint32_t w[32];
-          tmem_ld32(tmem + lane_base + TM_W + q * 32, w);
-          tmem_wait_ld();
-          uint8_t* wt = stp + (q >> 1) * L::KB_STRIDE + L::W_OFF;
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
-        }
       }
-      if (GATED) {  // Q <- diag(gamma) Q in place (the scores above used the plain Q)
+      if (GATED) {
+        cvec[b * 64 + row] = vs[64 + row];
+        // Q <- diag(gamma) Q in place (the scores above used the plain Q)
         const float gam = __expf(vs[64 + row]);
-        const int h = pt >> 6;
 #pragma unroll
-        for (int i = 0; i < DK / 16; ++i) {
-          const int c16 = h * (DK / 16) + i;  // this thread's half of the row's 16-byte chunks
+        for (int c16 = 0; c16 < DK / 8; ++c16) {
           uint8_t* ptr = stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16 & 7);
           uint4 u = *reinterpret_cast<uint4*>(ptr);
           uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
@@ -280,15 +397,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(kBarPrep, kWG);
-      if (pt == 0) mbar_arrive(bar + B_READY + 8 * b);
-    }
-    if (pt == 0) {
-      tc_fence_after();
-      mma_commit(bar + B_FINP);
-      int zero = 0;
-      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
-      (void)mbar_wait(bar + B_FINP, 0, fin);
+      named_bar_sync(kBarPrepP, 64);
+      if (row == 0) {
+        mbar_arrive(bar + B_PREADY + 8 * b);
+        if (GATED) mbar_arrive(bar + B_WREADY);
+      }
     }
   } else {
     // --------------------------------------------------------------- chain --
@@ -308,110 +421,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     named_bar_sync(kBarChain, kWG);
+    if (ct == 0) mbar_arrive(bar + B_SREADY);  // the initial state tile is in place
 
-    bool ok = true;
+    bool ok = true, ok_hi = true, ok_lo = true;
     for (int c = 0; c < nchunks && ok; ++c) {
-      const int b = c & 1, use = c >> 1;
+      const int b = c & 1;
       const int c0 = c * kC, n = min(kC, T - c0);
-      const uint32_t st = sb + b * L::STAGE;
       const uint32_t qw = tmem + TM_QW + 64 * b;
-      bool ok2 = true;
+      const float* vb = cvec + b * 64;
       if (ct >= 64) {
-        // warps 2-3: [Q;W] S, then U, then issue PU and K^T U
-        ok2 = named_bar_and(kBarChainHi, 64, mbar_wait(bar + B_READY + 8 * b, use & 1, wc));
-        if (ok2) {
-          if (ct == 64) {
-            tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 64, false, true);
-#pragma unroll
-            for (int ks = 0; ks < DK / 16; ++ks) {
-              const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-              mma_bf16_ss(qw, desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile), id, ks > 0);
-            }
-            mma_commit(bar + B_CMMA3);
-          }
-          ok2 = named_bar_and(kBarChainHi, 64, mbar_wait(bar + B_CMMA3, c & 1, wc));
-        }
-        if (ok2) {
+        // ---- U = Uh - WS (rows on lanes 64-127) ----
+        ok_hi = named_bar_and(kBarChainHi, 64, mbar_wait(bar + B_CMMA3, c & 1, wc));
+        if (ok_hi) {
           tc_fence_after();
-          const float wl = GATED ? __expf(cvec[b * 64 + n - 1] - cvec[b * 64 + row]) : 1.f;
+          const float wl = GATED ? __expf(vb[n - 1] - vb[row]) : 1.f;
+          uint32_t ws[64], uh[64];
+          tmem_ld32(qw + lane_base, *reinterpret_cast<uint32_t(*)[32]>(ws));
+          tmem_ld32(qw + lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(ws + 32));
+          tmem_ld32(tmem + lane_base + TM_UH, *reinterpret_cast<uint32_t(*)[32]>(uh));
+          tmem_ld32(tmem + lane_base + TM_UH + 32, *reinterpret_cast<uint32_t(*)[32]>(uh + 32));
+          tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t ws[32], uh[32];
-            tmem_ld32(qw + lane_base + q * 32, ws);
-            tmem_ld32(tmem + lane_base + TM_UH + 64 * b + q * 32, uh);
-            tmem_wait_ld();
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8], y[8];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              float x[8], y[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                x[e] = __uint_as_float(uh[cc * 8 + e]) - __uint_as_float(ws[cc * 8 + e]);
-                y[e] = x[e] * wl;
-              }
-              st_bf16x8(sm + L::U_OFF + sw128_off(row, q * 4 + cc), x);
-              if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(row, q * 4 + cc), y);
+            for (int e = 0; e < 8; ++e) {
+              x[e] = __uint_as_float(uh[c16 * 8 + e]) - __uint_as_float(ws[c16 * 8 + e]);
+              y[e] = x[e] * wl;
             }
+            st_bf16x8(sm + L::U_OFF + sw128_off(row, c16), x);
+            if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(row, c16), y);
           }
           fence_proxy_async_smem();
           tc_fence_before();
           named_bar_sync(kBarChainHi, 64);
-          if (ct == 64) {
-            tc_fence_after();
-            const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
-            const uint32_t pa = sb + L::P_OFF + b * kTile;
-            constexpr uint32_t idp = idesc_bf16(128, 64, false, true);
-            constexpr uint32_t ids = idesc_bf16(128, 64, true, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              mma_bf16_ss(qw, desc_k(pa + ks * 32), desc_mn(sb + L::U_OFF + ks * 2048, kTile), idp, 1);
-              mma_bf16_ss(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                          desc_mn(ut + ks * 2048, kTile), ids, ks > 0);
-            }
-            mma_commit(bar + B_CMMA4);
-            mma_commit(bar + B_EMPTY + 8 * b);  // the stage may be refilled
-          }
+          if (ct == 64) mbar_arrive(bar + B_UREADY);
         }
       }
-      ok = named_bar_and(kBarChain, kWG, ok2 && mbar_wait(bar + B_CMMA4, c & 1, wc));
+      ok = named_bar_and(kBarChain, kWG, ok_hi && ok_lo && mbar_wait(bar + B_CMMA4, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
 
-      // ---- state update (all lanes 0..DK-1), then release the next [Q;W]S ----
+      // ---- state update (lanes 0..DK-1) ----
       if (ct < DK) {
-        const float carry = GATED ? __expf(cvec[b * 64 + n - 1]) : 1.f;
+        const float carry = GATED ? __expf(vb[n - 1]) : 1.f;
+        uint32_t ds[64];
+        tmem_ld32(tmem + lane_base + TM_DS, *reinterpret_cast<uint32_t(*)[32]>(ds));
+        tmem_ld32(tmem + lane_base + TM_DS + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t ds[32];
-          tmem_ld32(tmem + lane_base + TM_DS + q * 32, ds);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sreg[q * 32 + e] = fmaf(carry, sreg[q * 32 + e], __uint_as_float(ds[e]));
-        }
+        for (int e = 0; e < 64; ++e) sreg[e] = fmaf(carry, sreg[e], __uint_as_float(ds[e]));
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarChain, kWG);
+      if (ct == 0) mbar_arrive(bar + B_SREADY);
 
       // ---- outputs O = gamma QS + PU (lanes 0-63), drained by warps 0-1 ----
       if (ct < 64) {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + row) * Dv + j0;
+        ok_lo = named_bar_and(kBarChainLo, 64, mbar_wait(bar + B_CMMA5 + 8 * b, (c >> 1) & 1, wc));
+        if (ok_lo) {
+          tc_fence_after();
+          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + row) * Dv + j0;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t ov[32];
-          tmem_ld32(qw + lane_base + q * 32, ov);
-          tmem_wait_ld();
-          if (row < n) {
+          for (int q = 0; q < 2; ++q) {
+            uint32_t ov[32];
+            tmem_ld32(qw + lane_base + q * 32, ov);
+            tmem_wait_ld();
+            if (row < n) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              st_bf16x8(orow + q * 32 + cc * 8, reinterpret_cast<const float*>(ov) + cc * 8);
+              for (int cc = 0; cc < 4; ++cc)
+                st_bf16x8(orow + q * 32 + cc * 8, reinterpret_cast<const float*>(ov) + cc * 8);
+            }
           }
+          tc_fence_before();
+          named_bar_sync(kBarChainLo, 64);
+          if (ct == 0) mbar_arrive(bar + B_OFREE + 8 * b);
         }
-        tc_fence_before();
-        named_bar_sync(kBarChainLo, 64);
-        if (ct == 0) mbar_arrive(bar + B_FREE + 8 * b);
       }
     }
     if (p.S_out && ct < DK) {
@@ -419,13 +507,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kDVS; j += 4)
         *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
-    }
-    if (ct == 64) {
-      tc_fence_after();
-      mma_commit(bar + B_FINC);
-      int zero = 0;
-      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
-      (void)mbar_wait(bar + B_FINC, 0, fin);
     }
   }
 

@@ -16,8 +16,8 @@
 //   3. A = mask / scale G in place.
 //   4. Four 16x16 diagonal inverses (one column per lane, right-looking
 //      substitution so only one multiply-add per step is on the dependency
-//      chain), then tf32 WMMA merges 16 -> 32 -> 64:
-//      T_ij = -T_ii A_ij T_jj,  T21 = -T22 A21 T11.
+//      chain), then each warp finishes one 16-column block of T by block
+//      forward substitution with tf32 WMMA products, T_iw = -D_i sum A_im T_mw.
 //   5. Tb, Tbg -> global (row-major bf16, 8 KB per tile).
 #include <cuda_bf16.h>
 #include <mma.h>
@@ -42,7 +42,7 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
 }
 
 template <int DK, bool GATED>
-__global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
                                                           const float* __restrict__ beta,
                                                           const float* __restrict__ alpha,
                                                           __nv_bfloat16* __restrict__ tb_out,
@@ -50,11 +50,12 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
                                                           float* __restrict__ g_out, int T,
                                                           int nchunks) {
   constexpr int KS = DK + kKpad;
+  constexpr int kRegion = (kC * KS * 2 > kC * kApad * 4) ? kC * KS * 2 : kC * kApad * 4;
   extern __shared__ __align__(128) uint8_t tsolve_smem[];
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(tsolve_smem);
-  float* Am = reinterpret_cast<float*>(tsolve_smem + kC * KS * 2);
-  float* Tm = Am + kC * kApad;
-  float* vb = Tm + kC * kApad;
+  float* Tm = reinterpret_cast<float*>(tsolve_smem);  // reuses the K tile after the Gram
+  float* Am = reinterpret_cast<float*>(tsolve_smem + kRegion);
+  float* vb = Am + kC * kApad;
   float* vg = vb + 64;
   float* veg = vg + 64;
 
@@ -93,15 +94,10 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
         g_out[((size_t)bh * nchunks + chunk) * kC + tid] = x;
       }
     }
-    // T's strictly-upper 16x16 blocks are read by the merges and must be zero
-    for (int i = tid; i < 64 * 64; i += kThreads) {
-      const int r = i >> 6, c = i & 63;
-      if ((c >> 4) > (r >> 4)) Tm[r * kApad + c] = 0.f;
-    }
   }
   __syncthreads();
 
-  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps)
+  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps), straight into A
   {
     wmma::fragment<wmma::matrix_a, 16, 16, 16, __nv_bfloat16, wmma::row_major> fa;
     wmma::fragment<wmma::matrix_b, 16, 16, 16, __nv_bfloat16, wmma::col_major> fb;
@@ -122,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
   }
   __syncthreads();
 
-  // 3. A = strict_lower(diag(beta) G * Gamma) in place; the upper part is zeroed
+  // 3. A = strict_lower(diag(beta) G * Gamma) in place; T's strictly-upper blocks = 0
   for (int i = tid; i < 64 * 64; i += kThreads) {
     const int r = i >> 6, s = i & 63;
     float a = 0.f;
@@ -131,10 +127,13 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
       if (GATED) a *= __expf(vg[r] - vg[s]);
     }
     Am[r * kApad + s] = a;
+    if ((s >> 4) > (r >> 4)) Tm[r * kApad + s] = 0.f;
   }
   __syncthreads();
 
-  // 4a. diagonal 16x16 inverses: warp w, lanes 0-15 own column j of block w
+  // 4. T = (I + A)^-1.  Diagonal 16x16 blocks D_w: warp w, lanes 0-15 own
+  //    column j; right-looking, so only one multiply-add per step is on the
+  //    dependency chain.
   if (lane < 16) {
     const int o = 16 * warp, j = lane;
     float col[16], acc[16];
@@ -143,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
       col[i] = 0.f;
       acc[i] = 0.f;
     }
-    // right-looking: once col[m] is final, fold it into every later row
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       col[m] = (m == j) ? 1.f : (m > j ? -acc[m] : 0.f);
@@ -154,67 +152,41 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
     for (int i = 0; i < 16; ++i) Tm[(o + i) * kApad + o + j] = col[i];
   }
   __syncthreads();
-  // 4b. T_{r,r-1} = -D_r A_{r,r-1} D_{r-1}, r = 1 (warp 0) and r = 3 (warp 2)
-  if ((warp & 1) == 0) {
-    const int o = 16 * (warp + 1), q0 = o - 16;
-    float* ys = Am + (warp == 0 ? 0 : 16) * kApad + 48;  // scratch in A's zero upper part
-    wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
-    wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
-    wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
-    wmma::fill_fragment(acc, 0.f);
-#pragma unroll
-    for (int kk = 0; kk < 16; kk += 8) {
-      wmma::load_matrix_sync(fa, Am + o * kApad + q0 + kk, kApad);
-      wmma::load_matrix_sync(fb, Tm + (q0 + kk) * kApad + q0, kApad);
-      to_tf32(fa);
-      to_tf32(fb);
-      wmma::mma_sync(acc, fa, fb, acc);
-    }
-    wmma::store_matrix_sync(ys, acc, kApad, wmma::mem_row_major);
-    __syncwarp();
-    wmma::fill_fragment(acc, 0.f);
-#pragma unroll
-    for (int kk = 0; kk < 16; kk += 8) {
-      wmma::load_matrix_sync(fa, Tm + o * kApad + o + kk, kApad);
-      wmma::load_matrix_sync(fb, ys + kk * kApad, kApad);
-      to_tf32(fa);
-      to_tf32(fb);
-      wmma::mma_sync(acc, fa, fb, acc);
-    }
-#pragma unroll
-    for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
-    wmma::store_matrix_sync(Tm + o * kApad + q0, acc, kApad, wmma::mem_row_major);
-  }
-  __syncthreads();
-  // 4c. Y = A21 T11, then T21 = -T22 Y (one 16x16 tile per warp)
+  //    Column block w (warp w) by block forward substitution:
+  //    T_iw = -D_i sum_{m=w}^{i-1} A_im T_mw  for i > w   (tf32 products)
   {
-    const int ti = warp >> 1, tj = warp & 1;
     wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
     wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
     wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
-    wmma::fill_fragment(acc, 0.f);
+    float* xs = Am + (16 * warp) * kApad + 48;  // 16x16 scratch in A's zero upper part
+    for (int i = warp + 1; i < 4; ++i) {
+      wmma::fill_fragment(acc, 0.f);
+      for (int m = warp; m < i; ++m) {
 #pragma unroll
-    for (int kk = 0; kk < 32; kk += 8) {
-      wmma::load_matrix_sync(fa, Am + (32 + 16 * ti) * kApad + kk, kApad);
-      wmma::load_matrix_sync(fb, Tm + kk * kApad + 16 * tj, kApad);
-      to_tf32(fa);
-      to_tf32(fb);
-      wmma::mma_sync(acc, fa, fb, acc);
+        for (int kk = 0; kk < 16; kk += 8) {
+          wmma::load_matrix_sync(fa, Am + (16 * i) * kApad + 16 * m + kk, kApad);
+          wmma::load_matrix_sync(fb, Tm + (16 * m + kk) * kApad + 16 * warp, kApad);
+          to_tf32(fa);
+          to_tf32(fb);
+          wmma::mma_sync(acc, fa, fb, acc);
+        }
+      }
+      wmma::store_matrix_sync(xs, acc, kApad, wmma::mem_row_major);
+      __syncwarp();
+      wmma::fill_fragment(acc, 0.f);
+#pragma unroll
+      for (int kk = 0; kk < 16; kk += 8) {
+        wmma::load_matrix_sync(fa, Tm + (16 * i) * kApad + 16 * i + kk, kApad);
+        wmma::load_matrix_sync(fb, xs + kk * kApad, kApad);
+        to_tf32(fa);
+        to_tf32(fb);
+        wmma::mma_sync(acc, fa, fb, acc);
+      }
+#pragma unroll
+      for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
+      wmma::store_matrix_sync(Tm + (16 * i) * kApad + 16 * warp, acc, kApad, wmma::mem_row_major);
+      __syncwarp();
     }
-    wmma::store_matrix_sync(Am + (16 * ti) * kApad + 32 + 16 * tj, acc, kApad, wmma::mem_row_major);
-    __syncthreads();
-    wmma::fill_fragment(acc, 0.f);
-#pragma unroll
-    for (int kk = 0; kk < 32; kk += 8) {
-      wmma::load_matrix_sync(fa, Tm + (32 + 16 * ti) * kApad + 32 + kk, kApad);
-      wmma::load_matrix_sync(fb, Am + kk * kApad + 32 + 16 * tj, kApad);
-      to_tf32(fa);
-      to_tf32(fb);
-      wmma::mma_sync(acc, fa, fb, acc);
-    }
-#pragma unroll
-    for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
-    wmma::store_matrix_sync(Tm + (32 + 16 * ti) * kApad + 16 * tj, acc, kApad, wmma::mem_row_major);
   }
   __syncthreads();
 
@@ -243,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 4) tsolve_kernel(const __nv_bfloat16
 template <int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   const int nchunks = (p.T + kC - 1) / kC;
-  constexpr size_t smem = (size_t)kC * (DK + kKpad) * 2 + 2 * (size_t)kC * kApad * 4 + 3 * 64 * 4;
+  constexpr size_t kKbytes = (size_t)kC * (DK + kKpad) * 2, kTbytes = (size_t)kC * kApad * 4;
+  constexpr size_t smem = (kKbytes > kTbytes ? kKbytes : kTbytes) + kTbytes + 3 * 64 * 4;
   auto kern = tsolve_kernel<DK, GATED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
