@@ -3,8 +3,8 @@
 
 Headline: the chunked DeltaNet forward on the prefill workload (B4 H16 T4096,
 Dk = Dv = 128, bf16 q/k/v, fp32 beta and state, C = 64, S0 = 0), tokens/s over
-all GPUs.  One step = one deltanet_chunk_fwd call over one batch (one launch
-of the chunk kernel).  Inputs are resident in HBM when the timed region starts;
+all GPUs.  One step = one deltanet_chunk_fwd call over one batch (two
+launches: the chunk-parallel WY pre-pass and the chunk kernel).  Inputs are resident in HBM when the timed region starts;
 two input sets alternate so consecutive steps touch disjoint 274 MB working
 sets (larger than the 126 MB L2).
 
@@ -178,6 +178,18 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def input_seeds(rank: int, nsets: int = 2):
+    """Seeds of the input sets a rank draws: every rank owns an independent
+    batch (weak scaling), so no two ranks share a seed."""
+    return [rank * nsets + i for i in range(nsets)]
+
+
+def whole_job_rate(world: int, units_per_rank: int, steps: int, ms_max: float) -> float:
+    """Units per second over all ranks: every rank processes ``units_per_rank``
+    per step, and the job takes the slowest rank's time (``ms_max``)."""
+    return world * units_per_rank * steps / (ms_max * 1e-3)
+
+
 def time_region(step, K, W, world, stream, sampler=None):
     """W warm-up steps, then exactly K timed steps bracketed by barrier + sync.
     Returns milliseconds (max over ranks) and the clock summary."""
@@ -208,9 +220,15 @@ class _Null:
         return False
 
 
+PROFILE_SUMMARY = "chunk_main_kernel_prefill_B4H16T4096D128.md"
+CHUNK_SOURCES = ("tsolve.cu", "chunk_main.cu", "common.cuh")
+LAUNCHES_PER_CALL = 2  # tsolve_kernel (WY pre-pass) + chunk_main_kernel
+
+
 def kernel_hash():
+    """Hash of the sources of the two kernels one deltanet_chunk_fwd call runs."""
     h = hashlib.sha256()
-    for fn in ("chunk_tc.cu", "common.cuh"):
+    for fn in CHUNK_SOURCES:
         p = os.path.join(ROOT, "deltanet_sequence_mixing_b200", "csrc", fn)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -218,9 +236,9 @@ def kernel_hash():
 
 
 def traffic_from_profile():
-    """DRAM bytes per launch of the chunk kernel from the committed ncu summary,
-    or None if it was taken on a different kernel source."""
-    p = os.path.join(ROOT, "profiles", "chunk_tc_kernel_prefill_B4H16T4096D128.md")
+    """DRAM bytes of one deltanet_chunk_fwd call (pre-pass + chunk kernel) from
+    the committed ncu summary, or None if it was taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", PROFILE_SUMMARY)
     if not os.path.exists(p):
         return None
     vals = {}
@@ -464,7 +482,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
     w = gen.PREFILL
-    sets = [gen.make_workload(w, seed=rank * 2 + i, device=dev) for i in range(2)]
+    sets = [gen.make_workload(w, seed=sd, device=dev) for sd in input_seeds(rank)]
     o = [torch.empty_like(s["v"]) for s in sets]
     S = [torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev) for _ in sets]
     ws = dn.workspace_for(dev, dn.lib().deltanet_workspace_bytes(w.B, w.H, w.T, w.Dk, w.Dv, w.C, 1))
@@ -482,7 +500,7 @@ def main():
         raise RuntimeError(f"device status {status} after the timed region")
     ms_step = ms / args.steps
     tokens = w.B * w.H * w.T
-    value = world * tokens * args.steps / (ms * 1e-3)
+    value = whole_job_rate(world, tokens, args.steps, ms)
 
     flop, byts = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
     achieved = byts / (ms_step * 1e-3) / 1e9
@@ -511,7 +529,7 @@ def main():
     e2e_ms = time_region(e2e_step, args.e2e_steps, 3, world, stream)
     h2d = sum(hx[k_].numel() * hx[k_].element_size() for k_ in ("q", "k", "v", "beta"))
     d2h = ho.numel() * ho.element_size() + hS.numel() * 4
-    e2e = {"value": world * tokens * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+    e2e = {"value": whole_job_rate(world, tokens, args.e2e_steps, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": e2e_ms / args.e2e_steps}
     del hx, ho, hS
@@ -538,7 +556,7 @@ def main():
                        "C": w.C, "state": "fp32", "per_gpu": "independent batch per GPU",
                        "parallelism": f"dp{world}",
                        "l2": "inputs larger than L2: two alternating input sets of 274 MB each"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * args.steps,
             "clocks": sampler.summary(), "extras": extras,
         }
         print(json.dumps(line), flush=True)

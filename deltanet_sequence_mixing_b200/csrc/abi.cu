@@ -94,7 +94,7 @@ int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
         dn::chunk_main_carve(static_cast<uint8_t*>(ws) + kStatusBytes, p.B, p.H, p.T);
     return map_cuda(dn::launch_chunk_main(p, w, st));
   }
-  if (dn::chunk_tc_supported(p)) return map_cuda(dn::launch_chunk_tc(p, st));
+  if (dn::linear_tc_supported(p)) return map_cuda(dn::launch_linear_tc(p, st));
   if (dn::chunk_simt_supported(p.Dk, p.Dv, p.C)) return map_cuda(dn::launch_chunk_simt(p, st));
   return DN_ERR_UNSUPPORTED;
 }

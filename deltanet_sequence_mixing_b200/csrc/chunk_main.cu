@@ -15,13 +15,14 @@
 //
 // One CTA per (b, h, 64-column slice of Dv), 9 warps:
 //   warp 9     MMA issuer (one thread): every tcgen05.mma of the CTA, in a
-//              fixed order chosen so the shared tensor pipe never holds the
-//              state chain behind state-independent work:
-//                [Q;W]S (c), QK^T (c), K^T U (c), W/Uh (c+1), PU (c)
-//              (gated: QK^T (c+1) right after W/Uh (c+1) instead, so that Q
-//              can be scaled by gamma before [Q;W]S (c+1))
-//   warp 8     producer: TMA of K, Q, V, Tb, Tbg (+ beta and g rows) into a
-//              two-stage ring, L2 prefetch two chunks ahead
+//              fixed order that keeps the state chain fed:
+//                [Q;W]S (c), W/Uh (c+1), QK^T (c+1), K^T U (c), PU (c)
+//              W/Uh (c+1) and QK^T (c+1) run while the U epilogue of chunk c
+//              drains (Uh is double-buffered in TMEM), so W (c+1) and the
+//              scores of chunk c+1 are ready before the state update of
+//              chunk c ends and only PU (c) shares the pipe with it.
+//   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
+//              a three-stage ring (gated: two), L2 prefetch two chunks ahead
 //   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead)
 //   warps 4-5  P rows to bf16; gated: Q <- diag(gamma) Q in place
 //   warps 2-3  U = Uh - WS;   warps 0-3 the state update;
@@ -49,37 +50,47 @@ constexpr int kWG = 128;
 constexpr int kThreads = 2 * kWG + 64;  // chain 0-3, prep 4-7, producer 8, issuer 9
 constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kBarPrepW = 5;
 
-// TMEM columns: G (P scores), W, Uh[2], QW[2] (lanes 0-63: O, lanes 64-127: WS), dS
-// Uh sits right after W (at TM_W + Dk) so that, ungated, one N = Dk + 64
-// product writes both.
-constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384;
+// TMEM columns: G (P scores), W, Uh[0], QW[2] (lanes 0-63: O, lanes 64-127: WS),
+// dS, Uh[1].  Uh[0] sits right after W (at TM_W + Dk) so that, ungated and for
+// even chunks, one N = Dk + 64 product writes both.
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384, TM_UH1 = 448;
 
-template <int DK>
+// Shared memory.  A stage holds one chunk's TMA tiles [K | Q | W] per 64
+// columns of Dk, V, Tb (gated also Tbg and the beta / g rows); W is written
+// there by the W warps, right after Q, so that [Q; W] is one M = 128 operand.
+// Ungated runs a three-stage ring (the chunk after next streams in while one
+// chunk is on the state chain and the next is being prepared) with a single
+// P tile; gated needs the Tbg tile, the decay-weighted U and the g rows, and
+// fits two stages and two P tiles.
+template <int DK, bool GATED>
 struct MainLayout {
   static constexpr int KB = DK / 64;
-  static constexpr uint32_t KB_STRIDE = 3 * kTile;  // [K | Q | W] per 64 columns of Dk
+  static constexpr int NST = GATED ? 2 : 3;           // ring stages
+  static constexpr int NP = GATED ? 2 : 1;            // P tiles
+  static constexpr uint32_t KB_STRIDE = 3 * kTile;    // [K | Q | W] per 64 columns of Dk
   static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
-  static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | Tbg | beta, g
+  static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | (Tbg | beta, g)
   static constexpr uint32_t TB_OFF = V_OFF + kTile;
   static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
   static constexpr uint32_t VEC_OFF = TBG_OFF + kTile;
-  static constexpr uint32_t STAGE = VEC_OFF + 1024;
-  static constexpr uint32_t P_OFF = 2 * STAGE;        // P[0] | P[1] | U | UT
-  static constexpr uint32_t U_OFF = P_OFF + 2 * kTile;
+  static constexpr uint32_t STAGE = GATED ? VEC_OFF + 1024 : TBG_OFF;
+  static constexpr uint32_t P_OFF = NST * STAGE;      // P[NP] | U | (UT)
+  static constexpr uint32_t U_OFF = P_OFF + NP * kTile;
   static constexpr uint32_t UT_OFF = U_OFF + kTile;
-  static constexpr uint32_t S_OFF = UT_OFF + kTile;   // bf16 state, DK rows x 128 B
-  static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // chain copy of g per parity: [2][64]
-  static constexpr uint32_t BAR_OFF = CV_OFF + 2 * 64 * 4;
-  static constexpr uint32_t BYTES = BAR_OFF + 192;
+  static constexpr uint32_t S_OFF = U_OFF + (GATED ? 2 : 1) * kTile;  // bf16 state, DK rows x 128 B
+  static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // gated: chain copy of g per parity, [2][64]
+  static constexpr uint32_t BAR_OFF = CV_OFF + (GATED ? 2 * 64 * 4 : 0);
+  static constexpr uint32_t BYTES = BAR_OFF + 256;
   static constexpr uint32_t ALLOC = BYTES + 1024;
+  static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle atoms)");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
-// mbarrier slots (8 bytes each)
-// (FULL, EMPTY, OFREE, CMMA5 and PREADY come in pairs, one per chunk parity)
-constexpr uint32_t B_FULL = 0, B_EMPTY = 16, B_OFREE = 32, B_CMMA3 = 48, B_CMMA4 = 56, B_CMMA5 = 64,
-                   B_PMMA1 = 80, B_PMMA2 = 88, B_UREADY = 96, B_SREADY = 104, B_PREADY = 112,
-                   B_WREADY = 128, B_FIN = 136, B_TMEM = 144, B_ABORT = 148;
+// mbarrier slots (8 bytes each).  FULL and EMPTY: one per ring stage;
+// OFREE, CMMA5 and PREADY: one per chunk parity.
+constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
+                   B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
+                   B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164;
 
 __device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -94,8 +105,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
                       const __grid_constant__ CUtensorMap tmTbg, const ChunkProblem p,
                       const float* __restrict__ gw) {
-  using L = MainLayout<DK>;
-  constexpr uint32_t TM_UH = TM_W + DK;
+  using L = MainLayout<DK, GATED>;
+  constexpr int NST = L::NST;
+  constexpr uint32_t TM_UH0 = TM_W + DK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -111,9 +123,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* cvec = reinterpret_cast<float*>(sm + L::CV_OFF);
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's vector rows
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's arrival (after the g rows)
       mbar_init(bar + B_EMPTY + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar + B_OFREE + 8 * i, 1);
       mbar_init(bar + B_CMMA5 + 8 * i, 1);
       mbar_init(bar + B_PREADY + 8 * i, 1);
@@ -152,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int issued = 0;
     for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1, use = c >> 1;
+      const int s = c % NST, use = c / NST;
       const int c0 = c * kC, n = min(kC, T - c0);
       bool ok = true;
       if (lane == 0 && use > 0) ok = mbar_wait(bar + B_EMPTY + 8 * s, (use - 1) & 1, wc);
@@ -170,15 +184,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(st + L::TB_OFF, &tmTb, full, 0, c0, bh);
         if (GATED) tma_load_3d(st + L::TBG_OFF, &tmTbg, full, 0, c0, bh);
       }
-      // beta and g rows of the chunk (rows >= n: beta 0, g flat)
-      float* vs = reinterpret_cast<float*>(sm + s * L::STAGE + L::VEC_OFF);
-      const size_t tb = (size_t)bh * T + c0;
+      if (GATED) {  // g rows of the chunk (rows >= n: g flat); beta is folded into Tb
+        float* vs = reinterpret_cast<float*>(sm + s * L::STAGE + L::VEC_OFF);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = lane + 32 * h;
-        vs[r] = r < n ? p.beta[tb + r] : 0.f;
-        if (GATED) vs[64 + r] = gw[((size_t)bh * nchunks + c) * kC + r];
+        for (int h = 0; h < 2; ++h) vs[64 + lane + 32 * h] = gw[((size_t)bh * nchunks + c) * kC + lane + 32 * h];
       }
+      (void)n;
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(full);
@@ -199,13 +210,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // never leave with copies in flight
       int zero = 0;
       const WaitCtl drain{&zero, p.status, kWaitLimitNs};
-      for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-        (void)mbar_wait(bar + B_FULL + 8 * (c & 1), (c >> 1) & 1, drain);
+      for (int c = issued > NST ? issued - NST : 0; c < issued; ++c)
+        (void)mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, drain);
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- issuer --
     if (lane == 0) {
-      auto stage = [&](int c) { return sb + (c & 1) * L::STAGE; };
+      auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
       // P scores = Q K^T of chunk c (lanes 0-63 of TM_G)
       auto issue_qkt = [&](int c) {
         const uint32_t st = stage(c);
@@ -216,12 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
         }
       };
-      // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of TM_UH).
+      // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of Uh[c & 1]).
       // Ungated both share the A operand Tb, and K's 64-column blocks and V sit
-      // KB_STRIDE apart, so [W | Uh] = Tb [K | V] is one N = Dk + 64 product.
+      // KB_STRIDE apart, so for even chunks [W | Uh[0]] = Tb [K | V] is one
+      // N = Dk + 64 product.
       auto issue_wu = [&](int c) {
         const uint32_t st = stage(c);
-        if (!GATED) {
+        if (!GATED && (c & 1) == 0) {
           constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
@@ -230,11 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
           constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+          // rows 64-127 of the A operand: Tbg (gated) or Tb
+          const uint32_t wa = st + (GATED ? L::TB_OFF : L::V_OFF);
+          const uint32_t uh = (c & 1) ? TM_UH1 : TM_UH0;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            mma_bf16_ss(tmem + TM_W, desc_k(st + L::TB_OFF + ks * 32),  // rows 64-127: Tbg
-                        desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), idw, ks > 0);
-            mma_bf16_ss(tmem + TM_UH, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
+            mma_bf16_ss(tmem + TM_W, desc_k(wa + ks * 32), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                        idw, ks > 0);
+            mma_bf16_ss(tmem + uh, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
                         desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
           }
         }
@@ -262,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
       auto issue_pu = [&](int c) {
-        const uint32_t pa = sb + L::P_OFF + (c & 1) * kTile;
+        const uint32_t pa = sb + L::P_OFF + (GATED ? (c & 1) : 0) * kTile;
         constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -274,10 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_wu(0);
         mma_commit(bar + B_PMMA2);
-        if (GATED) {
-          issue_qkt(0);
-          mma_commit(bar + B_PMMA1);
-        }
+        issue_qkt(0);
+        mma_commit(bar + B_PMMA1);
       }
       for (int c = 0; c < nchunks && ok; ++c) {
         const int b = c & 1;
@@ -288,32 +301,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_qw(c);
         mma_commit(bar + B_CMMA3);
-        if (!GATED) {  // this chunk's scores: needed only by PU (c), run during the U epilogue
-          issue_qkt(c);
-          mma_commit(bar + B_PMMA1);
-        }
-        ok = mbar_wait(bar + B_UREADY, c & 1, wc);  // Uh (single buffer) has been consumed
-        if (!ok) break;
-        tc_fence_after();
-        issue_ds(c);
-        mma_commit(bar + B_CMMA4);
-        if (nxt) {
-          ok = mbar_wait(bar + B_FULL + 8 * (b ^ 1), ((c + 1) >> 1) & 1, wc);
+        if (nxt) {  // W (c) is already in shared memory and Uh[(c+1) & 1] was consumed by chunk c-1
+          ok = mbar_wait(bar + B_FULL + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           issue_wu(c + 1);
           mma_commit(bar + B_PMMA2);
-          if (GATED) {
-            issue_qkt(c + 1);
-            mma_commit(bar + B_PMMA1);
-          }
         }
+        // QK^T (c+1) once the scores of chunk c have left TMEM (P_READY); it
+        // runs while the U epilogue of chunk c drains
         ok = mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc);
         if (!ok) break;
+        if (nxt) {
+          tc_fence_after();
+          issue_qkt(c + 1);
+          mma_commit(bar + B_PMMA1);
+        }
+        ok = mbar_wait(bar + B_UREADY, c & 1, wc);
+        if (!ok) break;
         tc_fence_after();
+        issue_ds(c);
+        mma_commit(bar + B_CMMA4);
+        // K^T U (c) was the last reader of stage c: the P / Q / W epilogues of
+        // chunk c are done (W_READY, and gated P_READY, came before it)
+        mma_commit(bar + B_EMPTY + 8 * (c % NST));
         issue_pu(c);
         mma_commit(bar + B_CMMA5 + 8 * b);
-        mma_commit(bar + B_EMPTY + 8 * b);  // stage b: every reader (MMAs and P/Q epilogue) is done
       }
       tc_fence_after();  // no MMA may outlive TMEM
       mma_commit(bar + B_FIN);
@@ -326,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = (tid - 192) & 63;
     bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
-      uint8_t* stp = sm + (c & 1) * L::STAGE;
+      uint8_t* stp = sm + (c % NST) * L::STAGE;
       ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_PMMA2, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
@@ -351,10 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
       const int b = c & 1;
-      uint8_t* stp = sm + b * L::STAGE;
-      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
+      uint8_t* stp = sm + (c % NST) * L::STAGE;
+      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);  // gated only
       ok = named_bar_and(kBarPrepP, 64,
-                         mbar_wait(bar + B_FULL + 8 * b, (c >> 1) & 1, wc) &&
+                         mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc) &&
                              mbar_wait(bar + B_PMMA1, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
@@ -363,8 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
         tmem_wait_ld();
+        if (!GATED && c > 0) {  // the single P tile: PU (c-1) must have read it
+          ok = named_bar_and(kBarPrepP, 64,
+                             mbar_wait(bar + B_CMMA5 + 8 * ((c - 1) & 1), ((c - 1) >> 1) & 1, wc));
+          if (!ok) break;
+        }
         const float gr = GATED ? vs[64 + row] : 0.f;
-        uint8_t* ptile = sm + L::P_OFF + b * kTile;
+        uint8_t* ptile = sm + L::P_OFF + (GATED ? b : 0) * kTile;
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {
           float x[8];
@@ -438,8 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t ws[64], uh[64];
           tmem_ld32(qw + lane_base, *reinterpret_cast<uint32_t(*)[32]>(ws));
           tmem_ld32(qw + lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(ws + 32));
-          tmem_ld32(tmem + lane_base + TM_UH, *reinterpret_cast<uint32_t(*)[32]>(uh));
-          tmem_ld32(tmem + lane_base + TM_UH + 32, *reinterpret_cast<uint32_t(*)[32]>(uh + 32));
+          const uint32_t uhc = tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0);
+          tmem_ld32(uhc, *reinterpret_cast<uint32_t(*)[32]>(uh));
+          tmem_ld32(uhc + 32, *reinterpret_cast<uint32_t(*)[32]>(uh + 32));
           tmem_wait_ld();
 #pragma unroll
           for (int c16 = 0; c16 < 8; ++c16) {
@@ -518,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  using L = MainLayout<DK>;
+  using L = MainLayout<DK, GATED>;
   const int BH = p.B * p.H;
   const int nchunks = (p.T + kC - 1) / kC;
   cudaError_t e = launch_tsolve(p, w, st);

@@ -39,9 +39,9 @@ struct ChunkProblem {
 cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t st);
 bool chunk_simt_supported(int Dk, int Dv, int C);
 
-// tcgen05 (bf16 operands, float32 accumulate) chunked kernels.
-cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t st);
-bool chunk_tc_supported(const ChunkProblem& p);
+// tcgen05 (bf16 operands, float32 accumulate) chunked ELU+1 linear attention.
+cudaError_t launch_linear_tc(const ChunkProblem& p, cudaStream_t st);
+bool linear_tc_supported(const ChunkProblem& p);
 
 // Decode step (in-place state update).
 struct DecodeProblem {

@@ -63,15 +63,20 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int c0 = chunk * kC, n = min(kC, T - c0);
 
-  // 1. K tile, beta and the log-decay prefix g (rows >= n: k = 0, beta = 0, alpha = 1)
+  // 1. K tile, beta and the log-decay prefix g (rows >= n: k = 0, beta = 0, alpha = 1).
+  //    Every thread's K loads are issued before any is stored (all in flight at
+  //    once), and the beta / alpha loads overlap them.
+  constexpr int kVecPerRow = DK / 8;
+  constexpr int kLoads = kC * kVecPerRow / kThreads;
+  uint4 kreg[kLoads];
   {
     const __nv_bfloat16* src = k + ((size_t)bh * T + c0) * DK;
-    constexpr int kVecPerRow = DK / 8;
-    for (int i = tid; i < kC * kVecPerRow; i += kThreads) {
+#pragma unroll
+    for (int it = 0; it < kLoads; ++it) {
+      const int i = tid + it * kThreads;
       const int r = i / kVecPerRow, v = i % kVecPerRow;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (r < n) u = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * DK) + v);
-      *reinterpret_cast<uint4*>(Ks + r * KS + v * 8) = u;
+      kreg[it] = r < n ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * DK) + v)
+                       : make_uint4(0, 0, 0, 0);
     }
     if (tid < 64) {
       const size_t tb = (size_t)bh * T + c0;
@@ -93,6 +98,12 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
         veg[tid] = __expf(x);
         g_out[((size_t)bh * nchunks + chunk) * kC + tid] = x;
       }
+    }
+#pragma unroll
+    for (int it = 0; it < kLoads; ++it) {
+      const int i = tid + it * kThreads;
+      const int r = i / kVecPerRow, v = i % kVecPerRow;
+      *reinterpret_cast<uint4*>(Ks + r * KS + v * 8) = kreg[it];
     }
   }
   __syncthreads();
@@ -190,24 +201,24 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   }
   __syncthreads();
 
-  // 5. Tb = T diag(beta) and Tbg = Tb diag(e^g), bf16 rows: thread -> (row, 32-column half)
+  // 5. Tb = T diag(beta) and Tbg = Tb diag(e^g) as bf16 rows; each pass writes
+  //    16 rows, a warp covering 4 whole rows (512 contiguous bytes)
   {
-    const int row = tid & 63, h = tid >> 6;
     const size_t tile = ((size_t)bh * nchunks + chunk) * kC * kC;
-    __nv_bfloat16* dst = tb_out + tile + row * kC + 32 * h;
-    __nv_bfloat16* dstg = GATED ? tbg_out + tile + row * kC + 32 * h : nullptr;
-    const float* trow = Tm + row * kApad + 32 * h;
+    const int c8 = (tid & 7) * 8;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int row = pass * 16 + (tid >> 3);
+      const float* trow = Tm + row * kApad + c8;
       float x[8], y[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int sc = 32 * h + cc * 8 + e;
-        x[e] = sc <= row ? trow[cc * 8 + e] * vb[sc] : 0.f;
+        const int sc = c8 + e;
+        x[e] = sc <= row ? trow[e] * vb[sc] : 0.f;
         if (GATED) y[e] = x[e] * veg[sc];
       }
-      st_bf16x8(dst + cc * 8, x);
-      if (GATED) st_bf16x8(dstg + cc * 8, y);
+      st_bf16x8(tb_out + tile + row * kC + c8, x);
+      if (GATED) st_bf16x8(tbg_out + tile + row * kC + c8, y);
     }
   }
 }
