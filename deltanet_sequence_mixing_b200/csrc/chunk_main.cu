@@ -16,11 +16,13 @@
 // One CTA per (b, h, 64-column slice of Dv), 9 warps:
 //   warp 9     MMA issuer (one thread): every tcgen05.mma of the CTA, in a
 //              fixed order that keeps the state chain fed:
-//                [Q;W]S (c), W/Uh (c+1), QK^T (c+1), K^T U (c), PU (c)
-//              W/Uh (c+1) and QK^T (c+1) run while the U epilogue of chunk c
-//              drains (Uh is double-buffered in TMEM), so W (c+1) and the
-//              scores of chunk c+1 are ready before the state update of
-//              chunk c ends and only PU (c) shares the pipe with it.
+//                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
+//              (gated: QK^T (c+1) before K^T U (c), so that the gamma-scaled
+//              Q of chunk c+1 is ready as early as the new state).  W/Uh (c+1)
+//              runs while the U epilogue of chunk c drains (Uh is double-
+//              buffered in TMEM); PU (c) and QK^T (c+1) run during the state
+//              update.  Ungated, the single P tile is rewritten only after
+//              PU (c) has completed (QK^T (c+1) is committed after it).
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
 //              a three-stage ring (gated: two), L2 prefetch two chunks ahead
 //   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead)
@@ -111,8 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sb = warp_uniform(smem_u32(sm));
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = (int)warp_uniform((uint32_t)tid >> 5);  // role branches stay warp-uniform
   const int bh = blockIdx.x;
   const int j0 = blockIdx.y * kDVS;
   const int T = p.T, Dv = p.Dv;
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = warp_uniform(*tmem_slot);
   const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t tile_bytes = (2 * L::KB + (GATED ? 3 : 2)) * kTile;
@@ -215,125 +218,136 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- issuer --
-    if (lane == 0) {
-      auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
-      // P scores = Q K^T of chunk c (lanes 0-63 of TM_G)
-      auto issue_qkt = [&](int c) {
-        const uint32_t st = stage(c);
-        constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+    // The whole warp runs the issuer (warp-uniform control flow and operands);
+    // each MMA and commit is issued by one elected lane.  Wait results are
+    // combined over the warp so every lane takes the same path.
+    auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
+    // P scores = Q K^T of chunk c (lanes 0-63 of TM_G)
+    auto issue_qkt = [&](int c) {
+      const uint32_t st = stage(c);
+      constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
-          mma_bf16_ss(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
-        }
-      };
-      // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of Uh[c & 1]).
-      // Ungated both share the A operand Tb, and K's 64-column blocks and V sit
-      // KB_STRIDE apart, so for even chunks [W | Uh[0]] = Tb [K | V] is one
-      // N = Dk + 64 product.
-      auto issue_wu = [&](int c) {
-        const uint32_t st = stage(c);
-        if (!GATED && (c & 1) == 0) {
-          constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + TM_W, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
-                        desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), id, ks > 0);
-        } else {
-          constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
-          constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
-          // rows 64-127 of the A operand: Tbg (gated) or Tb
-          const uint32_t wa = st + (GATED ? L::TB_OFF : L::V_OFF);
-          const uint32_t uh = (c & 1) ? TM_UH1 : TM_UH0;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            mma_bf16_ss(tmem + TM_W, desc_k(wa + ks * 32), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                        idw, ks > 0);
-            mma_bf16_ss(tmem + uh, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
-                        desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
-          }
-        }
-      };
-      // [gamma Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
-      auto issue_qw = [&](int c) {
-        const uint32_t st = stage(c);
-        constexpr uint32_t id = idesc_bf16(128, 64, false, true);
-#pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-          const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-          mma_bf16_ss(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
-                      id, ks > 0);
-        }
-      };
-      // dS = K^T U~
-      auto issue_ds = [&](int c) {
-        const uint32_t st = stage(c);
-        const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
-        constexpr uint32_t id = idesc_bf16(128, 64, true, true);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                      desc_mn(ut + ks * 2048, kTile), id, ks > 0);
-      };
-      // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
-      auto issue_pu = [&](int c) {
-        const uint32_t pa = sb + L::P_OFF + (GATED ? (c & 1) : 0) * kTile;
-        constexpr uint32_t id = idesc_bf16(128, 64, false, true);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32),
-                      desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
-      };
-      bool ok = mbar_wait(bar + B_FULL, 0, wc);
-      if (ok) {
-        tc_fence_after();
-        issue_wu(0);
-        mma_commit(bar + B_PMMA2);
-        issue_qkt(0);
-        mma_commit(bar + B_PMMA1);
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
+        mma_bf16_ss_elect(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
       }
-      for (int c = 0; c < nchunks && ok; ++c) {
-        const int b = c & 1;
-        const bool nxt = c + 1 < nchunks;
-        ok = mbar_wait(bar + B_WREADY, c & 1, wc) && mbar_wait(bar + B_SREADY, c & 1, wc) &&
-             (c < 2 || mbar_wait(bar + B_OFREE + 8 * b, ((c >> 1) - 1) & 1, wc));
+    };
+    // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of Uh[c & 1]).
+    // Ungated both share the A operand Tb, and K's 64-column blocks and V sit
+    // KB_STRIDE apart, so for even chunks [W | Uh[0]] = Tb [K | V] is one
+    // N = Dk + 64 product.
+    auto issue_wu = [&](int c) {
+      const uint32_t st = stage(c);
+      if (!GATED && (c & 1) == 0) {
+        constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss_elect(tmem + TM_W, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
+                            desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), id, ks > 0);
+      } else {
+        constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
+        constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+        // rows 64-127 of the A operand: Tbg (gated) or Tb
+        const uint32_t wa = st + (GATED ? L::TB_OFF : L::V_OFF);
+        const uint32_t uh = (c & 1) ? TM_UH1 : TM_UH0;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ss_elect(tmem + TM_W, desc_k(wa + ks * 32), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                            idw, ks > 0);
+          mma_bf16_ss_elect(tmem + uh, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
+                            desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
+        }
+      }
+    };
+    // [gamma Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
+    auto issue_qw = [&](int c) {
+      const uint32_t st = stage(c);
+      constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
+                          id, ks > 0);
+      }
+    };
+    // dS = K^T U~
+    auto issue_ds = [&](int c) {
+      const uint32_t st = stage(c);
+      const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
+      constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16_ss_elect(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                          desc_mn(ut + ks * 2048, kTile), id, ks > 0);
+    };
+    // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
+    auto issue_pu = [&](int c) {
+      const uint32_t pa = sb + L::P_OFF + (GATED ? (c & 1) : 0) * kTile;
+      constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32),
+                          desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
+    };
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL, 0, wc));
+    if (ok) {
+      tc_fence_after();
+      issue_wu(0);
+      mma_commit_elect(bar + B_PMMA2);
+      issue_qkt(0);
+      mma_commit_elect(bar + B_PMMA1);
+    }
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int b = c & 1;
+      const bool nxt = c + 1 < nchunks;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar + B_WREADY, c & 1, wc) && mbar_wait(bar + B_SREADY, c & 1, wc) &&
+                          (c < 2 || mbar_wait(bar + B_OFREE + 8 * b, ((c >> 1) - 1) & 1, wc)));
+      if (!ok) break;
+      tc_fence_after();
+      issue_qw(c);
+      mma_commit_elect(bar + B_CMMA3);
+      if (nxt) {  // W (c) is already in shared memory and Uh[(c+1) & 1] was consumed by chunk c-1
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        issue_qw(c);
-        mma_commit(bar + B_CMMA3);
-        if (nxt) {  // W (c) is already in shared memory and Uh[(c+1) & 1] was consumed by chunk c-1
-          ok = mbar_wait(bar + B_FULL + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          issue_wu(c + 1);
-          mma_commit(bar + B_PMMA2);
-        }
-        // QK^T (c+1) once the scores of chunk c have left TMEM (P_READY); it
-        // runs while the U epilogue of chunk c drains
-        ok = mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc);
+        issue_wu(c + 1);
+        mma_commit_elect(bar + B_PMMA2);
+      }
+      if (GATED) {  // QK^T (c+1) once the scores of chunk c have left TMEM (P_READY)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
         if (!ok) break;
         if (nxt) {
           tc_fence_after();
           issue_qkt(c + 1);
-          mma_commit(bar + B_PMMA1);
+          mma_commit_elect(bar + B_PMMA1);
         }
-        ok = mbar_wait(bar + B_UREADY, c & 1, wc);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_UREADY, c & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      issue_ds(c);
+      mma_commit_elect(bar + B_CMMA4);
+      // K^T U (c) was the last reader of stage c: the P / Q / W epilogues of
+      // chunk c are done (W_READY, and gated P_READY, came before it)
+      mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
+      if (!GATED) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        issue_ds(c);
-        mma_commit(bar + B_CMMA4);
-        // K^T U (c) was the last reader of stage c: the P / Q / W epilogues of
-        // chunk c are done (W_READY, and gated P_READY, came before it)
-        mma_commit(bar + B_EMPTY + 8 * (c % NST));
-        issue_pu(c);
-        mma_commit(bar + B_CMMA5 + 8 * b);
       }
-      tc_fence_after();  // no MMA may outlive TMEM
-      mma_commit(bar + B_FIN);
-      int zero = 0;
-      const WaitCtl fin{&zero, p.status, kWaitLimitNs};
-      (void)mbar_wait(bar + B_FIN, 0, fin);
+      issue_pu(c);
+      mma_commit_elect(bar + B_CMMA5 + 8 * b);
+      if (!GATED && nxt) {  // after PU (c): the single P tile is free once PMMA1 fires
+        issue_qkt(c + 1);
+        mma_commit_elect(bar + B_PMMA1);
+      }
     }
+    tc_fence_after();  // no MMA may outlive TMEM
+    mma_commit_elect(bar + B_FIN);
+    int zero = 0;
+    const WaitCtl fin{&zero, p.status, kWaitLimitNs};
+    (void)mbar_wait(bar + B_FIN, 0, fin);
   } else if (warp >= 6) {
     // ------------------------------------------------------- W rows (6-7) --
     const int row = (tid - 192) & 63;
@@ -376,11 +390,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
         tmem_wait_ld();
-        if (!GATED && c > 0) {  // the single P tile: PU (c-1) must have read it
-          ok = named_bar_and(kBarPrepP, 64,
-                             mbar_wait(bar + B_CMMA5 + 8 * ((c - 1) & 1), ((c - 1) >> 1) & 1, wc));
-          if (!ok) break;
-        }
         const float gr = GATED ? vs[64 + row] : 0.f;
         uint8_t* ptile = sm + L::P_OFF + (GATED ? b : 0) * kTile;
 #pragma unroll

@@ -129,6 +129,27 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same MMA issued by one elected lane of a warp whose 32 lanes all execute
+// the call with identical (warp-uniform) operands.  Keeping the issuing code
+// warp-uniform lets the descriptors stay in uniform registers; issuing from a
+// single divergent lane costs extra instructions per MMA.
+__device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred e, p; .reg .b32 x; elect.sync x|e, 0xffffffff; setp.ne.b32 p, %4, 0;"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Commit from one elected lane of a warp-uniform issuer (see mma_bf16_ss_elect).
+__device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{ .reg .pred e; .reg .b32 x; elect.sync x|e, 0xffffffff;"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0]; }" ::"r"(bar)
+      : "memory");
+}
+// A value every lane of the warp holds, made visibly warp-uniform (lane 0's).
+__device__ __forceinline__ uint32_t warp_uniform(uint32_t v) { return __shfl_sync(0xffffffffu, v, 0); }
 // Arrive on `bar` once every previously issued MMA of this thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
