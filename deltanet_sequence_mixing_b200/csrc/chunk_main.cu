@@ -25,9 +25,10 @@
 //              PU (c) has completed (QK^T (c+1) is committed after it).
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
 //              a three-stage ring (gated: two), L2 prefetch two chunks ahead
-//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead)
+//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead),
+//              then columns 32-63 of the U epilogue
 //   warps 4-5  P rows to bf16; gated: Q <- diag(gamma) Q in place
-//   warps 2-3  U = Uh - WS;   warps 0-3 the state update;
+//   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
 //   warps 0-1  drain the output tile O = gamma QS + PU
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
 // signal back; the issuer waits on their signals.  Every mbarrier completes
@@ -101,6 +102,29 @@ __device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* m, int x, int 
                : "memory");
 }
 
+// One half (32 columns, [col0, col0 + 32)) of the U epilogue for the row on
+// this thread's TMEM lane: U = Uh - WS to bf16 (gated also U~ = U e^(g_last - g_row)).
+template <bool GATED>
+__device__ __forceinline__ void u_epilogue_half(uint32_t ws_addr, uint32_t uh_addr, int col0, int row, float wl,
+                                                uint8_t* u_tile, uint8_t* ut_tile) {
+  uint32_t ws[32], uh[32];
+  tmem_ld32(ws_addr + col0, ws);
+  tmem_ld32(uh_addr + col0, uh);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float x[8], y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      x[e] = __uint_as_float(uh[q * 8 + e]) - __uint_as_float(ws[q * 8 + e]);
+      y[e] = x[e] * wl;
+    }
+    const int c16 = col0 / 8 + q;
+    st_bf16x8(u_tile + sw128_off(row, c16), x);
+    if (GATED) st_bf16x8(ut_tile + sw128_off(row, c16), y);
+  }
+}
+
 template <int DK, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -139,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_CMMA4, 1);
     mbar_init(bar + B_PMMA1, 1);
     mbar_init(bar + B_PMMA2, 1);
-    mbar_init(bar + B_UREADY, 1);
+    mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
     mbar_init(bar + B_WREADY, GATED ? 2 : 1);  // W rows (+ gamma-scaled Q when gated)
     mbar_init(bar + B_FIN, 1);
@@ -371,6 +395,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       named_bar_sync(kBarPrepW, 64);
       if (tid == 192) mbar_arrive(bar + B_WREADY);
+
+      // ---- columns 32-63 of the U epilogue of chunk c (rows on lanes 64-127) ----
+      ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_CMMA3, c & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int n = min(kC, T - c * kC);
+        const float* vb = cvec + (c & 1) * 64;
+        const float wl = GATED ? __expf(vb[n - 1] - vb[row]) : 1.f;
+        u_epilogue_half<GATED>(tmem + lane_base + TM_QW + 64 * (c & 1),
+                               tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0), 32, row, wl, sm + L::U_OFF,
+                               sm + L::UT_OFF);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarPrepW, 64);
+      if (tid == 192) mbar_arrive(bar + B_UREADY);
     }
   } else if (warp >= 4) {
     // -------------------------------------------- P rows, gamma Q (4-5) --
@@ -462,24 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok_hi) {
           tc_fence_after();
           const float wl = GATED ? __expf(vb[n - 1] - vb[row]) : 1.f;
-          uint32_t ws[64], uh[64];
-          tmem_ld32(qw + lane_base, *reinterpret_cast<uint32_t(*)[32]>(ws));
-          tmem_ld32(qw + lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(ws + 32));
-          const uint32_t uhc = tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0);
-          tmem_ld32(uhc, *reinterpret_cast<uint32_t(*)[32]>(uh));
-          tmem_ld32(uhc + 32, *reinterpret_cast<uint32_t(*)[32]>(uh + 32));
-          tmem_wait_ld();
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8], y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              x[e] = __uint_as_float(uh[c16 * 8 + e]) - __uint_as_float(ws[c16 * 8 + e]);
-              y[e] = x[e] * wl;
-            }
-            st_bf16x8(sm + L::U_OFF + sw128_off(row, c16), x);
-            if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(row, c16), y);
-          }
+          // columns 0-31 here, 32-63 in the W warps (same TMEM lanes)
+          u_epilogue_half<GATED>(qw + lane_base, tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0), 0, row, wl,
+                                 sm + L::U_OFF, sm + L::UT_OFF);
           fence_proxy_async_smem();
           tc_fence_before();
           named_bar_sync(kBarChainHi, 64);

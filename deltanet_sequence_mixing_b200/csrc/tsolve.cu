@@ -12,13 +12,13 @@
 // of dependent steps, so it is latency-bound per chunk and the grid's
 // parallelism over chunks hides that latency.
 //   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
-//   2. G = K K^T with bf16 WMMA (float32 accumulate) straight into the A scratch.
-//   3. A = mask / scale G in place.
-//   4. Four 16x16 diagonal inverses (one column per lane, right-looking
+//   2. G = K K^T with bf16 WMMA (float32 accumulate) straight into the A scratch,
+//      each warp masking and scaling its own tiles into A.
+//   3. Four 16x16 diagonal inverses (one column per lane, right-looking
 //      substitution so only one multiply-add per step is on the dependency
 //      chain), then each warp finishes one 16-column block of T by block
 //      forward substitution with tf32 WMMA products, T_iw = -D_i sum A_im T_mw.
-//   5. Tb, Tbg -> global (row-major bf16, 8 KB per tile).
+//   4. Tb, Tbg -> global (row-major bf16, 8 KB per tile).
 #include <cuda_bf16.h>
 #include <mma.h>
 
@@ -35,10 +35,13 @@ constexpr int kThreads = 128;
 constexpr int kApad = 68;
 constexpr int kKpad = 8;  // bf16 padding of the K rows (keeps WMMA rows 16-byte aligned)
 
+// tf32 operands by truncation: keep the sign, exponent and top 10 mantissa bits
+// (round toward zero, relative error < 2^-10; the factors leave this kernel
+// rounded to bf16, 2^-8).  One integer AND per element.
 template <typename Frag>
 __device__ __forceinline__ void to_tf32(Frag& f) {
 #pragma unroll
-  for (int t = 0; t < f.num_elements; ++t) f.x[t] = wmma::__float_to_tf32(f.x[t]);
+  for (int t = 0; t < f.num_elements; ++t) f.x[t] = __uint_as_float(__float_as_uint(f.x[t]) & 0xFFFFE000u);
 }
 
 template <int DK, bool GATED>
@@ -108,7 +111,11 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   }
   __syncthreads();
 
-  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps), straight into A
+  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps), straight into A,
+  //    and each warp turns its own tiles into A = strict_lower(diag(beta) G * Gamma).
+  //    Nothing reads A's upper tiles or T's strictly-upper tiles unmasked (the
+  //    diagonal solve writes whole diagonal tiles, the block solve reads tiles on
+  //    or below the diagonal, the output masks by column <= row).
   {
     wmma::fragment<wmma::matrix_a, 16, 16, 16, __nv_bfloat16, wmma::row_major> fa;
     wmma::fragment<wmma::matrix_b, 16, 16, 16, __nv_bfloat16, wmma::col_major> fb;
@@ -125,24 +132,24 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
         wmma::mma_sync(acc, fa, fb, acc);
       }
       wmma::store_matrix_sync(Am + (16 * ti) * kApad + 16 * tj, acc, kApad, wmma::mem_row_major);
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        const int r = 16 * ti + (e >> 4), c = 16 * tj + (e & 15);
+        float* ap = Am + r * kApad + c;
+        float a = 0.f;
+        if (c < r) {
+          a = vb[r] * *ap;
+          if (GATED) a *= __expf(vg[r] - vg[c]);
+        }
+        *ap = a;
+      }
     }
   }
   __syncthreads();
 
-  // 3. A = strict_lower(diag(beta) G * Gamma) in place; T's strictly-upper blocks = 0
-  for (int i = tid; i < 64 * 64; i += kThreads) {
-    const int r = i >> 6, s = i & 63;
-    float a = 0.f;
-    if (s < r) {
-      a = vb[r] * Am[r * kApad + s];
-      if (GATED) a *= __expf(vg[r] - vg[s]);
-    }
-    Am[r * kApad + s] = a;
-    if ((s >> 4) > (r >> 4)) Tm[r * kApad + s] = 0.f;
-  }
-  __syncthreads();
-
-  // 4. T = (I + A)^-1.  Diagonal 16x16 blocks D_w: warp w, lanes 0-15 own
+  // 3. T = (I + A)^-1.  Diagonal 16x16 blocks D_w: warp w, lanes 0-15 own
   //    column j; right-looking, so only one multiply-add per step is on the
   //    dependency chain.
   if (lane < 16) {
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   }
   __syncthreads();
 
-  // 5. Tb = T diag(beta) and Tbg = Tb diag(e^g) as bf16 rows; each pass writes
+  // 4. Tb = T diag(beta) and Tbg = Tb diag(e^g) as bf16 rows; each pass writes
   //    16 rows, a warp covering 4 whole rows (512 contiguous bytes)
   {
     const size_t tile = ((size_t)bh * nchunks + chunk) * kC * kC;
