@@ -191,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmTb);
       if (GATED) prefetch_tmap(&tmTbg);
     }
+    // Tb, Tbg and g come from the pre-pass launched just before this kernel
+    grid_dependency_wait();
     int issued = 0;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % NST, use = c / NST;
@@ -587,8 +589,19 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
-  kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, mtb, mtbg, p, w.g);
-  return cudaGetLastError();
+  // Programmatic dependent launch: CTAs may start (TMEM, barriers, state
+  // load) while the pre-pass drains; the producer waits for its results.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mtb, mtbg, p, w.g);
 }
 
 }  // namespace

@@ -26,6 +26,17 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
+// ------------------------------------------------ programmatic dependent launch --
+// Block until the grids this one depends on (launched before it on the stream
+// with programmatic serialisation) have completed and their writes are visible.
+// A no-op for a normal launch.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid begin launching (its CTAs still wait for this grid's
+// completion before reading its results).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -228,6 +228,9 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
       if (GATED) st_bf16x8(tbg_out + tile + row * kC + c8, y);
     }
   }
+  // The chunk kernel may begin launching once every CTA got here (it still
+  // waits for this grid to complete before reading the factors).
+  grid_launch_dependents();
 }
 
 template <int DK, bool GATED>
