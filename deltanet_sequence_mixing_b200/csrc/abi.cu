@@ -89,10 +89,10 @@ int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
   p.status = static_cast<unsigned int*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dn::chunk_main_supported(p)) {
+  if (dn::chunk_main_supported(p) || dn::chunk128_supported(p)) {
     const dn::WyWorkspace w =
-        dn::chunk_main_carve(static_cast<uint8_t*>(ws) + kStatusBytes, p.B, p.H, p.T);
-    return map_cuda(dn::launch_chunk_main(p, w, st));
+        dn::wy_carve(static_cast<uint8_t*>(ws) + kStatusBytes, p.B, p.H, p.T, p.C);
+    return map_cuda(p.C == 64 ? dn::launch_chunk_main(p, w, st) : dn::launch_chunk128(p, w, st));
   }
   if (dn::linear_tc_supported(p)) return map_cuda(dn::launch_linear_tc(p, st));
   if (dn::chunk_simt_supported(p.Dk, p.Dv, p.C)) return map_cuda(dn::launch_chunk_simt(p, st));
@@ -106,8 +106,8 @@ extern "C" {
 size_t deltanet_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
   if (B < 0 || H < 0 || T < 0 || !valid_dim(Dk) || !valid_dim(Dv)) return 0;
   if ((C != 64 && C != 128) || (dt != DN_F32 && dt != DN_BF16)) return 0;
-  // bf16 chunk size 64: room for the per-chunk WY factors of the pre-pass
-  if (dt == DN_BF16 && C == 64 && T > 0) return kStatusBytes + dn::chunk_main_workspace(B, H, T);
+  // bf16: room for the per-chunk WY factors of the pre-pass
+  if (dt == DN_BF16 && T > 0) return kStatusBytes + dn::wy_workspace_bytes(B, H, T, C);
   return kStatusBytes;
 }
 

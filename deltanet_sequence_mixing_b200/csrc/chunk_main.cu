@@ -95,13 +95,6 @@ constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREAD
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
                    B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164;
 
-__device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-
 // One half (32 columns, [col0, col0 + 32)) of the U epilogue for the row on
 // this thread's TMEM lane: U = Uh - WS to bf16 (gated also U~ = U e^(g_last - g_row)).
 template <bool GATED>
@@ -609,23 +602,6 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
 bool chunk_main_supported(const ChunkProblem& p) {
   return p.bf16 && p.mode == Mode::Delta && p.T > 0 && p.C == 64 && (p.Dk == 64 || p.Dk == 128) &&
          (p.Dv == 64 || p.Dv == 128);
-}
-
-size_t chunk_main_workspace(int B, int H, int T) {
-  const size_t nch = ((size_t)T + kC - 1) / kC;
-  const size_t tiles = (size_t)B * H * nch;
-  return tiles * (2 * (size_t)kC * kC * 2 + (size_t)kC * 4);  // Tb, Tbg (bf16) and g (f32)
-}
-
-WyWorkspace chunk_main_carve(void* base, int B, int H, int T) {
-  const size_t nch = ((size_t)T + kC - 1) / kC;
-  const size_t tiles = (size_t)B * H * nch;
-  uint8_t* p = static_cast<uint8_t*>(base);
-  WyWorkspace w;
-  w.tb = reinterpret_cast<__nv_bfloat16*>(p);
-  w.tbg = reinterpret_cast<__nv_bfloat16*>(p + tiles * kC * kC * 2);
-  w.g = reinterpret_cast<float*>(p + 2 * tiles * kC * kC * 2);
-  return w;
 }
 
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {

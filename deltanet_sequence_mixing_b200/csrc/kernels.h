@@ -61,19 +61,24 @@ cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t st);
 // rows past T read as zeros.
 bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, int D, int T, int BH);
 
-// Per-chunk WY factors written by the pre-pass and read by the chunk kernel.
+// Per-chunk WY factors written by the pre-pass and read by the chunk kernels
+// (C = 64 or 128 token chunks).
 struct WyWorkspace {
-  __nv_bfloat16* tb;   // [B*H][chunks][64][64]  T diag(beta)
-  __nv_bfloat16* tbg;  // [B*H][chunks][64][64]  T diag(beta) diag(exp(g))   (gated)
-  float* g;            // [B*H][chunks][64]      cumulative log decay        (gated)
+  __nv_bfloat16* tb;   // [B*H][chunks][C][C]  T diag(beta)
+  __nv_bfloat16* tbg;  // [B*H][chunks][C][C]  T diag(beta) diag(exp(g))   (gated)
+  float* g;            // [B*H][chunks][C]     cumulative log decay        (gated)
 };
+size_t wy_workspace_bytes(int B, int H, int T, int C);
+WyWorkspace wy_carve(void* base, int B, int H, int T, int C);
 cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 
 // tcgen05 chunked delta rule after the pre-pass (bf16, C = 64).
 bool chunk_main_supported(const ChunkProblem& p);
-size_t chunk_main_workspace(int B, int H, int T);
-WyWorkspace chunk_main_carve(void* base, int B, int H, int T);
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
+
+// tcgen05 chunked delta rule after the pre-pass (bf16, C = 128).
+bool chunk128_supported(const ChunkProblem& p);
+cudaError_t launch_chunk128(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(unsigned int* status, long long wait_ns, cudaStream_t st);

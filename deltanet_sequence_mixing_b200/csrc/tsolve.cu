@@ -1,24 +1,25 @@
 // Chunk-parallel WY pre-pass of the tcgen05 delta-rule forward: for every
-// (b, h, chunk) it forms T = (I + A)^-1 with
+// (b, h, chunk of C = 64 or 128 tokens) it forms T = (I + A)^-1 with
 //   A = strict_lower(diag(beta) (K K^T * Gamma)),   Gamma_rs = exp(g_r - g_s),
 // and writes Tb = T diag(beta) (and, gated, Tbg = Tb diag(exp(g))) as bf16
-// 64 x 64 tiles into the workspace, plus the chunk's decay prefix g.  These are
+// C x C tiles into the workspace, plus the chunk's decay prefix g.  These are
 // the state-independent parts of the Householder / WY reparameterisation
 // ("GPT-2 から Kimi K3 まで", news.ainew.jp, section "DeltaNet (Parallelizing linear
 // transformers with delta rule)"); the chunk kernel then applies them with
 // tensor-core products, keeping only matrix products on its serial state chain.
 //
-// One 128-thread CTA per chunk, several CTAs per SM: the solve is a short chain
+// One CTA of 2C threads (one warp per 16-row block) per chunk, several CTAs per
+// SM at C = 64: the solve is a short chain
 // of dependent steps, so it is latency-bound per chunk and the grid's
 // parallelism over chunks hides that latency.
 //   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
 //   2. G = K K^T with bf16 WMMA (float32 accumulate) straight into the A scratch,
 //      each warp masking and scaling its own tiles into A.
-//   3. Four 16x16 diagonal inverses (one column per lane, right-looking
+//   3. C/16 diagonal 16x16 inverses (one column per lane, right-looking
 //      substitution so only one multiply-add per step is on the dependency
 //      chain), then each warp finishes one 16-column block of T by block
 //      forward substitution with tf32 WMMA products, T_iw = -D_i sum A_im T_mw.
-//   4. Tb, Tbg -> global (row-major bf16, 8 KB per tile).
+//   4. Tb, Tbg -> global (row-major bf16 C x C tiles).
 #include <cuda_bf16.h>
 #include <mma.h>
 
@@ -30,10 +31,23 @@ namespace {
 
 using namespace nvcuda;
 
-constexpr int kC = 64;
-constexpr int kThreads = 128;
-constexpr int kApad = 68;
 constexpr int kKpad = 8;  // bf16 padding of the K rows (keeps WMMA rows 16-byte aligned)
+
+template <int C>
+struct TsolveShape {
+  static constexpr int kThreads = 2 * C;       // one warp per 16-row block
+  static constexpr int kWarps = kThreads / 32;  // == C / 16
+  static constexpr int kApad = C + 4;           // float row stride of the A / T scratch
+  static constexpr int kTiles = kWarps * (kWarps + 1) / 2;  // lower 16x16 tiles of the Gram
+  static_assert(kWarps == C / 16, "one warp per 16-row block");
+};
+
+template <int C, int DK>
+constexpr size_t tsolve_smem_bytes() {
+  return (C * (DK + kKpad) * 2 > C * TsolveShape<C>::kApad * 4 ? C * (DK + kKpad) * 2
+                                                                : C * TsolveShape<C>::kApad * 4) +
+         (size_t)C * TsolveShape<C>::kApad * 4 + (3 * C + 8) * 4;
+}
 
 // tf32 operands by truncation: keep the sign, exponent and top 10 mantissa bits
 // (round toward zero, relative error < 2^-10; the factors leave this kernel
@@ -44,14 +58,16 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
   for (int t = 0; t < f.num_elements; ++t) f.x[t] = __uint_as_float(__float_as_uint(f.x[t]) & 0xFFFFE000u);
 }
 
-template <int DK, bool GATED>
-__global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
+template <int C, int DK, bool GATED>
+__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
                                                           const float* __restrict__ beta,
                                                           const float* __restrict__ alpha,
                                                           __nv_bfloat16* __restrict__ tb_out,
                                                           __nv_bfloat16* __restrict__ tbg_out,
                                                           float* __restrict__ g_out, int T,
                                                           int nchunks) {
+  using Sh = TsolveShape<C>;
+  constexpr int kC = C, kThreads = Sh::kThreads, kApad = Sh::kApad;
   constexpr int KS = DK + kKpad;
   constexpr int kRegion = (kC * KS * 2 > kC * kApad * 4) ? kC * KS * 2 : kC * kApad * 4;
   extern __shared__ __align__(128) uint8_t tsolve_smem[];
@@ -59,8 +75,9 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   float* Tm = reinterpret_cast<float*>(tsolve_smem);  // reuses the K tile after the Gram
   float* Am = reinterpret_cast<float*>(tsolve_smem + kRegion);
   float* vb = Am + kC * kApad;
-  float* vg = vb + 64;
-  float* veg = vg + 64;
+  float* vg = vb + kC;
+  float* veg = vg + kC;
+  float* wsum = veg + kC;  // per-warp totals of the log-decay scan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, bh = blockIdx.y;
@@ -72,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   constexpr int kVecPerRow = DK / 8;
   constexpr int kLoads = kC * kVecPerRow / kThreads;
   uint4 kreg[kLoads];
+  float glog = 0.f;
   {
     const __nv_bfloat16* src = k + ((size_t)bh * T + c0) * DK;
 #pragma unroll
@@ -81,25 +99,17 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
       kreg[it] = r < n ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * DK) + v)
                        : make_uint4(0, 0, 0, 0);
     }
-    if (tid < 64) {
+    if (tid < kC) {
       const size_t tb = (size_t)bh * T + c0;
       vb[tid] = tid < n ? beta[tb + tid] : 0.f;
-      if (GATED) {
-        float x = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
+      if (GATED) {  // inclusive scan of max(log alpha, -87) within each warp
+        glog = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, x, off);
-          if (lane >= off) x += y;
+          const float y = __shfl_up_sync(0xffffffffu, glog, off);
+          if (lane >= off) glog += y;
         }
-        if (warp == 1) {
-          float l0 = lane < n ? fmaxf(__logf(alpha[tb + lane]), -87.f) : 0.f;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-          x += l0;
-        }
-        vg[tid] = x;
-        veg[tid] = __expf(x);
-        g_out[((size_t)bh * nchunks + chunk) * kC + tid] = x;
+        if (lane == 31) wsum[warp] = glog;
       }
     }
 #pragma unroll
@@ -110,8 +120,17 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
     }
   }
   __syncthreads();
+  if (GATED) {  // add the totals of the earlier warps: g = cumsum over the chunk
+    if (tid < kC) {
+      for (int w = 0; w < warp; ++w) glog += wsum[w];
+      vg[tid] = glog;
+      veg[tid] = __expf(glog);
+      g_out[((size_t)bh * nchunks + chunk) * kC + tid] = glog;
+    }
+    __syncthreads();
+  }
 
-  // 2. G = K K^T (lower 16x16 tiles only: 10 tiles over 4 warps), straight into A,
+  // 2. G = K K^T (lower 16x16 tiles only, spread over the warps), straight into A,
   //    and each warp turns its own tiles into A = strict_lower(diag(beta) G * Gamma).
   //    Nothing reads A's upper tiles or T's strictly-upper tiles unmasked (the
   //    diagonal solve writes whole diagonal tiles, the block solve reads tiles on
@@ -120,9 +139,10 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
     wmma::fragment<wmma::matrix_a, 16, 16, 16, __nv_bfloat16, wmma::row_major> fa;
     wmma::fragment<wmma::matrix_b, 16, 16, 16, __nv_bfloat16, wmma::col_major> fb;
     wmma::fragment<wmma::accumulator, 16, 16, 16, float> acc;
-    for (int t = warp; t < 10; t += 4) {
-      // t -> (ti, tj) with tj <= ti: 0:(0,0) 1:(1,0) 2:(1,1) 3:(2,0) 4:(2,1) 5:(2,2) 6..9:(3,*)
-      const int ti = t < 1 ? 0 : t < 3 ? 1 : t < 6 ? 2 : 3;
+    for (int t = warp; t < Sh::kTiles; t += Sh::kWarps) {
+      // t -> (ti, tj), tj <= ti, row-major over the lower triangle of tiles
+      int ti = 0;
+      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
       const int tj = t - ti * (ti + 1) / 2;
       wmma::fill_fragment(acc, 0.f);
 #pragma unroll
@@ -176,8 +196,8 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
     wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
     wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
     wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
-    float* xs = Am + (16 * warp) * kApad + 48;  // 16x16 scratch in A's zero upper part
-    for (int i = warp + 1; i < 4; ++i) {
+    float* xs = Am + (16 * warp) * kApad + (kC - 16);  // 16x16 scratch in A's unused upper part
+    for (int i = warp + 1; i < Sh::kWarps; ++i) {
       wmma::fill_fragment(acc, 0.f);
       for (int m = warp; m < i; ++m) {
 #pragma unroll
@@ -209,13 +229,14 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   __syncthreads();
 
   // 4. Tb = T diag(beta) and Tbg = Tb diag(e^g) as bf16 rows; each pass writes
-  //    16 rows, a warp covering 4 whole rows (512 contiguous bytes)
+  //    16 rows, consecutive threads covering whole rows (contiguous bytes)
   {
     const size_t tile = ((size_t)bh * nchunks + chunk) * kC * kC;
-    const int c8 = (tid & 7) * 8;
+    constexpr int kTpr = kC / 8;  // threads per row
+    const int c8 = (tid % kTpr) * 8;
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int row = pass * 16 + (tid >> 3);
+    for (int pass = 0; pass < kC / 16; ++pass) {
+      const int row = pass * 16 + tid / kTpr;
       const float* trow = Tm + row * kApad + c8;
       float x[8], y[8];
 #pragma unroll
@@ -233,27 +254,50 @@ __global__ void __launch_bounds__(kThreads, 6) tsolve_kernel(const __nv_bfloat16
   grid_launch_dependents();
 }
 
-template <int DK, bool GATED>
+template <int C, int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  const int nchunks = (p.T + kC - 1) / kC;
-  constexpr size_t kKbytes = (size_t)kC * (DK + kKpad) * 2, kTbytes = (size_t)kC * kApad * 4;
-  constexpr size_t smem = (kKbytes > kTbytes ? kKbytes : kTbytes) + kTbytes + 3 * 64 * 4;
-  auto kern = tsolve_kernel<DK, GATED>;
+  const int nchunks = (p.T + C - 1) / C;
+  constexpr size_t smem = tsolve_smem_bytes<C, DK>();
+  auto kern = tsolve_kernel<C, DK, GATED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nchunks, (unsigned)(p.B * p.H));
-  kern<<<grid, kThreads, smem, st>>>(
+  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(p.k), p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks);
   return cudaGetLastError();
+}
+
+template <int C>
+cudaError_t launch_c(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_t<C, 128, true>(p, w, st) : launch_t<C, 128, false>(p, w, st);
+  if (p.Dk == 64) return gated ? launch_t<C, 64, true>(p, w, st) : launch_t<C, 64, false>(p, w, st);
+  return cudaErrorNotSupported;
 }
 
 }  // namespace
 
 cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  const bool gated = p.alpha != nullptr;
-  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
-  if (p.Dk == 64) return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
+  if (p.C == 64) return launch_c<64>(p, w, st);
+  if (p.C == 128) return launch_c<128>(p, w, st);
   return cudaErrorNotSupported;
+}
+
+size_t wy_workspace_bytes(int B, int H, int T, int C) {
+  const size_t nch = ((size_t)T + C - 1) / C;
+  const size_t tiles = (size_t)B * H * nch;
+  return tiles * (2 * (size_t)C * C * 2 + (size_t)C * 4);  // Tb, Tbg (bf16) and g (f32)
+}
+
+WyWorkspace wy_carve(void* base, int B, int H, int T, int C) {
+  const size_t nch = ((size_t)T + C - 1) / C;
+  const size_t tiles = (size_t)B * H * nch;
+  uint8_t* q = static_cast<uint8_t*>(base);
+  WyWorkspace w;
+  w.tb = reinterpret_cast<__nv_bfloat16*>(q);
+  w.tbg = reinterpret_cast<__nv_bfloat16*>(q + tiles * C * C * 2);
+  w.g = reinterpret_cast<float*>(q + 2 * tiles * C * C * 2);
+  return w;
 }
 
 }  // namespace dn

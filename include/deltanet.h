@@ -58,10 +58,11 @@ typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
 
 /*
  * Bytes of device workspace the chunked calls need for this problem: 256 for
- * the sticky device status word and its padding, plus, for bf16 inputs with
- * C = 64, 16,640 bytes per (b, h, 64-token chunk) for the per-chunk factors
- * T diag(beta), T diag(beta) diag(gamma) and the decay prefix that the
- * chunk-parallel pre-pass hands to the chunk kernel.  The workspace must be
+ * the sticky device status word and its padding, plus, for bf16 inputs, per
+ * (b, h, chunk of C tokens) 4 C^2 + 4 C bytes (16,640 at C = 64, 66,048 at
+ * C = 128) for the per-chunk factors T diag(beta), T diag(beta) diag(gamma)
+ * (bf16 C x C) and the decay prefix (C floats) that the chunk-parallel
+ * pre-pass hands to the chunk kernel.  The workspace must be
  * cleared once with deltanet_workspace_init before its first use; it may then
  * be reused by any number of calls on the same stream.  Returns 0 for sizes
  * the library rejects.

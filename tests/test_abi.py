@@ -65,6 +65,12 @@ def test_workspace_bytes(L):
     assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 32, 1) == 0
     assert L.deltanet_workspace_bytes(-1, 16, 4096, 128, 128, 64, 1) == 0
     assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 64, 7) == 0
+    # bf16: status word + per (b, h, chunk) the bf16 C x C factors Tb, Tbg and C floats of g
+    for C, T in ((64, 4096), (64, 100), (128, 65536), (128, 300)):
+        nch = -(-T // C)
+        want = 256 + 4 * 16 * nch * (2 * C * C * 2 + C * 4)
+        assert L.deltanet_workspace_bytes(4, 16, T, 128, 128, C, 1) == want
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 128, 0) == 256  # f32: status only
 
 
 # Fake, never dereferenced device addresses: every call below must be rejected

@@ -70,7 +70,7 @@ def _run_chunk_like_bench(dn, w, x):
     return o, S
 
 
-@pytest.mark.parametrize("w", [gen.PREFILL, gen.FORGET, gen.LONG64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [gen.PREFILL, gen.FORGET, gen.LONG64, gen.LONG128], ids=lambda w: w.name)
 def test_full_size_chunk_forward_sampled_heads(dn, oracle_mod, w):
     dev = torch.device("cuda")
     x = gen.make_workload(w, seed=11, device=dev)

@@ -83,6 +83,33 @@ def test_gated(dn, oracle_mod, dtype, T):
     _check_delta(dn, oracle_mod, x)
 
 
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("Dk,Dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 127, 128, 129, 300, 700])
+def test_chunk128_bf16(dn, oracle_mod, gated, Dk, Dv, T):
+    """Chunk size 128 (bf16): one state application per 128 tokens."""
+    x = gen.make_inputs(2, 2, T, Dk, Dv, torch.bfloat16, gated=gated, seed=300 + T + Dk + Dv)
+    _check_delta(dn, oracle_mod, x, C=128)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_chunk128_initial_state_and_gate_zero(dn, oracle_mod, gated):
+    x = gen.make_inputs(1, 3, 333, 128, 128, torch.bfloat16, gated=gated, seed=41)
+    if gated:
+        x["alpha"][:, :, 150] = 0.0
+    S0 = torch.randn(1, 3, 128, 128, generator=torch.Generator().manual_seed(5)) * 0.2
+    _check_delta(dn, oracle_mod, x, C=128, S0=S0)
+
+
+def test_chunk_size_invariance_bf16(dn):
+    """C = 64 and C = 128 compute the same recurrence: the two results agree to
+    within the bf16 gate (each is within it of the oracle)."""
+    x = gen.make_inputs(2, 2, 1000, 128, 128, torch.bfloat16, gated=True, seed=42)
+    o1, S1 = _run_delta(dn, x, C=64)
+    o2, S2 = _run_delta(dn, x, C=128)
+    assert rel_l2(o2, o1) <= 2 * TOL[torch.bfloat16] and rel_l2(S2, S1) <= 2 * TOL[torch.bfloat16]
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_gate_zero_and_one(dn, oracle_mod, dtype):
     x = gen.make_inputs(1, 2, 190, 128, 128, dtype, gated=True, seed=8)
