@@ -243,13 +243,13 @@ def traffic_from_profile():
         return None
     vals = {}
     for line in open(p):
-        if line.startswith("traffic_bytes_per_launch:") or line.startswith("kernel_source_hash:"):
+        if line.startswith("traffic_bytes_per_call:") or line.startswith("kernel_source_hash:"):
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
     if vals.get("kernel_source_hash") != kernel_hash():
         return None
     try:
-        return float(vals["traffic_bytes_per_launch"])
+        return float(vals["traffic_bytes_per_call"])
     except (KeyError, ValueError):
         return None
 
