@@ -106,8 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sb = warp_uniform(smem_u32(sm));
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = (int)warp_uniform((uint32_t)tid >> 5);
   const int bh = blockIdx.x;
   const int j0 = blockIdx.y * kDVS;
   const int T = p.T, Dv = p.Dv;
@@ -122,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* zc = zs + 128;                                  // chunk column sums of K', DK
   float* dq = zc + 128;                                  // Q' z per row, 64
   float* rs = dq + 64;                                   // row sums of P, 64
+  // partial column sums of K' per row group: [128 / (DK / 8)][DK]
+  float* red = reinterpret_cast<float*>(sm + L::AM_OFF + 4096);
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = warp_uniform(*tmem_slot);
   const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
 
   if (warp == 4) {
@@ -223,15 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       bar_compute();
 
-      if (tid == 0) {
+      if (warp == 0) {  // warp-uniform issue, one elected lane
         tc_fence_after();
         constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::K_OFF + (ks & 3) * 32;
-          mma_bf16_ss(tmem + TM_G, kdesc(a), kdesc(a), id, ks > 0);
+          mma_bf16_ss_elect(tmem + TM_G, kdesc(a), kdesc(a), id, ks > 0);
         }
-        mma_commit(bar_mma);
+        mma_commit_elect(bar_mma);
       }
       // meanwhile: Q' z per row (threads 0-63) and K' column sums (threads < DK)
       if (tid < 64) {
@@ -250,13 +253,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         dq[row] = acc;
       }
-      if (tid < DK) {
-        const uint8_t* kt = stp + (tid >> 6) * L::KB_STRIDE + L::K_OFF;
-        const int c16 = (tid & 63) >> 3, e = tid & 7;
-        float acc = 0.f;
-        for (int r = 0; r < n; ++r)
-          acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kt + sw128_off(r, c16) + 2 * e));
-        zc[tid] = acc;
+      {  // partial column sums of K' (rows past n are zero): thread -> (8 columns, row group)
+        constexpr int kCC = DK / 8, kRG = kCompute / kCC, kRows = kC / kRG;
+        const int cc = tid % kCC, rg = tid / kCC;
+        const uint8_t* kt = stp + (cc >> 3) * L::KB_STRIDE + L::K_OFF;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+          const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_off(rg * kRows + i, cc & 7));
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[rg * DK + cc * 8 + e] = acc[e];
       }
       ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
       ++mma_count;
@@ -290,24 +304,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_compute();
 
       // ---- O = Q'S + P V (lanes 0-63), dS = K'^T V ----
-      if (tid == 0) {
+      if (warp == 0) {  // warp-uniform issue, one elected lane
         tc_fence_after();
         constexpr uint32_t ido = idesc_bf16(128, 64, false, true);
         constexpr uint32_t ids = idesc_bf16(128, 64, true, true);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-          mma_bf16_ss(tmem + TM_QW, kdesc(a), mndesc(sb + L::S_OFF + ks * 2048, kTile), ido, ks > 0);
+          mma_bf16_ss_elect(tmem + TM_QW, kdesc(a), mndesc(sb + L::S_OFF + ks * 2048, kTile), ido, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ss(tmem + TM_QW, kdesc(sb + L::PT_OFF + ks * 32),
-                      mndesc(st + L::V_OFF + ks * 2048, kTile), ido, 1);
-          mma_bf16_ss(tmem + TM_DS, mndesc(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                      mndesc(st + L::V_OFF + ks * 2048, kTile), ids, ks > 0);
+          mma_bf16_ss_elect(tmem + TM_QW, kdesc(sb + L::PT_OFF + ks * 32),
+                            mndesc(st + L::V_OFF + ks * 2048, kTile), ido, 1);
+          mma_bf16_ss_elect(tmem + TM_DS, mndesc(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                            mndesc(st + L::V_OFF + ks * 2048, kTile), ids, ks > 0);
         }
-        mma_commit(bar_mma);
-        mma_commit(bar_empty0 + 8 * s);
+        mma_commit_elect(bar_mma);
+        mma_commit_elect(bar_empty0 + 8 * s);
       }
       ok = bar_and(mbar_wait(bar_mma, mma_count & 1, wc));
       ++mma_count;
@@ -349,7 +363,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       bar_compute();  // every read of the old z is done
-      if (tid < DK) zs[tid] += zc[tid];
+      if (tid < DK) {
+        constexpr int kRG = kCompute / (DK / 8);
+        float a = 0.f;
+#pragma unroll
+        for (int rg = 0; rg < kRG; ++rg) a += red[rg * DK + tid];
+        zs[tid] += a;
+      }
     }
 
     if (tid < DK) {
@@ -361,9 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (p.z_out && blockIdx.y == 0) p.z_out[(size_t)bh * DK + tid] = zs[tid];
     }
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
-      mma_commit(bar_fin);
+      mma_commit_elect(bar_fin);
       int zero = 0;
       const WaitCtl fin{&zero, p.status, kWaitLimitNs};
       (void)mbar_wait(bar_fin, 0, fin);
