@@ -433,8 +433,9 @@ def profile_run(args):
 
     dev = torch.device("cuda", 0)
     n = args.warmup + 1
-    if args.profile in ("chunk", "gated", "linear"):
-        w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR}[args.profile]
+    if args.profile in ("chunk", "gated", "linear", "long64", "long128"):
+        w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR,
+             "long64": gen.LONG64, "long128": gen.LONG128}[args.profile]
         x = gen.make_workload(w, seed=0, device=dev)
         for _ in range(n):
             if args.profile == "linear":
@@ -462,7 +463,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--profile", choices=["chunk", "linear", "gated", "decode"], default=None,
+    ap.add_argument("--profile", choices=["chunk", "linear", "gated", "long64", "long128", "decode"],
+                    default=None,
                     help="untimed run for a profiler: --warmup launches of one kernel on its "
                          "workload, then one more (the one to capture)")
     args = ap.parse_args()
