@@ -31,8 +31,6 @@ namespace {
 
 using namespace nvcuda;
 
-constexpr int kKpad = 8;  // bf16 padding of the K rows (keeps WMMA rows 16-byte aligned)
-
 template <int C>
 struct TsolveShape {
   static constexpr int kThreads = 2 * C;       // one warp per 16-row block
@@ -42,12 +40,23 @@ struct TsolveShape {
   static_assert(kWarps == C / 16, "one warp per 16-row block");
 };
 
+// Shared memory: the K tile (128-byte swizzled, KB blocks of C rows x 128 B,
+// from TMA) shares its region with T, which is written only after the Gram has
+// read K; A follows.  At C = 64 the M = 128 Gram operand's rows 64-127 read
+// whatever follows a block (still inside this CTA's shared memory; those TMEM
+// rows are not used).
 template <int C, int DK>
-constexpr size_t tsolve_smem_bytes() {
-  return (C * (DK + kKpad) * 2 > C * TsolveShape<C>::kApad * 4 ? C * (DK + kKpad) * 2
-                                                                : C * TsolveShape<C>::kApad * 4) +
-         (size_t)C * TsolveShape<C>::kApad * 4 + (3 * C + 8) * 4;
-}
+struct TsolveSmem {
+  static constexpr uint32_t kKBytes = (DK / 64) * C * 128;
+  static constexpr uint32_t kTBytes = C * TsolveShape<C>::kApad * 4;
+  static constexpr uint32_t kRegion = ((kKBytes > kTBytes ? kKBytes : kTBytes) + 1023) / 1024 * 1024;
+  static constexpr uint32_t AM_OFF = kRegion;
+  static constexpr uint32_t VEC_OFF = AM_OFF + kTBytes;  // beta, g, e^g (C each), 8 warp totals
+  static constexpr uint32_t BAR_OFF = (VEC_OFF + (3 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
+  static constexpr uint32_t BYTES = BAR_OFF + 32;
+  static constexpr uint32_t ALLOC = BYTES + 1024;  // 1024-byte alignment of the K tile
+  static_assert(C == 128 || kRegion + 8192 <= BYTES, "M = 128 operand rows past the K tile stay inside");
+};
 
 // tf32 operands by truncation: keep the sign, exponent and top 10 mantissa bits
 // (round toward zero, relative error < 2^-10; the factors leave this kernel
@@ -59,65 +68,92 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
 }
 
 template <int C, int DK, bool GATED>
-__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1) tsolve_kernel(const __nv_bfloat16* __restrict__ k,
-                                                          const float* __restrict__ beta,
-                                                          const float* __restrict__ alpha,
-                                                          __nv_bfloat16* __restrict__ tb_out,
-                                                          __nv_bfloat16* __restrict__ tbg_out,
-                                                          float* __restrict__ g_out, int T,
-                                                          int nchunks) {
+__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
+    tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
+                  const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
+                  __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out, int T, int nchunks,
+                  unsigned int* status) {
   using Sh = TsolveShape<C>;
+  using SL = TsolveSmem<C, DK>;
   constexpr int kC = C, kThreads = Sh::kThreads, kApad = Sh::kApad;
-  constexpr int KS = DK + kKpad;
-  constexpr int kRegion = (kC * KS * 2 > kC * kApad * 4) ? kC * KS * 2 : kC * kApad * 4;
-  extern __shared__ __align__(128) uint8_t tsolve_smem[];
-  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(tsolve_smem);
-  float* Tm = reinterpret_cast<float*>(tsolve_smem);  // reuses the K tile after the Gram
-  float* Am = reinterpret_cast<float*>(tsolve_smem + kRegion);
-  float* vb = Am + kC * kApad;
+  extern __shared__ uint8_t tsolve_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsolve_smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = warp_uniform(smem_u32(sm));
+  float* Tm = reinterpret_cast<float*>(sm);  // reuses the K tile after the Gram
+  float* Am = reinterpret_cast<float*>(sm + SL::AM_OFF);
+  float* vb = reinterpret_cast<float*>(sm + SL::VEC_OFF);
   float* vg = vb + kC;
   float* veg = vg + kC;
   float* wsum = veg + kC;  // per-warp totals of the log-decay scan
+  const uint32_t bar_full = sb + SL::BAR_OFF, bar_mma = sb + SL::BAR_OFF + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SL::BAR_OFF + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SL::BAR_OFF + 20);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int warp = (int)warp_uniform((uint32_t)tid >> 5);
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int c0 = chunk * kC, n = min(kC, T - c0);
 
-  // 1. K tile, beta and the log-decay prefix g (rows >= n: k = 0, beta = 0, alpha = 1).
-  //    Every thread's K loads are issued before any is stored (all in flight at
-  //    once), and the beta / alpha loads overlap them.
-  constexpr int kVecPerRow = DK / 8;
-  constexpr int kLoads = kC * kVecPerRow / kThreads;
-  uint4 kreg[kLoads];
+  // 1. K tile by TMA (rows past T read as zero), beta and the log-decay prefix g
+  //    (rows >= n: beta = 0, alpha = 1) while it lands.
+  if (tid == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kC);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = warp_uniform(*tmem_slot);
+  const WaitCtl wc{abort_flag, status, kWaitLimitNs};
+  if (tid == 0) {
+    mbar_expect_tx(bar_full, (uint32_t)SL::kKBytes);
+#pragma unroll
+    for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+      for (int rb = 0; rb < kC / 64; ++rb)
+        tma_load_3d(sb + kb * (kC * 128) + rb * 8192, &tmK, bar_full, kb * 64, c0 + rb * 64, bh);
+  }
   float glog = 0.f;
-  {
-    const __nv_bfloat16* src = k + ((size_t)bh * T + c0) * DK;
+  if (tid < kC) {
+    const size_t tb = (size_t)bh * T + c0;
+    vb[tid] = tid < n ? beta[tb + tid] : 0.f;
+    if (GATED) {  // inclusive scan of max(log alpha, -87) within each warp
+      glog = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
 #pragma unroll
-    for (int it = 0; it < kLoads; ++it) {
-      const int i = tid + it * kThreads;
-      const int r = i / kVecPerRow, v = i % kVecPerRow;
-      kreg[it] = r < n ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * DK) + v)
-                       : make_uint4(0, 0, 0, 0);
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, glog, off);
+        if (lane >= off) glog += y;
+      }
+      if (lane == 31) wsum[warp] = glog;
     }
-    if (tid < kC) {
-      const size_t tb = (size_t)bh * T + c0;
-      vb[tid] = tid < n ? beta[tb + tid] : 0.f;
-      if (GATED) {  // inclusive scan of max(log alpha, -87) within each warp
-        glog = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
+  }
+  // 2. G = K K^T on the tensor cores (M = 128, N = C, into TMEM), issued by one
+  //    elected lane of warp 0 once the tile has landed.
+  bool ok = true;
+  if (warp == 0) {
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_full, 0, wc));
+    if (!ok && lane == 0) {  // never leave with the copy in flight
+      int zero = 0;
+      const WaitCtl drain{&zero, status, kWaitLimitNs};
+      (void)mbar_wait(bar_full, 0, drain);
+    }
+    if (ok) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16(128, kC, false, false);
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, glog, off);
-          if (lane >= off) glog += y;
-        }
-        if (lane == 31) wsum[warp] = glog;
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        const uint32_t a = sb + (ks >> 2) * (kC * 128) + (ks & 3) * 32;
+        mma_bf16_ss_elect(tmem, desc_k(a), desc_k(a), id, ks > 0);
       }
     }
-#pragma unroll
-    for (int it = 0; it < kLoads; ++it) {
-      const int i = tid + it * kThreads;
-      const int r = i / kVecPerRow, v = i % kVecPerRow;
-      *reinterpret_cast<uint4*>(Ks + r * KS + v * 8) = kreg[it];
-    }
+    mma_commit_elect(bar_mma);  // arrives even with no MMA in flight
   }
   __syncthreads();
   if (GATED) {  // add the totals of the earlier warps: g = cumsum over the chunk
@@ -129,44 +165,38 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1) tsolve_kernel(const __
     }
     __syncthreads();
   }
-
-  // 2. G = K K^T (lower 16x16 tiles only, spread over the warps), straight into A,
-  //    and each warp turns its own tiles into A = strict_lower(diag(beta) G * Gamma).
-  //    Nothing reads A's upper tiles or T's strictly-upper tiles unmasked (the
-  //    diagonal solve writes whole diagonal tiles, the block solve reads tiles on
-  //    or below the diagonal, the output masks by column <= row).
-  {
-    wmma::fragment<wmma::matrix_a, 16, 16, 16, __nv_bfloat16, wmma::row_major> fa;
-    wmma::fragment<wmma::matrix_b, 16, 16, 16, __nv_bfloat16, wmma::col_major> fb;
-    wmma::fragment<wmma::accumulator, 16, 16, 16, float> acc;
-    for (int t = warp; t < Sh::kTiles; t += Sh::kWarps) {
-      // t -> (ti, tj), tj <= ti, row-major over the lower triangle of tiles
-      int ti = 0;
-      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-      const int tj = t - ti * (ti + 1) / 2;
-      wmma::fill_fragment(acc, 0.f);
+  //    A = strict_lower(diag(beta) G * Gamma): TMEM row r -> A row r (64 columns
+  //    per thread).  Nothing reads A's upper part or T's strictly-upper tiles
+  //    unmasked (the diagonal solve writes whole diagonal tiles, the block
+  //    solve reads tiles on or below the diagonal, the output masks by column).
+  ok = mbar_wait(bar_mma, 0, wc) && ok;
+  tc_fence_after();
+  if (tid < (kC == 64 ? 64 : 256)) {
+    const int r = tid & 127;  // = 32 (warp % 4) + lane: this warp's TMEM lanes
+    const int col0 = (kC == 128) ? (tid >> 7) * 64 : 0;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const float br = vb[r], gr = GATED ? vg[r] : 0.f;
+    float* arow = Am + r * kApad + col0;
 #pragma unroll
-      for (int kk = 0; kk < DK; kk += 16) {
-        wmma::load_matrix_sync(fa, Ks + (16 * ti) * KS + kk, KS);
-        wmma::load_matrix_sync(fb, Ks + (16 * tj) * KS + kk, KS);
-        wmma::mma_sync(acc, fa, fb, acc);
-      }
-      wmma::store_matrix_sync(Am + (16 * ti) * kApad + 16 * tj, acc, kApad, wmma::mem_row_major);
-      __syncwarp();
+    for (int q = 0; q < 2; ++q) {
+      uint32_t gv[32];
+      tmem_ld32(tmem + lane_base + col0 + q * 32, gv);
+      tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        const int r = 16 * ti + (e >> 4), c = 16 * tj + (e & 15);
-        float* ap = Am + r * kApad + c;
-        float a = 0.f;
-        if (c < r) {
-          a = vb[r] * *ap;
-          if (GATED) a *= __expf(vg[r] - vg[c]);
+      for (int e4 = 0; e4 < 32; e4 += 4) {
+        float a4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = col0 + q * 32 + e4 + e;
+          float a = br * __uint_as_float(gv[e4 + e]);
+          if (GATED) a *= __expf(gr - vg[c]);
+          a4[e] = c < r ? a : 0.f;
         }
-        *ap = a;
+        *reinterpret_cast<float4*>(arow + q * 32 + e4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
       }
     }
   }
+  tc_fence_before();
   __syncthreads();
 
   // 3. T = (I + A)^-1.  Diagonal 16x16 blocks D_w: warp w, lanes 0-15 own
@@ -249,6 +279,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1) tsolve_kernel(const __
       if (GATED) st_bf16x8(tbg_out + tile + row * kC + c8, y);
     }
   }
+  if (warp == 0) tmem_dealloc(tmem, kC);  // every TMEM read finished before the last barrier
   // The chunk kernel may begin launching once every CTA got here (it still
   // waits for this grid to complete before reading the factors).
   grid_launch_dependents();
@@ -257,13 +288,15 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1) tsolve_kernel(const __
 template <int C, int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   const int nchunks = (p.T + C - 1) / C;
-  constexpr size_t smem = tsolve_smem_bytes<C, DK>();
+  constexpr size_t smem = TsolveSmem<C, DK>::ALLOC;
+  CUtensorMap mk;
+  if (!make_tmap_3d_bf16(&mk, p.k, DK, p.T, p.B * p.H)) return cudaErrorInvalidValue;
   auto kern = tsolve_kernel<C, DK, GATED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)nchunks, (unsigned)(p.B * p.H));
-  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(p.k), p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks);
+  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks,
+                                                      p.status);
   return cudaGetLastError();
 }
 
