@@ -36,7 +36,6 @@ struct TsolveShape {
   static constexpr int kThreads = 2 * C;       // one warp per 16-row block
   static constexpr int kWarps = kThreads / 32;  // == C / 16
   static constexpr int kApad = C + 4;           // float row stride of the A / T scratch
-  static constexpr int kTiles = kWarps * (kWarps + 1) / 2;  // lower 16x16 tiles of the Gram
   static_assert(kWarps == C / 16, "one warp per 16-row block");
 };
 
@@ -75,7 +74,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
                   unsigned int* status) {
   using Sh = TsolveShape<C>;
   using SL = TsolveSmem<C, DK>;
-  constexpr int kC = C, kThreads = Sh::kThreads, kApad = Sh::kApad;
+  constexpr int kC = C, kApad = Sh::kApad;
   extern __shared__ uint8_t tsolve_smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsolve_smem_raw) + 1023) &
                                            ~uintptr_t(1023));
