@@ -10,21 +10,23 @@
 //   P = tril(Q' K'^T)                                (M = 128 MMA [K'; Q'] K'^T)
 //   O = (Q' S + P V) / (Q' z + P 1)                  (Q'S + PV in one TMEM tile)
 //   S <- S + K'^T V,  z <- z + K'^T 1
-// Only S (and z) carry from chunk to chunk, and S's update K'^T V does not
-// depend on S, so everything but the state accumulate is pipelined ahead of it.
+// The normaliser rides along in the products: V is augmented with a column of
+// ones and S with z as an extra column ([V | 1], [S | z], N = 80), so K'^T [V|1]
+// gives both state increments, Q'[S|z] + P[V|1] both numerator and
+// denominator.  Only S and z carry from chunk to chunk, and their increment
+// does not depend on them, so everything but the accumulate is pipelined ahead.
 //
 // One CTA per (b, h, 64-column slice of Dv), 10 warps:
 //   warp 8     producer: TMA of K, Q, V into a three-stage ring
 //   warp 9     MMA issuer (warp-uniform, one elected lane): Gram (c+1) and
-//              K'^T V (c+1) while chunk c waits for its state tile, then
-//              O (c) = Q'S + PV
-//   warps 4-7  prep: feature maps in place, K' column sums, Q' z per row,
-//              P rows to bf16 with their row sums (warps 6-7, TMEM lanes
-//              64-127)
-//   warps 0-3  state: S += K'^T V in float32 registers, the bf16 state tile
-//              for the next chunk (double-buffered); warps 0-1 also drain
-//              O / (Q' z + P 1) to global memory
-// Accumulators live in TMEM (G[2], dS[2], O[2]: 384 of 512 columns).  Every
+//              K'^T [V|1] (c+1) while chunk c waits for its state tile, then
+//              O (c) = Q'[S|z] + P[V|1]
+//   warps 4-7  prep: feature maps in place (rows past T zeroed)
+//   warps 0-3  state: [S|z] += K'^T [V|1] in float32 registers, the bf16
+//              state tile for the next chunk (double-buffered); warps 2-3 turn
+//              the Gram rows (TMEM lanes 64-127) into P; warps 0-1 drain
+//              O / (Q'z + P 1) to global memory
+// Accumulators live in TMEM (G[2], dS[2], O[2]: 448 of 512 columns).  Every
 // mbarrier completes once per chunk or per use of a parity, so parity waits
 // are unambiguous.  All waits are bounded; a wait that runs out sets the
 // status word and the CTA winds down (copies drained, MMAs retired, TMEM
@@ -44,10 +46,11 @@ constexpr int NST = 3;
 constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
 constexpr int kWG = 128;
 constexpr int kThreads = 2 * kWG + 64;  // state 0-3, prep 4-7, producer 8, issuer 9
-constexpr int kBarState = 1, kBarLo = 2, kBarPrep = 3, kBarPrepHi = 4;
+constexpr int kBarState = 1, kBarLo = 2, kBarHi = 3, kBarPrep = 4;
+constexpr int kNA = 80;  // augmented width: 64 columns of V (or S) + the ones (or z) column, padded to 16
 
-// TMEM columns: Gram[2] (lanes 64-127: Q'K'^T), dS[2] (K'^T V), O[2] (lanes 0-63)
-constexpr uint32_t TM_G = 0, TM_DS = 128, TM_O = 256;
+// TMEM columns: Gram[2] (lanes 64-127: Q'K'^T), dS[2] (K'^T [V|1]), O[2] (lanes 0-63)
+constexpr uint32_t TM_G = 0, TM_DS = 128, TM_O = 320, kAugStride = 96;
 
 template <int DK>
 struct LinLayout {
@@ -56,22 +59,23 @@ struct LinLayout {
   static constexpr uint32_t K_OFF = 0, Q_OFF = kTile;
   static constexpr uint32_t V_OFF = KB * KB_STRIDE;
   static constexpr uint32_t STAGE = V_OFF + kTile;
-  static constexpr uint32_t P_OFF = NST * STAGE;           // P[2]
-  static constexpr uint32_t S_OFF = P_OFF + 2 * kTile;     // bf16 state tiles [2], DK rows x 128 B
-  static constexpr uint32_t Z_OFF = S_OFF + 2 * DK * 128;  // z (DK), Q'z [2][64], row sums [2][64]
-  static constexpr uint32_t RED_OFF = Z_OFF + (DK + 4 * 64) * 4;  // K' column partial sums [16][DK]
-  static constexpr uint32_t BAR_OFF = RED_OFF + 16 * DK * 4;
+  static constexpr uint32_t ONES_OFF = NST * STAGE;       // 64 x 64 bf16: column 0 ones, rest zero
+  static constexpr uint32_t P_OFF = ONES_OFF + kTile;      // P[2]
+  // bf16 [S | z] tiles [2]: block 0 = S (DK rows x 128 B), block 1 = z in column 0
+  static constexpr uint32_t SBLK = DK * 128;
+  static constexpr uint32_t S_OFF = P_OFF + 2 * kTile;
+  static constexpr uint32_t BAR_OFF = S_OFF + 4 * SBLK;
   static constexpr uint32_t BYTES = BAR_OFF + 256;
   static constexpr uint32_t ALLOC = BYTES + 1024;
   static_assert(STAGE % 1024 == 0 && P_OFF % 1024 == 0, "128-byte swizzle atoms stay aligned");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
-// mbarrier slots (8 bytes each).  FULL / EMPTY per stage; the rest per chunk
-// parity except FMAP (once per chunk, never two phases ahead of its waiter).
-constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_GDONE = 48, B_DSDONE = 64, B_PREADY = 80,
-                   B_DSFREE = 96, B_SREADY = 112, B_ODONE = 128, B_OFREE = 144, B_FMAP = 160,
-                   B_FIN = 168, B_TMEM = 176, B_ABORT = 180;
+// mbarrier slots (8 bytes each).  FULL, EMPTY and FMAP per stage; the rest per
+// chunk parity.
+constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_FMAP = 48, B_GDONE = 72, B_DSDONE = 88, B_PREADY = 104,
+                   B_DSFREE = 120, B_SREADY = 136, B_ODONE = 152, B_OFREE = 168, B_FIN = 184,
+                   B_TMEM = 192, B_ABORT = 196;
 
 // ELU(x) + 1: x + 1 for x > 0, and e^x (= (e^x - 1) + 1) otherwise.
 __device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
@@ -94,15 +98,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar = sb + L::BAR_OFF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::BAR_OFF + B_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR_OFF + B_ABORT);
-  float* zs = reinterpret_cast<float*>(sm + L::Z_OFF);  // z entering the chunk the prep is on
-  float* dq = zs + DK;                                   // Q' z per row, [2][64]
-  float* rs = dq + 128;                                  // row sums of P, [2][64]
-  float* red = reinterpret_cast<float*>(sm + L::RED_OFF);
 
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(bar + B_FULL + 8 * i, 1);
       mbar_init(bar + B_EMPTY + 8 * i, 1);
+      mbar_init(bar + B_FMAP + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + B_GDONE + 8 * i, 1);
@@ -113,11 +114,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar + B_ODONE + 8 * i, 1);
       mbar_init(bar + B_OFREE + 8 * i, 1);
     }
-    mbar_init(bar + B_FMAP, 1);
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // constant column of ones next to V; the z blocks of the state tiles start at zero
+  for (int i = tid; i < (int)(kTile / 16); i += kThreads) {
+    const int r = i >> 3, c16 = i & 7;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (c16 == 0) u.x = 0x3F80u;  // bf16 1.0 in the first element of the row's first chunk
+    *reinterpret_cast<uint4*>(sm + L::ONES_OFF + sw128_off(r, c16)) = u;
+  }
+  for (int i = tid; i < (int)(2 * L::SBLK / 16); i += kThreads)
+    *reinterpret_cast<uint4*>(sm + L::S_OFF + (i / (L::SBLK / 16)) * 2 * L::SBLK + L::SBLK +
+                              (i % (L::SBLK / 16)) * 16) = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -177,32 +188,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_bf16_ss_elect(tmem + TM_G + 64 * b, desc_k(a), desc_k(a), idg, ks > 0);
       }
       mma_commit_elect(bar + B_GDONE + 8 * b);
-      constexpr uint32_t idd = idesc_bf16(128, 64, true, true);
+      constexpr uint32_t idd = idesc_bf16(128, kNA, true, true);
+      const uint32_t ones_lbo = sb + L::ONES_OFF - (st + L::V_OFF);  // [V | 1]: the ones block follows V
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_DS + 64 * b, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                          desc_mn(st + L::V_OFF + ks * 2048, kTile), idd, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_DS + kAugStride * b, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+                          desc_mn(st + L::V_OFF + ks * 2048, ones_lbo), idd, ks > 0);
       mma_commit_elect(bar + B_DSDONE + 8 * b);
     };
-    // O (c) = Q' S + P V into O[c & 1] (lanes 0-63)
+    // O (c) = Q' [S|z] + P [V|1] into O[c & 1] (lanes 0-63)
     auto issue_o = [&](int c) {
       const uint32_t st = stage(c);
       const int b = c & 1;
-      constexpr uint32_t ido = idesc_bf16(128, 64, false, true);
+      constexpr uint32_t ido = idesc_bf16(128, kNA, false, true);
+      const uint32_t ones_lbo = sb + L::ONES_OFF - (st + L::V_OFF);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
         const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem + TM_O + 64 * b, desc_k(a),
-                          desc_mn(sb + L::S_OFF + b * (DK * 128) + ks * 2048, kTile), ido, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_k(a),
+                          desc_mn(sb + L::S_OFF + b * 2 * L::SBLK + ks * 2048, L::SBLK), ido, ks > 0);
       }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_O + 64 * b, desc_k(sb + L::P_OFF + b * kTile + ks * 32),
-                          desc_mn(st + L::V_OFF + ks * 2048, kTile), ido, 1);
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_k(sb + L::P_OFF + b * kTile + ks * 32),
+                          desc_mn(st + L::V_OFF + ks * 2048, ones_lbo), ido, 1);
       mma_commit_elect(bar + B_ODONE + 8 * b);
       mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));  // stage c: Gram, dS and O have read it
     };
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP, 0, wc));
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP, 0, wc));  // stage 0, first use
     if (ok) {
       tc_fence_after();
       issue_gram_ds(0);
@@ -212,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c + 1 < nchunks) {  // the next chunk's Gram and K'^T V run while chunk c waits for its state
         // G[(c+1) & 1] was read by the P rows of chunk c-1 (PREADY waited below in
         // iteration c-1); dS[(c+1) & 1] must have been added to S (DSFREE of chunk c-1)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP, (c + 1) & 1, wc) &&
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc) &&
                                          (c < 1 || mbar_wait(bar + B_DSFREE + 8 * (b ^ 1), ((c - 1) >> 1) & 1, wc)));
         if (!ok) break;
         tc_fence_after();
@@ -234,119 +247,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- prep --
     const int pt = tid - kWG;
-    const int row = pt & 63;
-    if (pt < DK) zs[pt] = p.z0 ? p.z0[(size_t)bh * DK + pt] : 0.f;
-    bool ok = true, okp = true;
+    bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
-      const int b = c & 1;
       const int n = min(kC, T - c * kC);
       uint8_t* stp = sm + (c % NST) * L::STAGE;
-      ok = named_bar_and(kBarPrep, kWG, okp && mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
+      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
-      // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0) ----
+      // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0), 4 pieces in flight ----
       constexpr int kPieces = L::KB * 2 * (int)(kTile / 16);  // 16-byte pieces of the K and Q tiles
-      for (int i = pt; i < kPieces; i += kWG) {
-        const int t16 = i / (int)(kTile / 16), off = (i % (int)(kTile / 16)) * 16;
-        uint8_t* ptr = stp + (t16 >> 1) * L::KB_STRIDE + (t16 & 1) * kTile + off;
-        uint4 u = *reinterpret_cast<uint4*>(ptr);
-        if ((off >> 7) >= n) {
-          u = make_uint4(0, 0, 0, 0);
-        } else {
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+      static_assert(kPieces % (4 * kWG) == 0, "whole rounds of four pieces per thread");
+      for (int i0 = pt; i0 < kPieces; i0 += 4 * kWG) {
+        uint4 u[4];
+        uint8_t* ptr[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack2_bf16(elu1(f.x), elu1(f.y));
-          }
+        for (int j = 0; j < 4; ++j) {
+          const int i = i0 + j * kWG;
+          const int t16 = i / (int)(kTile / 16), off = (i % (int)(kTile / 16)) * 16;
+          ptr[j] = stp + (t16 >> 1) * L::KB_STRIDE + (t16 & 1) * kTile + off;
+          u[j] = (off >> 7) < n ? *reinterpret_cast<const uint4*>(ptr[j]) : make_uint4(0, 0, 0, 0);
         }
-        *reinterpret_cast<uint4*>(ptr) = u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int off = ((i0 + j * kWG) % (int)(kTile / 16)) * 16;
+          if ((off >> 7) < n) {
+            uint32_t* w = reinterpret_cast<uint32_t*>(&u[j]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+              w[e] = pack2_bf16(elu1(f.x), elu1(f.y));
+            }
+          }
+          *reinterpret_cast<uint4*>(ptr[j]) = u[j];
+        }
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPrep, kWG);
-      if (pt == 0) mbar_arrive(bar + B_FMAP);
-      {  // partial column sums of K': thread -> (8 columns, row group)
-        constexpr int kCC = DK / 8, kRG = kWG / kCC, kRows = kC / kRG;
-        const int cc = pt % kCC, rg = pt / kCC;
-        const uint8_t* kt = stp + (cc >> 3) * L::KB_STRIDE + L::K_OFF;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-          const uint4 u = *reinterpret_cast<const uint4*>(kt + sw128_off(rg * kRows + i, cc & 7));
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-            acc[2 * e] += f.x;
-            acc[2 * e + 1] += f.y;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) red[rg * DK + cc * 8 + e] = acc[e];
-      }
-      // ---- Q' z per row, z entering chunk c (dq[b] was read by the output of chunk c-2) ----
-      bool okq = true;
-      if (pt < 64) {
-        okq = c < 2 || mbar_wait(bar + B_OFREE + 8 * b, ((c >> 1) - 1) & 1, wc);
-        float acc = 0.f;
-#pragma unroll
-        for (int c16 = 0; c16 < DK / 8; ++c16) {
-          const uint4 u = *reinterpret_cast<const uint4*>(stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF +
-                                                          sw128_off(row, c16 & 7));
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-            acc = fmaf(f.x, zs[c16 * 8 + 2 * e], acc);
-            acc = fmaf(f.y, zs[c16 * 8 + 2 * e + 1], acc);
-          }
-        }
-        dq[b * 64 + row] = acc;
-      }
-      ok = named_bar_and(kBarPrep, kWG, okq);  // every read of the old z is done
-      if (!ok) break;
-      if (pt < DK) {
-        constexpr int kRG = kWG / (DK / 8);
-        float a = 0.f;
-#pragma unroll
-        for (int rg = 0; rg < kRG; ++rg) a += red[rg * DK + pt];
-        zs[pt] += a;
-      }
-      // ---- P rows (TMEM lanes 64-127) to bf16, with their sums ----
-      if (pt >= 64) {
-        okp = named_bar_and(kBarPrepHi, 64, mbar_wait(bar + B_GDONE + 8 * b, (c >> 1) & 1, wc));
-        if (okp) {
-          tc_fence_after();
-          uint32_t g[64];
-          tmem_ld32(tmem + lane_base + TM_G + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(g));
-          tmem_ld32(tmem + lane_base + TM_G + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
-          tmem_wait_ld();
-          float sum = 0.f;
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int sc = c16 * 8 + e;
-              x[e] = sc <= row ? __uint_as_float(g[sc]) : 0.f;
-              sum += x[e];
-            }
-            st_bf16x8(sm + L::P_OFF + b * kTile + sw128_off(row, c16), x);
-          }
-          rs[b * 64 + row] = sum;
-          fence_proxy_async_smem();
-          tc_fence_before();
-          named_bar_sync(kBarPrepHi, 64);
-          if (pt == 64) mbar_arrive(bar + B_PREADY + 8 * b);
-        }
-      }
+      if (pt == 0) mbar_arrive(bar + B_FMAP + 8 * (c % NST));
     }
-    if (p.z_out && blockIdx.y == 0 && pt < DK) p.z_out[(size_t)bh * DK + pt] = zs[pt];
   } else {
     // --------------------------------------------------------------- state --
     const int ct = tid;
     const int row = ct & 63;
     const size_t s_base = (size_t)bh * DK * Dv;
-    float sreg[kDVS];
+    float sreg[kDVS], zreg = 0.f;
+    // one row of [S | z] as bf16 into tile t (z in column 0 of the second block)
+    auto put_state = [&](int t) {
+      uint8_t* tile = sm + L::S_OFF + t * 2 * L::SBLK;
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(tile + sw128_off(ct, c16), sreg + 8 * c16);
+      const float zrow[8] = {zreg, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      st_bf16x8(tile + L::SBLK + sw128_off(ct, 0), zrow);
+    };
     if (ct < DK) {
       const float* src = p.S0 ? p.S0 + s_base + (size_t)ct * Dv + j0 : nullptr;
 #pragma unroll
@@ -354,28 +305,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
       }
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
+      zreg = p.z0 ? p.z0[(size_t)bh * DK + ct] : 0.f;
+      put_state(0);
     }
     fence_proxy_async_smem();
     named_bar_sync(kBarState, kWG);
     if (ct == 0) mbar_arrive(bar + B_SREADY);  // the state entering chunk 0, in tile 0
 
-    bool ok = true, ok_lo = true;
+    bool ok = true, ok_lo = true, ok_hi = true;
     for (int c = 0; c < nchunks && ok; ++c) {
       const int b = c & 1;
       const int n = min(kC, T - c * kC);
-      // ---- S += K'^T V (c) ----
-      ok = named_bar_and(kBarState, kWG, ok_lo && mbar_wait(bar + B_DSDONE + 8 * b, (c >> 1) & 1, wc));
+      // ---- P = tril(Q'K'^T) rows (TMEM lanes 64-127) to bf16 (warps 2-3) ----
+      if (ct >= 64) {
+        ok_hi = named_bar_and(kBarHi, 64, mbar_wait(bar + B_GDONE + 8 * b, (c >> 1) & 1, wc));
+        if (ok_hi) {
+          tc_fence_after();
+          uint32_t g[64];
+          tmem_ld32(tmem + lane_base + TM_G + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(g));
+          tmem_ld32(tmem + lane_base + TM_G + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
+          tmem_wait_ld();
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int sc = c16 * 8 + e;
+              x[e] = sc <= row ? __uint_as_float(g[sc]) : 0.f;
+            }
+            st_bf16x8(sm + L::P_OFF + b * kTile + sw128_off(row, c16), x);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          named_bar_sync(kBarHi, 64);
+          if (ct == 64) mbar_arrive(bar + B_PREADY + 8 * b);
+        }
+      }
+      // ---- [S | z] += K'^T [V | 1] (c) ----
+      ok = named_bar_and(kBarState, kWG,
+                         ok_hi && ok_lo && mbar_wait(bar + B_DSDONE + 8 * b, (c >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
       if (ct < DK) {
-        uint32_t ds[64];
-        tmem_ld32(tmem + lane_base + TM_DS + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(ds));
-        tmem_ld32(tmem + lane_base + TM_DS + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
+        const uint32_t d0 = tmem + lane_base + TM_DS + kAugStride * b;
+        uint32_t ds[64], dz[32];
+        tmem_ld32(d0, *reinterpret_cast<uint32_t(*)[32]>(ds));
+        tmem_ld32(d0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
+        tmem_ld32(d0 + 64, dz);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 64; ++e) sreg[e] += __uint_as_float(ds[e]);
+        zreg += __uint_as_float(dz[0]);
       }
       tc_fence_before();
       named_bar_sync(kBarState, kWG);
@@ -385,35 +365,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = named_bar_and(kBarState, kWG,
                            c < 1 || mbar_wait(bar + B_ODONE + 8 * (b ^ 1), ((c - 1) >> 1) & 1, wc));
         if (!ok) break;
-        if (ct < DK) {
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16)
-            st_bf16x8(sm + L::S_OFF + (b ^ 1) * (DK * 128) + sw128_off(ct, c16), sreg + 8 * c16);
-        }
+        if (ct < DK) put_state(b ^ 1);
         fence_proxy_async_smem();
         named_bar_sync(kBarState, kWG);
         if (ct == 0) mbar_arrive(bar + B_SREADY + 8 * (b ^ 1));
       }
-      // ---- O (c) / (Q' z + P 1) -> global (warps 0-1, TMEM lanes 0-63) ----
+      // ---- O (c) / (Q'z + P 1) -> global (warps 0-1, TMEM lanes 0-63) ----
       if (ct < 64) {
         ok_lo = named_bar_and(kBarLo, 64, mbar_wait(bar + B_ODONE + 8 * b, (c >> 1) & 1, wc));
         if (ok_lo) {
           tc_fence_after();
-          const float inv = 1.f / (dq[b * 64 + row] + rs[b * 64 + row]);
-          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c * kC + row) * Dv + j0;
+          const uint32_t o0 = tmem + lane_base + TM_O + kAugStride * b;
+          uint32_t ov[64], od[32];
+          tmem_ld32(o0, *reinterpret_cast<uint32_t(*)[32]>(ov));
+          tmem_ld32(o0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
+          tmem_ld32(o0 + 64, od);
+          tmem_wait_ld();
+          if (row < n) {
+            const float inv = 1.f / __uint_as_float(od[0]);
+            __nv_bfloat16* orow =
+                static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c * kC + row) * Dv + j0;
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t ov[32];
-            tmem_ld32(tmem + lane_base + TM_O + 64 * b + q * 32, ov);
-            tmem_wait_ld();
-            if (row < n) {
+            for (int cc = 0; cc < 8; ++cc) {
+              float x[8];
 #pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[cc * 8 + e]) * inv;
-                st_bf16x8(orow + q * 32 + cc * 8, x);
-              }
+              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[cc * 8 + e]) * inv;
+              st_bf16x8(orow + cc * 8, x);
             }
           }
           tc_fence_before();
@@ -422,11 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (p.S_out && ct < DK) {
-      float* dst = p.S_out + s_base + (size_t)ct * Dv + j0;
+    if (ct < DK) {
+      if (p.S_out) {
+        float* dst = p.S_out + s_base + (size_t)ct * Dv + j0;
 #pragma unroll
-      for (int j = 0; j < kDVS; j += 4)
-        *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
+        for (int j = 0; j < kDVS; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
+      }
+      if (p.z_out && blockIdx.y == 0) p.z_out[(size_t)bh * DK + ct] = zreg;
     }
   }
 
