@@ -25,9 +25,10 @@
 //              PU (c) has completed (QK^T (c+1) is committed after it).
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
 //              a three-stage ring (gated: two), L2 prefetch two chunks ahead
-//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead),
-//              then columns 32-63 of the U epilogue
-//   warps 4-5  P rows to bf16; gated: Q <- diag(gamma) Q in place
+//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead;
+//              gated: then Q <- diag(gamma) Q once QK^T has read it), then
+//              columns 32-63 of the U epilogue
+//   warps 4-5  P rows to bf16 (gated: with the decay Gamma)
 //   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
 //   warps 0-1  drain the output tile O = gamma QS + PU
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_PMMA2, 1);
     mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
-    mbar_init(bar + B_WREADY, GATED ? 2 : 1);  // W rows (+ gamma-scaled Q when gated)
+    mbar_init(bar + B_WREADY, 1);  // W rows (gated: and the gamma-scaled Q)
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -386,6 +387,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < 4; ++cc)
           st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
       }
+      if (GATED) {  // once QK^T (c) has read the plain Q: Q <- diag(gamma) Q in place
+        ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_PMMA1, c & 1, wc));
+        if (!ok) break;
+        const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
+        cvec[(c & 1) * 64 + row] = vs[64 + row];  // the chain's copy of g (the stage is released early)
+        const float gam = __expf(vs[64 + row]);
+#pragma unroll
+        for (int c16 = 0; c16 < DK / 8; ++c16) {
+          uint8_t* ptr = stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16 & 7);
+          uint4 u = *reinterpret_cast<uint4*>(ptr);
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
+            wv[e] = pack2_bf16(f.x * gam, f.y * gam);
+          }
+          *reinterpret_cast<uint4*>(ptr) = u;
+        }
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrepW, 64);
@@ -441,30 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_bf16x8(ptile + sw128_off(row, c16), x);
         }
       }
-      if (GATED) {
-        cvec[b * 64 + row] = vs[64 + row];
-        // Q <- diag(gamma) Q in place (the scores above used the plain Q)
-        const float gam = __expf(vs[64 + row]);
-#pragma unroll
-        for (int c16 = 0; c16 < DK / 8; ++c16) {
-          uint8_t* ptr = stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16 & 7);
-          uint4 u = *reinterpret_cast<uint4*>(ptr);
-          uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
-            wv[e] = pack2_bf16(f.x * gam, f.y * gam);
-          }
-          *reinterpret_cast<uint4*>(ptr) = u;
-        }
-      }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrepP, 64);
-      if (row == 0) {
-        mbar_arrive(bar + B_PREADY + 8 * b);
-        if (GATED) mbar_arrive(bar + B_WREADY);
-      }
+      if (row == 0) mbar_arrive(bar + B_PREADY + 8 * b);
     }
   } else {
     // --------------------------------------------------------------- chain --
