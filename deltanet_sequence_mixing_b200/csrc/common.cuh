@@ -77,14 +77,33 @@ __device__ __forceinline__ void record_timeout(const WaitCtl& w) {
   if (w.status) atomicOr(w.status, kStatusTimeoutBit);
 }
 
+// Longest time one suspended poll may keep the thread asleep (the hardware
+// wakes it as soon as the phase completes).
+constexpr uint32_t kSuspendHintNs = 200000u;
+
+// One poll that may suspend the thread until the phase completes or the hint
+// runs out, so a waiting warp leaves its scheduler's issue slots to the warps
+// that are working.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false if the
 // limit ran out (the timeout is recorded) or another thread already gave up.
+// kSuspend: poll with suspension (the default) or spin on plain polls.
+template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
+    if (kSuspend ? mbar_try_wait_suspend(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (kSuspend || (it & 15u) == 0) {
       if (*w.abort_flag) return false;
       if (global_ns() - t0 > w.limit_ns) {
         record_timeout(w);

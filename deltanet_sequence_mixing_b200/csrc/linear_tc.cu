@@ -77,9 +77,6 @@ constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_FMAP = 48, B_GDONE = 72, B_DSDONE
                    B_DSFREE = 120, B_SREADY = 136, B_ODONE = 152, B_OFREE = 168, B_FIN = 184,
                    B_TMEM = 192, B_ABORT = 196;
 
-// ELU(x) + 1: x + 1 for x > 0, and e^x (= (e^x - 1) + 1) otherwise.
-__device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
-
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -253,31 +250,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* stp = sm + (c % NST) * L::STAGE;
       ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
-      // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0), 4 pieces in flight ----
+      // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0) ----
+      // Four 16-byte pieces per thread per round, in stages (all loads, all
+      // exponentials, then the packs and stores) so the exponentials of 32
+      // elements are in flight together.
       constexpr int kPieces = L::KB * 2 * (int)(kTile / 16);  // 16-byte pieces of the K and Q tiles
-      static_assert(kPieces % (4 * kWG) == 0, "whole rounds of four pieces per thread");
-      for (int i0 = pt; i0 < kPieces; i0 += 4 * kWG) {
-        uint4 u[4];
-        uint8_t* ptr[4];
+      constexpr int kNpf = 4;
+      static_assert(kPieces % (kNpf * kWG) == 0, "whole rounds of pieces per thread");
+      for (int i0 = pt; i0 < kPieces; i0 += kNpf * kWG) {
+        uint4 u[kNpf];
+        uint8_t* ptr[kNpf];
+        bool live[kNpf];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kNpf; ++j) {
           const int i = i0 + j * kWG;
           const int t16 = i / (int)(kTile / 16), off = (i % (int)(kTile / 16)) * 16;
           ptr[j] = stp + (t16 >> 1) * L::KB_STRIDE + (t16 & 1) * kTile + off;
-          u[j] = (off >> 7) < n ? *reinterpret_cast<const uint4*>(ptr[j]) : make_uint4(0, 0, 0, 0);
+          live[j] = (off >> 7) < n;
+          u[j] = live[j] ? *reinterpret_cast<const uint4*>(ptr[j]) : make_uint4(0, 0, 0, 0);
+        }
+        float f[kNpf * 8], ex[kNpf * 8];
+#pragma unroll
+        for (int j = 0; j < kNpf; ++j) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u[j]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {  // bf16 pair -> two floats (low element first)
+            f[j * 8 + 2 * e] = __uint_as_float(w[e] << 16);
+            f[j * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int off = ((i0 + j * kWG) % (int)(kTile / 16)) * 16;
-          if ((off >> 7) < n) {
-            uint32_t* w = reinterpret_cast<uint32_t*>(&u[j]);
+        for (int k = 0; k < kNpf * 8; ++k) ex[k] = __expf(fminf(f[k], 0.f));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-              w[e] = pack2_bf16(elu1(f.x), elu1(f.y));
-            }
-          }
-          *reinterpret_cast<uint4*>(ptr[j]) = u[j];
+        for (int j = 0; j < kNpf; ++j) {
+          uint4 r;
+          uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)  // ELU(x) + 1 = max(x, 0) + e^min(x, 0)
+            w[e] = pack2_bf16(fmaxf(f[j * 8 + 2 * e], 0.f) + ex[j * 8 + 2 * e],
+                              fmaxf(f[j * 8 + 2 * e + 1], 0.f) + ex[j * 8 + 2 * e + 1]);
+          if (!live[j]) r = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(ptr[j]) = r;
         }
       }
       fence_proxy_async_smem();
