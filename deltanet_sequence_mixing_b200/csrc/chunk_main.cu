@@ -13,9 +13,10 @@
 //   O  = gamma Q S + P U        (accumulated onto the same TMEM tile)
 //   S <- gamma_last S + K^T (diag(Gamma_last,.) U)             (float32 registers)
 //
-// One CTA per (b, h, 64-column slice of Dv), 9 warps:
-//   warp 9     MMA issuer (one thread): every tcgen05.mma of the CTA, in a
-//              fixed order that keeps the state chain fed:
+// One CTA per (b, h, 64-column slice of Dv), 10 warps:
+//   warp 9     MMA issuer (warp-uniform, one elected lane issues): every
+//              tcgen05.mma of the CTA, in a fixed order that keeps the state
+//              chain fed:
 //                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
 //              (gated: QK^T (c+1) before K^T U (c), so that the gamma-scaled
 //              Q of chunk c+1 is ready as early as the new state).  W/Uh (c+1)
@@ -435,10 +436,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < nchunks && ok; ++c) {
       const int b = c & 1;
       uint8_t* stp = sm + (c % NST) * L::STAGE;
-      const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);  // gated only
-      ok = named_bar_and(kBarPrepP, 64,
-                         mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc) &&
-                             mbar_wait(bar + B_PMMA1, c & 1, wc));
+      float* vs = reinterpret_cast<float*>(stp + L::VEC_OFF);  // gated only: g at [64, 128)
+      ok = named_bar_and(kBarPrepP, 64, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
+      if (!ok) break;
+      // Gated: Gamma_rs = e^(g_r - g_s) (s <= r) as a_r b_s, a_r = e^(g_r - m),
+      // b_s = e^(m - g_s) with m the midpoint of the chunk's g range (g is
+      // non-increasing, rows past T flat).  Both factors stay within e^(+-80)
+      // while the range is at most 160; a wider range (gates near zero) takes
+      // one exponential per element.  b_s goes next to the g rows of the stage.
+      float gr = 0.f, ar = 1.f;
+      bool fact = true;
+      if (GATED) {
+        const float mid = 0.5f * (vs[64] + vs[127]);
+        fact = vs[64] - vs[127] <= 160.f;
+        gr = vs[64 + row];
+        ar = __expf(gr - mid);
+        vs[128 + row] = __expf(mid - gr);
+      }
+      ok = named_bar_and(kBarPrepP, 64, mbar_wait(bar + B_PMMA1, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
       {
@@ -446,19 +461,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
         tmem_wait_ld();
-        const float gr = GATED ? vs[64 + row] : 0.f;
         uint8_t* ptile = sm + L::P_OFF + (GATED ? b : 0) * kTile;
+        if (!GATED || fact) {
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          float x[8];
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int sc = c16 * 8 + e;
-            float val = __uint_as_float(g[sc]);
-            if (GATED) val *= __expf(gr - vs[64 + sc]);
-            x[e] = sc <= row ? val : 0.f;
+            for (int e = 0; e < 8; ++e) {
+              const int sc = c16 * 8 + e;
+              float val = __uint_as_float(g[sc]);
+              if (GATED) val *= ar * vs[128 + sc];
+              x[e] = sc <= row ? val : 0.f;
+            }
+            st_bf16x8(ptile + sw128_off(row, c16), x);
           }
-          st_bf16x8(ptile + sw128_off(row, c16), x);
+        } else {
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int sc = c16 * 8 + e;
+              const float val = __uint_as_float(g[sc]) * __expf(gr - vs[64 + sc]);
+              x[e] = sc <= row ? val : 0.f;
+            }
+            st_bf16x8(ptile + sw128_off(row, c16), x);
+          }
         }
       }
       fence_proxy_async_smem();

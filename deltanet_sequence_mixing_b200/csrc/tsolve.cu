@@ -13,8 +13,8 @@
 // of dependent steps, so it is latency-bound per chunk and the grid's
 // parallelism over chunks hides that latency.
 //   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
-//   2. G = K K^T with bf16 WMMA (float32 accumulate) straight into the A scratch,
-//      each warp masking and scaling its own tiles into A.
+//   2. G = K K^T by tcgen05 (bf16 operands from the swizzled K tile, float32
+//      accumulator in TMEM), read back row by row into A, masked and scaled.
 //   3. C/16 diagonal 16x16 inverses (one column per lane, right-looking
 //      substitution so only one multiply-add per step is on the dependency
 //      chain), then each warp finishes one 16-column block of T by block
@@ -50,8 +50,8 @@ struct TsolveSmem {
   static constexpr uint32_t kTBytes = C * TsolveShape<C>::kApad * 4;
   static constexpr uint32_t kRegion = ((kKBytes > kTBytes ? kKBytes : kTBytes) + 1023) / 1024 * 1024;
   static constexpr uint32_t AM_OFF = kRegion;
-  static constexpr uint32_t VEC_OFF = AM_OFF + kTBytes;  // beta, g, e^g (C each), 8 warp totals
-  static constexpr uint32_t BAR_OFF = (VEC_OFF + (3 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
+  static constexpr uint32_t VEC_OFF = AM_OFF + kTBytes;  // beta, g, e^g, e^(m-g) (C each), 8 warp totals
+  static constexpr uint32_t BAR_OFF = (VEC_OFF + (4 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
   static constexpr uint32_t BYTES = BAR_OFF + 32;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // 1024-byte alignment of the K tile
   static_assert(C == 128 || kRegion + 8192 <= BYTES, "M = 128 operand rows past the K tile stay inside");
@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
   float* vb = reinterpret_cast<float*>(sm + SL::VEC_OFF);
   float* vg = vb + kC;
   float* veg = vg + kC;
-  float* wsum = veg + kC;  // per-warp totals of the log-decay scan
+  float* vinv = veg + kC;  // e^(m - g), m the midpoint of the chunk's g range
+  float* wsum = vinv + kC;  // per-warp totals of the log-decay scan
   const uint32_t bar_full = sb + SL::BAR_OFF, bar_mma = sb + SL::BAR_OFF + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SL::BAR_OFF + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SL::BAR_OFF + 20);
@@ -163,6 +164,8 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
       g_out[((size_t)bh * nchunks + chunk) * kC + tid] = glog;
     }
     __syncthreads();
+    if (tid < kC) vinv[tid] = __expf(0.5f * (vg[0] + vg[kC - 1]) - vg[tid]);
+    __syncthreads();
   }
   //    A = strict_lower(diag(beta) G * Gamma): TMEM row r -> A row r (64 columns
   //    per thread).  Nothing reads A's upper part or T's strictly-upper tiles
@@ -174,24 +177,44 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
     const int r = tid & 127;  // = 32 (warp % 4) + lane: this warp's TMEM lanes
     const int col0 = (kC == 128) ? (tid >> 7) * 64 : 0;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const float br = vb[r], gr = GATED ? vg[r] : 0.f;
+    // Gated: Gamma_rc = e^(g_r - g_c) (c < r) as e^(g_r - m) e^(m - g_c), both
+    // factors within e^(+-80) while the chunk's g range is at most 160 (g is
+    // non-increasing); a wider range (gates near zero) takes one exponential
+    // per element.
+    const float gr = GATED ? vg[r] : 0.f;
+    const bool fact = !GATED || vg[0] - vg[kC - 1] <= 160.f;
+    const float br = GATED && fact ? vb[r] * __expf(gr - 0.5f * (vg[0] + vg[kC - 1])) : vb[r];
     float* arow = Am + r * kApad + col0;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       uint32_t gv[32];
       tmem_ld32(tmem + lane_base + col0 + q * 32, gv);
       tmem_wait_ld();
+      if (fact) {
 #pragma unroll
-      for (int e4 = 0; e4 < 32; e4 += 4) {
-        float a4[4];
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          float a4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = col0 + q * 32 + e4 + e;
-          float a = br * __uint_as_float(gv[e4 + e]);
-          if (GATED) a *= __expf(gr - vg[c]);
-          a4[e] = c < r ? a : 0.f;
+          for (int e = 0; e < 4; ++e) {
+            const int c = col0 + q * 32 + e4 + e;
+            float a = br * __uint_as_float(gv[e4 + e]);
+            if (GATED) a *= vinv[c];
+            a4[e] = c < r ? a : 0.f;
+          }
+          *reinterpret_cast<float4*>(arow + q * 32 + e4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         }
-        *reinterpret_cast<float4*>(arow + q * 32 + e4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+      } else {
+#pragma unroll
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          float a4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = col0 + q * 32 + e4 + e;
+            const float a = br * __uint_as_float(gv[e4 + e]) * __expf(gr - vg[c]);
+            a4[e] = c < r ? a : 0.f;
+          }
+          *reinterpret_cast<float4*>(arow + q * 32 + e4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        }
       }
     }
   }
