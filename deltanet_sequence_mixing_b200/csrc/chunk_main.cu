@@ -18,18 +18,16 @@
 //              tcgen05.mma of the CTA, in a fixed order that keeps the state
 //              chain fed:
 //                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
-//              (gated: QK^T (c+1) before K^T U (c), so that the gamma-scaled
-//              Q of chunk c+1 is ready as early as the new state).  W/Uh (c+1)
-//              runs while the U epilogue of chunk c drains (Uh is double-
-//              buffered in TMEM); PU (c) and QK^T (c+1) run during the state
-//              update.  Ungated, the single P tile is rewritten only after
-//              PU (c) has completed (QK^T (c+1) is committed after it).
+//              W/Uh (c+1) runs while the U epilogue of chunk c drains (Uh is
+//              double-buffered in TMEM); PU (c) and QK^T (c+1) run during the
+//              state update.  The single P tile is rewritten only after PU (c)
+//              has completed (QK^T (c+1) is committed after it).
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
 //              a three-stage ring (gated: two), L2 prefetch two chunks ahead
-//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead;
-//              gated: then Q <- diag(gamma) Q once QK^T has read it), then
-//              columns 32-63 of the U epilogue
-//   warps 4-5  P rows to bf16 (gated: with the decay Gamma)
+//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead),
+//              then columns 32-63 of the U epilogue
+//   warps 4-5  gated: diag(gamma) Q into its own tile as soon as the chunk
+//              lands; P rows to bf16 (gated: with the decay Gamma)
 //   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
 //   warps 0-1  drain the output tile O = gamma QS + PU
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
@@ -61,26 +59,28 @@ constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kB
 constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384, TM_UH1 = 448;
 
 // Shared memory.  A stage holds one chunk's TMA tiles [K | Q | W] per 64
-// columns of Dk, V, Tb (gated also Tbg and the beta / g rows); W is written
-// there by the W warps, right after Q, so that [Q; W] is one M = 128 operand.
+// columns of Dk (gated [K | Q | gamma Q | W]), V, Tb (gated also Tbg and the
+// g rows); W (and gamma Q) are written there by the W warps, so that [Q; W]
+// (gated [gamma Q; W]) is one M = 128 operand while QK^T reads the plain Q.
 // Ungated runs a three-stage ring (the chunk after next streams in while one
-// chunk is on the state chain and the next is being prepared) with a single
-// P tile; gated needs the Tbg tile, the decay-weighted U and the g rows, and
-// fits two stages and two P tiles.
+// chunk is on the state chain and the next is being prepared); gated needs
+// the gamma Q and Tbg tiles, the decay-weighted U and the g rows, and fits
+// two stages.
 template <int DK, bool GATED>
 struct MainLayout {
   static constexpr int KB = DK / 64;
   static constexpr int NST = GATED ? 2 : 3;           // ring stages
-  static constexpr int NP = GATED ? 2 : 1;            // P tiles
-  static constexpr uint32_t KB_STRIDE = 3 * kTile;    // [K | Q | W] per 64 columns of Dk
-  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
+  static constexpr uint32_t KB_STRIDE = (GATED ? 4 : 3) * kTile;  // [K | Q | (gamma Q) | W] per 64 columns of Dk
+  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile;
+  static constexpr uint32_t QS_OFF = GATED ? 2 * kTile : kTile;  // rows 0-63 of the [Q; W] S operand
+  static constexpr uint32_t W_OFF = QS_OFF + kTile;
   static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | (Tbg | beta, g)
   static constexpr uint32_t TB_OFF = V_OFF + kTile;
   static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
   static constexpr uint32_t VEC_OFF = TBG_OFF + kTile;
   static constexpr uint32_t STAGE = GATED ? VEC_OFF + 1024 : TBG_OFF;
-  static constexpr uint32_t P_OFF = NST * STAGE;      // P[NP] | U | (UT)
-  static constexpr uint32_t U_OFF = P_OFF + NP * kTile;
+  static constexpr uint32_t P_OFF = NST * STAGE;      // P | U | (UT)
+  static constexpr uint32_t U_OFF = P_OFF + kTile;
   static constexpr uint32_t UT_OFF = U_OFF + kTile;
   static constexpr uint32_t S_OFF = U_OFF + (GATED ? 2 : 1) * kTile;  // bf16 state, DK rows x 128 B
   static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // gated: chain copy of g per parity, [2][64]
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_PMMA2, 1);
     mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
-    mbar_init(bar + B_WREADY, 1);  // W rows (gated: and the gamma-scaled Q)
+    mbar_init(bar + B_WREADY, GATED ? 2 : 1);  // W rows (gated: and the gamma-scaled Q from the P warps)
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,7 +226,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           prefetch_l2_3d(&tmV, j0, cn, bh);
           prefetch_l2_3d(&tmTb, 0, cn, bh);
-          if (GATED) prefetch_l2_3d(&tmTbg, 0, cn, bh);
+          if (GATED) {
+            prefetch_l2_3d(&tmTbg, 0, cn, bh);
+            const float* gn = gw + ((size_t)bh * nchunks + c + 2) * kC;  // its g rows: two 128-byte lines
+            prefetch_l2(gn);
+            prefetch_l2(gn + 32);
+          }
         }
       }
       issued = c + 1;
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::QS_OFF + (ks & 3) * 32;
         mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
                           id, ks > 0);
       }
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
     auto issue_pu = [&](int c) {
-      const uint32_t pa = sb + L::P_OFF + (GATED ? (c & 1) : 0) * kTile;
+      const uint32_t pa = sb + L::P_OFF;
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
@@ -335,31 +340,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_wu(c + 1);
         mma_commit_elect(bar + B_PMMA2);
       }
-      if (GATED) {  // QK^T (c+1) once the scores of chunk c have left TMEM (P_READY)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
-        if (!ok) break;
-        if (nxt) {
-          tc_fence_after();
-          issue_qkt(c + 1);
-          mma_commit_elect(bar + B_PMMA1);
-        }
-      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar + B_UREADY, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
       issue_ds(c);
       mma_commit_elect(bar + B_CMMA4);
-      // K^T U (c) was the last reader of stage c: the P / Q / W epilogues of
-      // chunk c are done (W_READY, and gated P_READY, came before it)
-      mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
-      if (!GATED) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
-        if (!ok) break;
-        tc_fence_after();
-      }
+      // K^T U (c) is the last MMA that reads stage c.  Ungated the stage is
+      // free now (its W / Q epilogues came before W_READY); gated the P rows
+      // of chunk c still read its g rows, so it goes once they are done.
+      if (!GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      if (GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
       issue_pu(c);
       mma_commit_elect(bar + B_CMMA5 + 8 * b);
-      if (!GATED && nxt) {  // after PU (c): the single P tile is free once PMMA1 fires
+      if (nxt) {  // after PU (c): the single P tile is free once PMMA1 fires
         issue_qkt(c + 1);
         mma_commit_elect(bar + B_PMMA1);
       }
@@ -375,7 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
       uint8_t* stp = sm + (c % NST) * L::STAGE;
-      ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_PMMA2, c & 1, wc));
+      // (gated: the FULL wait orders the producer's g rows before the copy below)
+      ok = named_bar_and(kBarPrepW, 64,
+                         (!GATED || mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc)) &&
+                             mbar_wait(bar + B_PMMA2, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -388,24 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < 4; ++cc)
           st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
       }
-      if (GATED) {  // once QK^T (c) has read the plain Q: Q <- diag(gamma) Q in place
-        ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_PMMA1, c & 1, wc));
-        if (!ok) break;
+      if (GATED) {  // the chain's copy of g (the stage is released before the chain is done)
         const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
-        cvec[(c & 1) * 64 + row] = vs[64 + row];  // the chain's copy of g (the stage is released early)
-        const float gam = __expf(vs[64 + row]);
-#pragma unroll
-        for (int c16 = 0; c16 < DK / 8; ++c16) {
-          uint8_t* ptr = stp + (c16 >> 3) * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16 & 7);
-          uint4 u = *reinterpret_cast<uint4*>(ptr);
-          uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
-            wv[e] = pack2_bf16(f.x * gam, f.y * gam);
-          }
-          *reinterpret_cast<uint4*>(ptr) = u;
-        }
+        cvec[(c & 1) * 64 + row] = vs[64 + row];
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -430,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 192) mbar_arrive(bar + B_UREADY);
     }
   } else if (warp >= 4) {
-    // -------------------------------------------- P rows, gamma Q (4-5) --
+    // -------------------------------------------- gamma Q, P rows (4-5) --
     const int row = tid - 128;
     bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
@@ -439,6 +423,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* vs = reinterpret_cast<float*>(stp + L::VEC_OFF);  // gated only: g at [64, 128)
       ok = named_bar_and(kBarPrepP, 64, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
+      if (GATED) {  // diag(gamma) Q into its own tile (QK^T reads the plain Q), while the
+                    // chunk before is still on the chain
+        const float gam = __expf(vs[64 + row]);
+#pragma unroll
+        for (int kb = 0; kb < DK / 64; ++kb) {  // a 64-column block: all loads, then the stores
+          uint4 u[8];
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8)
+            u[c8] = *reinterpret_cast<const uint4*>(stp + kb * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c8));
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&u[c8]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
+              wv[e] = pack2_bf16(f.x * gam, f.y * gam);
+            }
+            *reinterpret_cast<uint4*>(stp + kb * L::KB_STRIDE + L::QS_OFF + sw128_off(row, c8)) = u[c8];
+          }
+        }
+        fence_proxy_async_smem();
+        // W_READY of the chunk before must have completed, so this arrival
+        // counts toward chunk c (the W warps arrive for c only after it).
+        ok = named_bar_and(kBarPrepP, 64, c < 1 || mbar_wait(bar + B_WREADY, (c - 1) & 1, wc));
+        if (!ok) break;
+        if (row == 0) mbar_arrive(bar + B_WREADY);
+      }
       // Gated: Gamma_rs = e^(g_r - g_s) (s <= r) as a_r b_s, a_r = e^(g_r - m),
       // b_s = e^(m - g_s) with m the midpoint of the chunk's g range (g is
       // non-increasing, rows past T flat).  Both factors stay within e^(+-80)
@@ -461,33 +472,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
         tmem_wait_ld();
-        uint8_t* ptile = sm + L::P_OFF + (GATED ? b : 0) * kTile;
+        uint8_t* ptile = sm + L::P_OFF;
+        // every value of the row in registers (the shared-memory reads of the
+        // decay factors all come before the first store of the P tile)
+        float* pv = reinterpret_cast<float*>(g);
         if (!GATED || fact) {
 #pragma unroll
           for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8];
+            float bc[8];
+            if (GATED) {
+              *reinterpret_cast<float4*>(bc) = *reinterpret_cast<const float4*>(vs + 128 + c16 * 8);
+              *reinterpret_cast<float4*>(bc + 4) = *reinterpret_cast<const float4*>(vs + 132 + c16 * 8);
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int sc = c16 * 8 + e;
-              float val = __uint_as_float(g[sc]);
-              if (GATED) val *= ar * vs[128 + sc];
-              x[e] = sc <= row ? val : 0.f;
+              float val = pv[sc];
+              if (GATED) val *= ar * bc[e];
+              pv[sc] = sc <= row ? val : 0.f;
             }
-            st_bf16x8(ptile + sw128_off(row, c16), x);
           }
         } else {
 #pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int sc = c16 * 8 + e;
-              const float val = __uint_as_float(g[sc]) * __expf(gr - vs[64 + sc]);
-              x[e] = sc <= row ? val : 0.f;
-            }
-            st_bf16x8(ptile + sw128_off(row, c16), x);
-          }
+          for (int sc = 0; sc < 64; ++sc) pv[sc] = sc <= row ? pv[sc] * __expf(gr - vs[64 + sc]) : 0.f;
         }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(ptile + sw128_off(row, c16), pv + c16 * 8);
       }
       fence_proxy_async_smem();
       tc_fence_before();

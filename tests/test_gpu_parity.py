@@ -111,6 +111,18 @@ def test_chunk_size_invariance_bf16(dn):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gated_strong_decay_both_sides_of_the_factor_range(dn, oracle_mod, dtype):
+    """Steep gates: per 64-token chunk the log-decay spans about 145 in head 0
+    (the decay factors split about the chunk's midpoint) and about 170 in
+    head 1 (one exponential per element); head 2 mixes steep and mild gates."""
+    x = gen.make_inputs(1, 3, 300, 128, 128, dtype, gated=True, seed=13)
+    x["alpha"][:, 0] = float(np.exp(-2.3))
+    x["alpha"][:, 1] = float(np.exp(-2.7))
+    x["alpha"][:, 2, ::3] = float(np.exp(-6.0))
+    _check_delta(dn, oracle_mod, x)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_gate_zero_and_one(dn, oracle_mod, dtype):
     x = gen.make_inputs(1, 2, 190, 128, 128, dtype, gated=True, seed=8)
     x["alpha"][:, :, 70] = 0.0
