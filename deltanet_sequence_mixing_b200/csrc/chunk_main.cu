@@ -8,9 +8,10 @@
 // rule)"; gate from the Gated DeltaNet paragraph of "How a Baseten Engineer
 // Traced 7 Years of Attention Mechanism Evolution"):
 //   P  = tril(Q K^T) * Gamma,  W = Tbg K,  Uh = Tb V          (state-independent)
-//   [gamma Q S ; W S] = [diag(gamma) Q ; W] S                  (one M = 128 MMA)
+//   [Q S ; W S] = [Q ; W] S                                    (one M = 128 MMA)
 //   U  = Uh - W S                                              (the chunk's deltas)
-//   O  = gamma Q S + P U        (accumulated onto the same TMEM tile)
+//   O  = diag(gamma) Q S + P U  (Q S rows scaled in TMEM, then P U
+//                                accumulated onto the same tile)
 //   S <- gamma_last S + K^T (diag(Gamma_last,.) U)             (float32 registers)
 //
 // One CTA per (b, h, 64-column slice of Dv), 10 warps:
@@ -26,10 +27,10 @@
 //              a three-stage ring (gated: two), L2 prefetch two chunks ahead
 //   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead),
 //              then columns 32-63 of the U epilogue
-//   warps 4-5  gated: diag(gamma) Q into its own tile as soon as the chunk
-//              lands; P rows to bf16 (gated: with the decay Gamma)
+//   warps 4-5  P rows to bf16 (gated: with the decay Gamma)
 //   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
-//   warps 0-1  drain the output tile O = gamma QS + PU
+//   warps 0-1  gated: QS rows times gamma in TMEM while the U epilogue runs;
+//              drain the output tile O = diag(gamma) QS + PU
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
 // signal back; the issuer waits on their signals.  Every mbarrier completes
 // once per chunk (or per use of a parity), so parity waits are unambiguous.
@@ -59,21 +60,17 @@ constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kB
 constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384, TM_UH1 = 448;
 
 // Shared memory.  A stage holds one chunk's TMA tiles [K | Q | W] per 64
-// columns of Dk (gated [K | Q | gamma Q | W]), V, Tb (gated also Tbg and the
-// g rows); W (and gamma Q) are written there by the W warps, so that [Q; W]
-// (gated [gamma Q; W]) is one M = 128 operand while QK^T reads the plain Q.
+// columns of Dk, V, Tb (gated also Tbg and the g rows); W is written there
+// by the W warps, right after Q, so that [Q; W] is one M = 128 operand.
 // Ungated runs a three-stage ring (the chunk after next streams in while one
 // chunk is on the state chain and the next is being prepared); gated needs
-// the gamma Q and Tbg tiles, the decay-weighted U and the g rows, and fits
-// two stages.
+// the Tbg tile, the decay-weighted U and the g rows, and fits two stages.
 template <int DK, bool GATED>
 struct MainLayout {
   static constexpr int KB = DK / 64;
   static constexpr int NST = GATED ? 2 : 3;           // ring stages
-  static constexpr uint32_t KB_STRIDE = (GATED ? 4 : 3) * kTile;  // [K | Q | (gamma Q) | W] per 64 columns of Dk
-  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile;
-  static constexpr uint32_t QS_OFF = GATED ? 2 * kTile : kTile;  // rows 0-63 of the [Q; W] S operand
-  static constexpr uint32_t W_OFF = QS_OFF + kTile;
+  static constexpr uint32_t KB_STRIDE = 3 * kTile;    // [K | Q | W] per 64 columns of Dk
+  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
   static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | (Tbg | beta, g)
   static constexpr uint32_t TB_OFF = V_OFF + kTile;
   static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
@@ -95,7 +92,7 @@ struct MainLayout {
 // OFREE, CMMA5 and PREADY: one per chunk parity.
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
-                   B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164;
+                   B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168;
 
 // One half (32 columns, [col0, col0 + 32)) of the U epilogue for the row on
 // this thread's TMEM lane: U = Uh - WS to bf16 (gated also U~ = U e^(g_last - g_row)).
@@ -160,7 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_PMMA2, 1);
     mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
-    mbar_init(bar + B_WREADY, GATED ? 2 : 1);  // W rows (gated: and the gamma-scaled Q from the P warps)
+    mbar_init(bar + B_WREADY, 1);
+    mbar_init(bar + B_QSCALED, 1);  // gated: the QS rows of TM_QW scaled by gamma
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -285,13 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    // [gamma Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
+    // [Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
     auto issue_qw = [&](int c) {
       const uint32_t st = stage(c);
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::QS_OFF + (ks & 3) * 32;
+        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
         mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
                           id, ks > 0);
       }
@@ -306,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_bf16_ss_elect(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
                           desc_mn(ut + ks * 2048, kTile), id, ks > 0);
     };
-    // O = gamma QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
+    // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
     auto issue_pu = [&](int c) {
       const uint32_t pa = sb + L::P_OFF;
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
@@ -349,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // free now (its W / Q epilogues came before W_READY); gated the P rows
       // of chunk c still read its g rows, so it goes once they are done.
       if (!GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
-      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc) &&
+                                       (!GATED || mbar_wait(bar + B_QSCALED, c & 1, wc)));
       if (!ok) break;
       tc_fence_after();
       if (GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
@@ -414,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 192) mbar_arrive(bar + B_UREADY);
     }
   } else if (warp >= 4) {
-    // -------------------------------------------- gamma Q, P rows (4-5) --
+    // ---------------------------------------------------- P rows (4-5) --
     const int row = tid - 128;
     bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
@@ -423,33 +422,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* vs = reinterpret_cast<float*>(stp + L::VEC_OFF);  // gated only: g at [64, 128)
       ok = named_bar_and(kBarPrepP, 64, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
-      if (GATED) {  // diag(gamma) Q into its own tile (QK^T reads the plain Q), while the
-                    // chunk before is still on the chain
-        const float gam = __expf(vs[64 + row]);
-#pragma unroll
-        for (int kb = 0; kb < DK / 64; ++kb) {  // a 64-column block: all loads, then the stores
-          uint4 u[8];
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8)
-            u[c8] = *reinterpret_cast<const uint4*>(stp + kb * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c8));
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&u[c8]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
-              wv[e] = pack2_bf16(f.x * gam, f.y * gam);
-            }
-            *reinterpret_cast<uint4*>(stp + kb * L::KB_STRIDE + L::QS_OFF + sw128_off(row, c8)) = u[c8];
-          }
-        }
-        fence_proxy_async_smem();
-        // W_READY of the chunk before must have completed, so this arrival
-        // counts toward chunk c (the W warps arrive for c only after it).
-        ok = named_bar_and(kBarPrepP, 64, c < 1 || mbar_wait(bar + B_WREADY, (c - 1) & 1, wc));
-        if (!ok) break;
-        if (row == 0) mbar_arrive(bar + B_WREADY);
-      }
       // Gated: Gamma_rs = e^(g_r - g_s) (s <= r) as a_r b_s, a_r = e^(g_r - m),
       // b_s = e^(m - g_s) with m the midpoint of the chunk's g range (g is
       // non-increasing, rows past T flat).  Both factors stay within e^(+-80)
@@ -543,6 +515,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           named_bar_sync(kBarChainHi, 64);
           if (ct == 64) mbar_arrive(bar + B_UREADY);
+        }
+      }
+      if (GATED && ct < 64) {
+        // ---- QS rows (lanes 0-63) times gamma, in TMEM, before P U lands on them ----
+        ok_lo = named_bar_and(kBarChainLo, 64, ok_lo && mbar_wait(bar + B_CMMA3, c & 1, wc));
+        if (ok_lo) {
+          tc_fence_after();
+          const float gam = __expf(vb[row]);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t v[32];
+            tmem_ld32(qw + lane_base + q * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * gam);
+            tmem_st32(qw + lane_base + q * 32, v);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          named_bar_sync(kBarChainLo, 64);
+          if (ct == 0) mbar_arrive(bar + B_QSCALED);
         }
       }
       ok = named_bar_and(kBarChain, kWG, ok_hi && ok_lo && mbar_wait(bar + B_CMMA4, c & 1, wc));
