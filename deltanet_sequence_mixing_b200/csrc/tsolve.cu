@@ -242,40 +242,92 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
     for (int i = 0; i < 16; ++i) Tm[(o + i) * kApad + o + j] = col[i];
   }
   __syncthreads();
-  //    Column block w (warp w) by block forward substitution:
-  //    T_iw = -D_i sum_{m=w}^{i-1} A_im T_mw  for i > w   (tf32 products)
+  //    The blocks below the diagonal (tf32 tensor-core products of 16 x 16
+  //    tiles).  C = 64, by halves, four dependent levels: with L = I + A split
+  //    into 32 x 32 blocks, T = [[T1, 0], [-T2 L21 T1, T2]], where T1, T2 are
+  //    the inverses of the diagonal halves, each [[D_a, 0], [-D_b A_ba D_a, D_b]]:
+  //      1. A10 D0, A32 D2            2. T10 = -D1 (A10 D0), T32 = -D3 (A32 D2)
+  //      3. X = L21 T1 (four tiles)   4. T21 = -T2 X (four tiles)
+  //    Scratch tiles sit in A's unused upper blocks.  C = 128, column block
+  //    w (warp w) by block forward substitution, T_iw = -D_i sum_m A_im T_mw.
   {
-    wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fa;
-    wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major> fb;
-    wmma::fragment<wmma::accumulator, 16, 16, 8, float> acc;
-    float* xs = Am + (16 * warp) * kApad + (kC - 16);  // 16x16 scratch in A's unused upper part
-    for (int i = warp + 1; i < Sh::kWarps; ++i) {
-      wmma::fill_fragment(acc, 0.f);
-      for (int m = warp; m < i; ++m) {
-#pragma unroll
-        for (int kk = 0; kk < 16; kk += 8) {
-          wmma::load_matrix_sync(fa, Am + (16 * i) * kApad + 16 * m + kk, kApad);
-          wmma::load_matrix_sync(fb, Tm + (16 * m + kk) * kApad + 16 * warp, kApad);
-          to_tf32(fa);
-          to_tf32(fb);
-          wmma::mma_sync(acc, fa, fb, acc);
-        }
-      }
-      wmma::store_matrix_sync(xs, acc, kApad, wmma::mem_row_major);
-      __syncwarp();
-      wmma::fill_fragment(acc, 0.f);
+    using FragA = wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major>;
+    using FragB = wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major>;
+    using FragC = wmma::fragment<wmma::accumulator, 16, 16, 8, float>;
+    // acc += X Y for 16 x 16 tiles X, Y (row-major, row stride kApad)
+    auto mac = [&](FragC& acc, const float* x, const float* y) {
+      FragA fa;
+      FragB fb;
 #pragma unroll
       for (int kk = 0; kk < 16; kk += 8) {
-        wmma::load_matrix_sync(fa, Tm + (16 * i) * kApad + 16 * i + kk, kApad);
-        wmma::load_matrix_sync(fb, xs + kk * kApad, kApad);
+        wmma::load_matrix_sync(fa, x + kk, kApad);
+        wmma::load_matrix_sync(fb, y + kk * kApad, kApad);
         to_tf32(fa);
         to_tf32(fb);
         wmma::mma_sync(acc, fa, fb, acc);
       }
+    };
+    auto put = [&](float* dst, FragC& acc, bool negate) {
+      if (negate) {
 #pragma unroll
-      for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
-      wmma::store_matrix_sync(Tm + (16 * i) * kApad + 16 * warp, acc, kApad, wmma::mem_row_major);
-      __syncwarp();
+        for (int t = 0; t < acc.num_elements; ++t) acc.x[t] = -acc.x[t];
+      }
+      wmma::store_matrix_sync(dst, acc, kApad, wmma::mem_row_major);
+    };
+    auto At = [&](int i, int j) { return Am + (16 * i) * kApad + 16 * j; };  // also the scratch tiles (j > i)
+    auto Tt = [&](int i, int j) { return Tm + (16 * i) * kApad + 16 * j; };
+    if constexpr (kC == 64) {
+      FragC acc;
+      if (warp < 2) {  // level 1: A10 D0 -> S01, A32 D2 -> S23
+        const int a = 2 * warp;
+        wmma::fill_fragment(acc, 0.f);
+        mac(acc, At(a + 1, a), Tt(a, a));
+        put(At(a, a + 1), acc, false);
+      }
+      __syncthreads();
+      if (warp < 2) {  // level 2: T10 = -D1 S01, T32 = -D3 S23
+        const int a = 2 * warp;
+        wmma::fill_fragment(acc, 0.f);
+        mac(acc, Tt(a + 1, a + 1), At(a, a + 1));
+        put(Tt(a + 1, a), acc, true);
+      }
+      __syncthreads();
+      {  // level 3: X_rc = sum_m A_rm T1_mc for r in {2, 3}, c in {0, 1} -> S_c(r)
+        const int r = 2 + (warp >> 1), cc = warp & 1;
+        wmma::fill_fragment(acc, 0.f);
+        if (cc == 0) {
+          mac(acc, At(r, 0), Tt(0, 0));
+          mac(acc, At(r, 1), Tt(1, 0));
+        } else {
+          mac(acc, At(r, 1), Tt(1, 1));
+        }
+        put(At(cc, r), acc, false);
+      }
+      __syncthreads();
+      {  // level 4: T_rc = -sum_m T2_rm X_mc
+        const int r = 2 + (warp >> 1), cc = warp & 1;
+        wmma::fill_fragment(acc, 0.f);
+        if (r == 2) {
+          mac(acc, Tt(2, 2), At(cc, 2));
+        } else {
+          mac(acc, Tt(3, 2), At(cc, 2));
+          mac(acc, Tt(3, 3), At(cc, 3));
+        }
+        put(Tt(r, cc), acc, true);
+      }
+    } else {
+      FragC acc;
+      float* xs = At(warp, Sh::kWarps - 1);  // 16 x 16 scratch in A's unused upper part
+      for (int i = warp + 1; i < Sh::kWarps; ++i) {
+        wmma::fill_fragment(acc, 0.f);
+        for (int m = warp; m < i; ++m) mac(acc, At(i, m), Tt(m, warp));
+        put(xs, acc, false);
+        __syncwarp();
+        wmma::fill_fragment(acc, 0.f);
+        mac(acc, Tt(i, i), xs);
+        put(Tt(i, warp), acc, true);
+        __syncwarp();
+      }
     }
   }
   __syncthreads();
