@@ -19,7 +19,8 @@ from . import _lib
 from ._lib import DeltaNetError, check, lib, status_string  # noqa: F401
 
 __all__ = [
-    "deltanet_chunk_fwd", "deltanet_decode_step", "linear_attn_fwd", "workspace_for",
+    "deltanet_chunk_fwd", "deltanet_chunk_fwd_host", "deltanet_decode_step", "linear_attn_fwd",
+    "workspace_for", "host_workspace_for",
     "deltanet_get_device_status", "deltanet_selftest_wait_timeout", "DeltaNetError",
 ]
 
@@ -97,6 +98,64 @@ def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, 
     check("deltanet_chunk_fwd", lib().deltanet_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
         B, H, T, Dk, Dv, C, dt, _ptr(ws), ws.numel(), _stream(dev)))
+    return o, S_out
+
+
+def _need_host(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor for the host-buffer call")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def host_workspace_for(device, B, H, T, Dk, Dv, C, dtype) -> torch.Tensor:
+    """A device workspace for deltanet_chunk_fwd_host (cleared, not cached)."""
+    device = torch.device(device)
+    nb = lib().deltanet_host_workspace_bytes(B, H, T, Dk, Dv, C, _DT[dtype])
+    if nb == 0:
+        raise DeltaNetError("deltanet_host_workspace_bytes", _lib.DN_ERR_UNSUPPORTED)
+    ws = torch.empty(nb, dtype=torch.uint8, device=device)
+    check("deltanet_workspace_init", lib().deltanet_workspace_init(_ptr(ws), ws.numel(), _stream(device)))
+    return ws
+
+
+def deltanet_chunk_fwd_host(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, S_out=None,
+                            workspace=None, device=None):
+    """deltanet_chunk_fwd on host tensors (page-locked for overlapped copies):
+    the heads stream through the device in groups, copies overlapping the
+    compute.  Asynchronous on the device's current stream: synchronize it
+    before reading (o, S_out)."""
+    _need_host(q, "q")
+    dtype = q.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for t, n in ((k, "k"), (v, "v")):
+        _need_host(t, n, dtype)
+    _need_host(beta, "beta", torch.float32)
+    for t, n in ((alpha, "alpha"), (S0, "S0")):
+        if t is not None:
+            _need_host(t, n, torch.float32)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, T, Dv, dtype=dtype).pin_memory()
+    if S_out is None:
+        S_out = torch.empty(B, H, Dk, Dv, dtype=torch.float32).pin_memory()
+    _need_host(o, "o", dtype)
+    _need_host(S_out, "S_out", torch.float32)
+    device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if workspace is None:
+        workspace = host_workspace_for(device, B, H, T, Dk, Dv, C, dtype)
+    _need(workspace, "workspace", torch.uint8, device)
+    with torch.cuda.device(device):
+        check("deltanet_chunk_fwd_host", lib().deltanet_chunk_fwd_host(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
+            B, H, T, Dk, Dv, C, _DT[dtype], _ptr(workspace), workspace.numel(), _stream(device)))
     return o, S_out
 
 

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <climits>
+#include <mutex>
 
 #include "deltanet.h"
 #include "kernels.h"
@@ -35,8 +36,8 @@ int map_cuda(cudaError_t e) {
   return DN_ERR_CUDA;
 }
 
-// Shared validation of the chunked calls.  Returns DN_OK or an error.
-int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws) {
+// Shape and presence checks shared by the chunked calls.
+int validate_problem(const dn::ChunkProblem& p) {
   if (p.B < 0 || p.H < 0 || p.T < 0) return DN_ERR_INVALID_ARG;
   if (p.bf16 != 0 && p.bf16 != 1) return DN_ERR_INVALID_ARG;
   if (!valid_dim(p.Dk) || !valid_dim(p.Dv)) return DN_ERR_UNSUPPORTED;
@@ -48,16 +49,12 @@ int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws)
     if (!p.q || !p.k || !p.v || !p.o) return DN_ERR_INVALID_ARG;
     if (p.mode == dn::Mode::Delta && !p.beta) return DN_ERR_INVALID_ARG;
   }
-  if (!ws) return DN_ERR_WORKSPACE;
-  if (ws_bytes < deltanet_workspace_bytes(p.B, p.H, p.T, p.Dk, p.Dv, p.C,
-                                          p.bf16 ? DN_BF16 : DN_F32))
-    return DN_ERR_WORKSPACE;
-  if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.o))
-    return DN_ERR_ALIGNMENT;
-  if ((p.S0 && !aligned16(p.S0)) || (p.S_out && !aligned16(p.S_out)) ||
-      (p.z0 && !aligned16(p.z0)) || (p.z_out && !aligned16(p.z_out)) || !aligned16(ws))
-    return DN_ERR_ALIGNMENT;
+  return DN_OK;
+}
 
+// Overlap rules of the chunked calls: o overlaps nothing, S_out / z_out only
+// exactly S0 / z0, and the workspace none of the caller's buffers.
+int validate_overlaps(const dn::ChunkProblem& p, const void* ws, size_t ws_bytes) {
   const size_t es = p.bf16 ? 2 : 4;
   const size_t BH = (size_t)p.B * p.H, T = (size_t)p.T;
   const Range q = range_of(p.q, BH * T * p.Dk * es), k = range_of(p.k, BH * T * p.Dk * es);
@@ -85,18 +82,102 @@ int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws)
   return DN_OK;
 }
 
-int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
+// Full validation of a chunked call on device buffers.  Returns DN_OK or an error.
+int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws) {
+  int rc = validate_problem(p);
+  if (rc != DN_OK) return rc;
+  if (!ws) return DN_ERR_WORKSPACE;
+  if (ws_bytes < deltanet_workspace_bytes(p.B, p.H, p.T, p.Dk, p.Dv, p.C,
+                                          p.bf16 ? DN_BF16 : DN_F32))
+    return DN_ERR_WORKSPACE;
+  if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.o))
+    return DN_ERR_ALIGNMENT;
+  if ((p.S0 && !aligned16(p.S0)) || (p.S_out && !aligned16(p.S_out)) ||
+      (p.z0 && !aligned16(p.z0)) || (p.z_out && !aligned16(p.z_out)) || !aligned16(ws))
+    return DN_ERR_ALIGNMENT;
+  return validate_overlaps(p, ws, ws_bytes);
+}
+
+// Launch the kernels of a validated chunked problem; `status` is the device
+// status word, `wy` the start of the pre-pass factor region.
+int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStream_t st) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
-  p.status = static_cast<unsigned int*>(ws);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  p.status = status;
   if (dn::chunk_main_supported(p) || dn::chunk128_supported(p)) {
-    const dn::WyWorkspace w =
-        dn::wy_carve(static_cast<uint8_t*>(ws) + kStatusBytes, p.B, p.H, p.T, p.C);
+    const dn::WyWorkspace w = dn::wy_carve(wy, p.B, p.H, p.T, p.C);
     return map_cuda(p.C == 64 ? dn::launch_chunk_main(p, w, st) : dn::launch_chunk128(p, w, st));
   }
   if (dn::linear_tc_supported(p)) return map_cuda(dn::launch_linear_tc(p, st));
   if (dn::chunk_simt_supported(p.Dk, p.Dv, p.C)) return map_cuda(dn::launch_chunk_simt(p, st));
   return DN_ERR_UNSUPPORTED;
+}
+
+int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
+  return run_chunked_at(p, static_cast<unsigned int*>(ws), static_cast<uint8_t*>(ws) + kStatusBytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ host buffers --
+// The host-buffer call streams the heads through the device in kHostGroups
+// groups, two staging slots in the workspace, on three library streams.
+constexpr int kHostGroups = 8;
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int host_group_heads(long long BH) { return (int)((BH + kHostGroups - 1) / kHostGroups); }
+
+struct HostSlot {  // byte offsets inside one staging slot
+  size_t q, k, v, o, beta, alpha, S0, S_out, wy, bytes;
+};
+
+HostSlot host_slot(int Hg, int T, int Dk, int Dv, int C, bool bf16) {
+  const size_t es = bf16 ? 2 : 4, tok = (size_t)Hg * T, st = (size_t)Hg * Dk * Dv * 4;
+  HostSlot L{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t at = off;
+    off += round256(n);
+    return at;
+  };
+  L.q = take(tok * Dk * es);
+  L.k = take(tok * Dk * es);
+  L.v = take(tok * Dv * es);
+  L.o = take(tok * Dv * es);
+  L.beta = take(tok * 4);
+  L.alpha = take(tok * 4);
+  L.S0 = take(st);
+  L.S_out = take(st);
+  L.wy = take(bf16 && T > 0 ? dn::wy_workspace_bytes(1, Hg, T, C) : 0);
+  L.bytes = off;
+  return L;
+}
+
+// Streams and events of the host-buffer call, created once per device.
+struct HostQueues {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t loaded[2] = {}, computed[2] = {}, drained[2] = {};
+};
+constexpr int kMaxDevices = 64;
+HostQueues g_host_queues[kMaxDevices];
+std::mutex g_host_mutex;  // held while a call creates or enqueues on them
+
+cudaError_t host_queues(int dev, HostQueues** out) {
+  HostQueues& h = g_host_queues[dev];
+  if (!h.ready) {
+    cudaError_t e = cudaSuccess;
+    for (cudaStream_t* s : {&h.h2d, &h.comp, &h.d2h})
+      if (e == cudaSuccess) e = cudaStreamCreateWithFlags(s, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&h.start, &h.end, &h.loaded[0], &h.loaded[1], &h.computed[0],
+                          &h.computed[1], &h.drained[0], &h.drained[1]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    h.ready = true;
+  }
+  *out = &h;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -131,6 +212,102 @@ int deltanet_chunk_fwd(const void* q, const void* k, const void* v, const float*
   const int rc = validate_chunked(p, ws_bytes, workspace);
   if (rc != DN_OK) return rc;
   return run_chunked(p, workspace, cuda_stream);
+}
+
+size_t deltanet_host_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
+  if (deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt) == 0) return 0;
+  const long long BH = (long long)B * H;
+  if (BH > INT_MAX) return 0;
+  return kStatusBytes + 2 * host_slot(host_group_heads(BH), T, Dk, Dv, C, dt == DN_BF16).bytes;
+}
+
+int deltanet_chunk_fwd_host(const void* q, const void* k, const void* v, const float* beta,
+                            const float* alpha, const float* S0, void* o, float* S_out, int B,
+                            int H, int T, int Dk, int Dv, int C, dn_dtype dt, void* workspace,
+                            size_t ws_bytes, void* cuda_stream) {
+  if (dt != DN_F32 && dt != DN_BF16) return DN_ERR_UNSUPPORTED;
+  dn::ChunkProblem p{};
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.alpha = alpha; p.S0 = S0;
+  p.o = o; p.S_out = S_out;
+  p.B = B; p.H = H; p.T = T; p.Dk = Dk; p.Dv = Dv; p.C = C;
+  p.bf16 = dt == DN_BF16;
+  p.mode = dn::Mode::Delta;
+  int rc = validate_problem(p);
+  if (rc != DN_OK) return rc;
+  if (!workspace) return DN_ERR_WORKSPACE;
+  if (ws_bytes < deltanet_host_workspace_bytes(B, H, T, Dk, Dv, C, dt)) return DN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DN_ERR_ALIGNMENT;
+  rc = validate_overlaps(p, workspace, ws_bytes);
+  if (rc != DN_OK) return rc;
+  const long long BH = (long long)B * H;
+  if (BH == 0) return DN_OK;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return DN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_host_mutex);
+  HostQueues* hq = nullptr;
+  if (host_queues(dev, &hq) != cudaSuccess) return DN_ERR_CUDA;
+
+  const int Hg = host_group_heads(BH);
+  const HostSlot L = host_slot(Hg, T, Dk, Dv, C, p.bf16 != 0);
+  const size_t es = p.bf16 ? 2 : 4;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* status = reinterpret_cast<unsigned int*>(ws);
+  cudaStream_t cs = static_cast<cudaStream_t>(cuda_stream);
+  auto ok = [&](cudaError_t r) { return (e = (e == cudaSuccess ? r : e)) == cudaSuccess; };
+  auto h2d = [&](void* dst, const void* src, size_t n) {
+    return n == 0 || ok(cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, hq->h2d));
+  };
+  auto d2h = [&](void* dst, const void* src, size_t n) {
+    return n == 0 || ok(cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, hq->d2h));
+  };
+  // everything already queued on the caller's stream comes first
+  ok(cudaEventRecord(hq->start, cs));
+  for (cudaStream_t s : {hq->h2d, hq->comp, hq->d2h}) ok(cudaStreamWaitEvent(s, hq->start, 0));
+  int launch_rc = DN_OK;
+  for (long long h0 = 0, g = 0; h0 < BH && e == cudaSuccess && launch_rc == DN_OK; h0 += Hg, ++g) {
+    const int hn = (int)(BH - h0 < Hg ? BH - h0 : Hg), sl = (int)(g & 1);
+    uint8_t* slot = ws + kStatusBytes + sl * L.bytes;
+    const size_t tok = (size_t)hn * T, t0 = (size_t)h0 * T;
+    const size_t st = (size_t)hn * Dk * Dv * 4, s0 = (size_t)h0 * Dk * Dv * 4;
+    // 1. inputs of group g into slot g % 2, once group g - 2 has left it
+    ok(cudaStreamWaitEvent(hq->h2d, hq->drained[sl], 0));
+    if (T > 0) {  // with T == 0 the token buffers may be null
+      h2d(slot + L.q, static_cast<const uint8_t*>(q) + t0 * Dk * es, tok * Dk * es);
+      h2d(slot + L.k, static_cast<const uint8_t*>(k) + t0 * Dk * es, tok * Dk * es);
+      h2d(slot + L.v, static_cast<const uint8_t*>(v) + t0 * Dv * es, tok * Dv * es);
+      if (beta) h2d(slot + L.beta, beta + t0, tok * 4);
+      if (alpha) h2d(slot + L.alpha, alpha + t0, tok * 4);
+    }
+    if (S0) h2d(slot + L.S0, reinterpret_cast<const uint8_t*>(S0) + s0, st);
+    ok(cudaEventRecord(hq->loaded[sl], hq->h2d));
+    // 2. the group's chunked forward on the compute stream
+    ok(cudaStreamWaitEvent(hq->comp, hq->loaded[sl], 0));
+    if (e != cudaSuccess) break;
+    dn::ChunkProblem pg = p;
+    pg.q = slot + L.q; pg.k = slot + L.k; pg.v = slot + L.v; pg.o = slot + L.o;
+    pg.beta = beta ? reinterpret_cast<const float*>(slot + L.beta) : nullptr;
+    pg.alpha = alpha ? reinterpret_cast<const float*>(slot + L.alpha) : nullptr;
+    pg.S0 = S0 ? reinterpret_cast<const float*>(slot + L.S0) : nullptr;
+    pg.S_out = S_out ? reinterpret_cast<float*>(slot + L.S_out) : nullptr;
+    pg.B = 1;
+    pg.H = hn;
+    launch_rc = run_chunked_at(pg, status, slot + L.wy, hq->comp);
+    ok(cudaEventRecord(hq->computed[sl], hq->comp));
+    // 3. outputs of group g back to the host
+    ok(cudaStreamWaitEvent(hq->d2h, hq->computed[sl], 0));
+    if (T > 0) d2h(static_cast<uint8_t*>(o) + t0 * Dv * es, slot + L.o, tok * Dv * es);
+    if (S_out) d2h(reinterpret_cast<uint8_t*>(S_out) + s0, slot + L.S_out, st);
+    ok(cudaEventRecord(hq->drained[sl], hq->d2h));
+  }
+  // the caller's stream continues once the last group is back on the host
+  // (also after a failed launch, so that nothing queued here outlives the call
+  // on the caller's stream)
+  ok(cudaEventRecord(hq->end, hq->d2h));
+  ok(cudaStreamWaitEvent(cs, hq->end, 0));
+  return launch_rc != DN_OK ? launch_rc : map_cuda(e);
 }
 
 int linear_attn_fwd(const void* q, const void* k, const void* v, const float* S0,

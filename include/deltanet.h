@@ -206,6 +206,43 @@ int deltanet_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
                                void *cuda_stream);
 
+/*
+ * Bytes of DEVICE workspace deltanet_chunk_fwd_host needs: the 256-byte status
+ * word, then two staging slots, each holding one group of heads' q, k, v, o,
+ * beta, alpha, S0 and S_out plus that group's pre-pass factors (the per-chunk
+ * factors of deltanet_workspace_bytes for the group's heads).  The heads are
+ * taken in groups of ceil(B*H / 8).  Each region starts on a 256-byte boundary.
+ * Returns 0 for sizes the library rejects.
+ */
+size_t deltanet_host_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt);
+
+/*
+ * deltanet_chunk_fwd on HOST buffers: q, k, v, beta, alpha, S0, o and S_out
+ * have the shapes, types and meaning of deltanet_chunk_fwd's arguments but
+ * live in host memory (no alignment needed).  The heads pass through the
+ * device in groups of ceil(B*H / 8): the host-to-device copy of one group,
+ * the computation of the group before it and the device-to-host copy of the
+ * group before that run at the same time, on three streams the library
+ * creates once per device.  Those streams start after the work already queued
+ * on cuda_stream, and cuda_stream waits for the last copy back, so the call is
+ * asynchronous on cuda_stream like the device entry points: the host buffers
+ * must stay valid, and o and S_out must not be read, until cuda_stream has
+ * passed this call (cudaStreamSynchronize).  The copies only overlap when the
+ * host buffers are page-locked (cudaHostAlloc / cudaHostRegister); pageable
+ * memory gives the same results more slowly.
+ *
+ *   workspace  DEVICE buffer of deltanet_host_workspace_bytes(...) bytes,
+ *              16-byte aligned, cleared once with deltanet_workspace_init;
+ *              its status word is read with deltanet_get_device_status.
+ * Errors as deltanet_chunk_fwd; o must not overlap an input, S_out may equal
+ * S0.  Concurrent calls on one device are queued one after the other.
+ */
+int deltanet_chunk_fwd_host(const void *q, const void *k, const void *v,
+                            const float *beta, const float *alpha, const float *S0,
+                            void *o, float *S_out,
+                            int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                            void *workspace, size_t ws_bytes, void *cuda_stream);
+
 /* Static string for a status code. */
 const char *deltanet_status_string(int status);
 

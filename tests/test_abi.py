@@ -116,6 +116,52 @@ def test_chunk_rejects_overlaps(L):
     assert _chunk(L, ws=A + 256 * MB) == E.DN_ERR_INVALID_ARG  # workspace inside o
 
 
+def test_host_workspace_bytes(L):
+    """Status word + two staging slots of ceil(B*H/8) heads, every region on a
+    256-byte boundary: q, k, v, o, beta, alpha, S0, S_out and the group's
+    pre-pass factors (4 C^2 + 4 C bytes per chunk for bf16)."""
+    r = lambda x: (x + 255) // 256 * 256
+    for (B, H, T, Dk, Dv, C, dt) in [(4, 16, 4096, 128, 128, 64, 1), (3, 5, 333, 128, 64, 64, 0),
+                                     (1, 1, 200, 64, 128, 128, 1), (2, 3, 0, 64, 64, 64, 1)]:
+        Hg = (B * H + 7) // 8
+        es = 2 if dt == 1 else 4
+        tok = Hg * T
+        wy = Hg * ((T + C - 1) // C) * (4 * C * C + 4 * C) if (dt == 1 and T > 0) else 0
+        slot = (2 * r(tok * Dk * es) + 2 * r(tok * Dv * es) + 2 * r(tok * 4)
+                + 2 * r(Hg * Dk * Dv * 4) + r(wy))
+        assert L.deltanet_host_workspace_bytes(B, H, T, Dk, Dv, C, dt) == 256 + 2 * slot
+    assert L.deltanet_host_workspace_bytes(4, 16, 4096, 96, 128, 64, 1) == 0
+    assert L.deltanet_host_workspace_bytes(4, 16, 4096, 128, 128, 64, 7) == 0
+    assert L.deltanet_host_workspace_bytes(-1, 16, 4096, 128, 128, 64, 1) == 0
+
+
+def _chunk_host(L, q=A, k=A + 64 * MB, v=A + 128 * MB, beta=A + 192 * MB, alpha=None, S0=None,
+                o=A + 256 * MB, S_out=A + 320 * MB, B=2, H=2, T=100, Dk=64, Dv=64, C=64, dt=1,
+                ws=A + 400 * MB, ws_bytes=None):
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    if ws_bytes is None:
+        ws_bytes = max(256, L.deltanet_host_workspace_bytes(max(B, 0), max(H, 0), max(T, 0), 64, 64, 64, 1))
+    return L.deltanet_chunk_fwd_host(vp(q), vp(k), vp(v), vp(beta), vp(alpha), vp(S0), vp(o),
+                                     vp(S_out), B, H, T, Dk, Dv, C, dt, vp(ws), ws_bytes, None)
+
+
+def test_chunk_host_rejects_bad_arguments(L):
+    """The host-buffer call validates like the device call, before any CUDA
+    call; its host pointers need no alignment, its workspace does."""
+    E = _lib
+    assert _chunk_host(L, q=None) == E.DN_ERR_INVALID_ARG
+    assert _chunk_host(L, beta=None) == E.DN_ERR_INVALID_ARG
+    assert _chunk_host(L, B=-1) == E.DN_ERR_INVALID_ARG
+    assert _chunk_host(L, Dk=96) == E.DN_ERR_UNSUPPORTED
+    assert _chunk_host(L, C=32) == E.DN_ERR_UNSUPPORTED
+    assert _chunk_host(L, ws=None) == E.DN_ERR_WORKSPACE
+    assert _chunk_host(L, ws_bytes=1024) == E.DN_ERR_WORKSPACE
+    assert _chunk_host(L, ws=A + 400 * MB + 8) == E.DN_ERR_ALIGNMENT
+    assert _chunk_host(L, o=A + 4096) == E.DN_ERR_INVALID_ARG  # o inside q
+    S0 = A + 500 * MB
+    assert _chunk_host(L, S0=S0, S_out=S0 + 256) == E.DN_ERR_INVALID_ARG  # partial overlap
+
+
 def test_decode_rejects_bad_arguments(L):
     E = _lib
     vp = ctypes.c_void_p
