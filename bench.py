@@ -536,7 +536,7 @@ def main():
     e2e = {"value": whole_job_rate(world, tokens, args.e2e_steps, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": e2e_ms / args.e2e_steps,
-           "path": "deltanet_chunk_fwd_host: pinned host buffers in and out, heads in 8 groups"}
+           "path": "deltanet_chunk_fwd_host: pinned host buffers in and out, heads in 4 groups"}
     del hx, ho, hS, hws
 
     extras = None

@@ -120,7 +120,7 @@ int run_chunked(dn::ChunkProblem& p, void* ws, void* stream) {
 // ------------------------------------------------------------ host buffers --
 // The host-buffer call streams the heads through the device in kHostGroups
 // groups, two staging slots in the workspace, on three library streams.
-constexpr int kHostGroups = 8;
+constexpr int kHostGroups = 4;
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 

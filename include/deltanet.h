@@ -211,7 +211,7 @@ int deltanet_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
  * word, then two staging slots, each holding one group of heads' q, k, v, o,
  * beta, alpha, S0 and S_out plus that group's pre-pass factors (the per-chunk
  * factors of deltanet_workspace_bytes for the group's heads).  The heads are
- * taken in groups of ceil(B*H / 8).  Each region starts on a 256-byte boundary.
+ * taken in groups of ceil(B*H / 4).  Each region starts on a 256-byte boundary.
  * Returns 0 for sizes the library rejects.
  */
 size_t deltanet_host_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt);
@@ -220,7 +220,7 @@ size_t deltanet_host_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C,
  * deltanet_chunk_fwd on HOST buffers: q, k, v, beta, alpha, S0, o and S_out
  * have the shapes, types and meaning of deltanet_chunk_fwd's arguments but
  * live in host memory (no alignment needed).  The heads pass through the
- * device in groups of ceil(B*H / 8): the host-to-device copy of one group,
+ * device in groups of ceil(B*H / 4): the host-to-device copy of one group,
  * the computation of the group before it and the device-to-host copy of the
  * group before that run at the same time, on three streams the library
  * creates once per device.  Those streams start after the work already queued

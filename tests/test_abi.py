@@ -117,13 +117,13 @@ def test_chunk_rejects_overlaps(L):
 
 
 def test_host_workspace_bytes(L):
-    """Status word + two staging slots of ceil(B*H/8) heads, every region on a
+    """Status word + two staging slots of ceil(B*H/4) heads, every region on a
     256-byte boundary: q, k, v, o, beta, alpha, S0, S_out and the group's
     pre-pass factors (4 C^2 + 4 C bytes per chunk for bf16)."""
     r = lambda x: (x + 255) // 256 * 256
     for (B, H, T, Dk, Dv, C, dt) in [(4, 16, 4096, 128, 128, 64, 1), (3, 5, 333, 128, 64, 64, 0),
                                      (1, 1, 200, 64, 128, 128, 1), (2, 3, 0, 64, 64, 64, 1)]:
-        Hg = (B * H + 7) // 8
+        Hg = (B * H + 3) // 4
         es = 2 if dt == 1 else 4
         tok = Hg * T
         wy = Hg * ((T + C - 1) // C) * (4 * C * C + 4 * C) if (dt == 1 and T > 0) else 0

@@ -50,7 +50,7 @@ def _host_call(dn, x, S0, C, in_place=False):
 
 @pytest.mark.parametrize("B,H,T,Dk,Dv,dtype,gated,C", [
     (1, 1, 200, 128, 128, torch.bfloat16, False, 64),   # one group of one head
-    (3, 5, 333, 128, 64, torch.bfloat16, True, 64),     # 15 heads: groups of 2, last one short
+    (3, 5, 333, 128, 64, torch.bfloat16, True, 64),     # 15 heads: groups of 4, last one short
     (2, 8, 256, 128, 128, torch.bfloat16, False, 128),  # C = 128
     (2, 3, 150, 64, 64, torch.float32, True, 64),       # the float32 path
 ])
