@@ -17,8 +17,10 @@
 //      accumulator in TMEM), read back row by row into A, masked and scaled.
 //   3. C/16 diagonal 16x16 inverses (one column per lane, right-looking
 //      substitution so only one multiply-add per step is on the dependency
-//      chain), then each warp finishes one 16-column block of T by block
-//      forward substitution with tf32 WMMA products, T_iw = -D_i sum A_im T_mw.
+//      chain), then the blocks below the diagonal from the 2 x 2 block
+//      inverse [[L11, 0], [L21, L22]]^-1 = [[T1, 0], [-T2 L21 T1, T2]] applied
+//      recursively (64 x 64 halves of 32 x 32 halves), with tf32 WMMA products
+//      spread over all warps: four dependent levels at C = 64, six at C = 128.
 //   4. Tb, Tbg -> global (row-major bf16 C x C tiles).
 #include <cuda_bf16.h>
 #include <mma.h>
@@ -248,8 +250,9 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
   //    the inverses of the diagonal halves, each [[D_a, 0], [-D_b A_ba D_a, D_b]]:
   //      1. A10 D0, A32 D2            2. T10 = -D1 (A10 D0), T32 = -D3 (A32 D2)
   //      3. X = L21 T1 (four tiles)   4. T21 = -T2 X (four tiles)
-  //    Scratch tiles sit in A's unused upper blocks.  C = 128, column block
-  //    w (warp w) by block forward substitution, T_iw = -D_i sum_m A_im T_mw.
+  //    Scratch tiles sit in A's unused upper blocks.  C = 128 applies the same
+  //    split once more: both 64 x 64 halves by the four levels, then
+  //    T21 = -T2 (L21 T1) in two levels.
   {
     using FragA = wmma::fragment<wmma::matrix_a, 16, 16, 8, wmma::precision::tf32, wmma::row_major>;
     using FragB = wmma::fragment<wmma::matrix_b, 16, 16, 8, wmma::precision::tf32, wmma::row_major>;
@@ -276,57 +279,77 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
     };
     auto At = [&](int i, int j) { return Am + (16 * i) * kApad + 16 * j; };  // also the scratch tiles (j > i)
     auto Tt = [&](int i, int j) { return Tm + (16 * i) * kApad + 16 * j; };
-    if constexpr (kC == 64) {
+    // Levels 1-4 on the 64 x 64 diagonal block starting at 16 x 16 block b0,
+    // by the four warps with local index wl (every thread passes the barriers).
+    auto half_solve = [&](int b0, int wl) {
       FragC acc;
-      if (warp < 2) {  // level 1: A10 D0 -> S01, A32 D2 -> S23
-        const int a = 2 * warp;
+      if (wl < 2) {  // level 1: A10 D0 -> S01, A32 D2 -> S23
+        const int a = b0 + 2 * wl;
         wmma::fill_fragment(acc, 0.f);
         mac(acc, At(a + 1, a), Tt(a, a));
         put(At(a, a + 1), acc, false);
       }
       __syncthreads();
-      if (warp < 2) {  // level 2: T10 = -D1 S01, T32 = -D3 S23
-        const int a = 2 * warp;
+      if (wl < 2) {  // level 2: T10 = -D1 S01, T32 = -D3 S23
+        const int a = b0 + 2 * wl;
         wmma::fill_fragment(acc, 0.f);
         mac(acc, Tt(a + 1, a + 1), At(a, a + 1));
         put(Tt(a + 1, a), acc, true);
       }
       __syncthreads();
       {  // level 3: X_rc = sum_m A_rm T1_mc for r in {2, 3}, c in {0, 1} -> S_c(r)
-        const int r = 2 + (warp >> 1), cc = warp & 1;
+        const int r = b0 + 2 + (wl >> 1), cc = b0 + (wl & 1);
         wmma::fill_fragment(acc, 0.f);
-        if (cc == 0) {
-          mac(acc, At(r, 0), Tt(0, 0));
-          mac(acc, At(r, 1), Tt(1, 0));
+        if (cc == b0) {
+          mac(acc, At(r, b0), Tt(b0, b0));
+          mac(acc, At(r, b0 + 1), Tt(b0 + 1, b0));
         } else {
-          mac(acc, At(r, 1), Tt(1, 1));
+          mac(acc, At(r, b0 + 1), Tt(b0 + 1, b0 + 1));
         }
         put(At(cc, r), acc, false);
       }
       __syncthreads();
       {  // level 4: T_rc = -sum_m T2_rm X_mc
-        const int r = 2 + (warp >> 1), cc = warp & 1;
+        const int r = b0 + 2 + (wl >> 1), cc = b0 + (wl & 1);
         wmma::fill_fragment(acc, 0.f);
-        if (r == 2) {
-          mac(acc, Tt(2, 2), At(cc, 2));
+        if (r == b0 + 2) {
+          mac(acc, Tt(b0 + 2, b0 + 2), At(cc, b0 + 2));
         } else {
-          mac(acc, Tt(3, 2), At(cc, 2));
-          mac(acc, Tt(3, 3), At(cc, 3));
+          mac(acc, Tt(b0 + 3, b0 + 2), At(cc, b0 + 2));
+          mac(acc, Tt(b0 + 3, b0 + 3), At(cc, b0 + 3));
         }
         put(Tt(r, cc), acc, true);
       }
+    };
+    if constexpr (kC == 64) {
+      half_solve(0, warp);
     } else {
+      // C = 128: the two 64 x 64 halves at once (warps 0-3 and 4-7), then the
+      // block below them, T21 = -T2 (L21 T1), in two more levels of 16 tiles
+      // (two per warp, paired so that every warp does five products).
+      half_solve(4 * (warp >> 2), warp & 3);
+      __syncthreads();
       FragC acc;
-      float* xs = At(warp, Sh::kWarps - 1);  // 16 x 16 scratch in A's unused upper part
-      for (int i = warp + 1; i < Sh::kWarps; ++i) {
-        wmma::fill_fragment(acc, 0.f);
-        for (int m = warp; m < i; ++m) mac(acc, At(i, m), Tt(m, warp));
-        put(xs, acc, false);
-        __syncwarp();
-        wmma::fill_fragment(acc, 0.f);
-        mac(acc, Tt(i, i), xs);
-        put(Tt(i, warp), acc, true);
-        __syncwarp();
+      {  // level 5: X_rc = sum_{m=c..3} A_rm T1_mc, r in 4..7, c in 0..3 -> S(c, r)
+        const int r = 4 + (warp >> 1);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int cc = (warp & 1) ? 1 + t : 3 * t;
+          wmma::fill_fragment(acc, 0.f);
+          for (int m = cc; m < 4; ++m) mac(acc, At(r, m), Tt(m, cc));
+          put(At(cc, r), acc, false);
+        }
+      }
+      __syncthreads();
+      {  // level 6: T_rc = -sum_{m=4..r} T2_rm X_mc
+        const int cc = warp >> 1;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int r = (warp & 1) ? 5 + t : 4 + 3 * t;
+          wmma::fill_fragment(acc, 0.f);
+          for (int m = 4; m <= r; ++m) mac(acc, Tt(r, m), At(cc, m));
+          put(Tt(r, cc), acc, true);
+        }
       }
     }
   }
