@@ -361,16 +361,25 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
     const size_t tile = ((size_t)bh * nchunks + chunk) * kC * kC;
     constexpr int kTpr = kC / 8;  // threads per row
     const int c8 = (tid % kTpr) * 8;
+    // this thread's eight columns of beta (and e^g): 16-byte aligned vector loads
+    float bcol[8], ecol[8];
+    *reinterpret_cast<float4*>(bcol) = *reinterpret_cast<const float4*>(vb + c8);
+    *reinterpret_cast<float4*>(bcol + 4) = *reinterpret_cast<const float4*>(vb + c8 + 4);
+    if (GATED) {
+      *reinterpret_cast<float4*>(ecol) = *reinterpret_cast<const float4*>(veg + c8);
+      *reinterpret_cast<float4*>(ecol + 4) = *reinterpret_cast<const float4*>(veg + c8 + 4);
+    }
 #pragma unroll
     for (int pass = 0; pass < kC / 16; ++pass) {
       const int row = pass * 16 + tid / kTpr;
-      const float* trow = Tm + row * kApad + c8;
-      float x[8], y[8];
+      const float* trow = Tm + row * kApad + c8;  // 16-byte aligned (kApad * 4 and c8 * 4 are)
+      float t8[8], x[8], y[8];
+      *reinterpret_cast<float4*>(t8) = *reinterpret_cast<const float4*>(trow);
+      *reinterpret_cast<float4*>(t8 + 4) = *reinterpret_cast<const float4*>(trow + 4);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int sc = c8 + e;
-        x[e] = sc <= row ? trow[e] * vb[sc] : 0.f;
-        if (GATED) y[e] = x[e] * veg[sc];
+        x[e] = c8 + e <= row ? t8[e] * bcol[e] : 0.f;
+        if (GATED) y[e] = x[e] * ecol[e];
       }
       st_bf16x8(tb_out + tile + row * kC + c8, x);
       if (GATED) st_bf16x8(tbg_out + tile + row * kC + c8, y);
