@@ -42,15 +42,19 @@ struct TsolveShape {
 };
 
 // Shared memory: the K tile (128-byte swizzled, KB blocks of C rows x 128 B,
-// from TMA) shares its region with T, which is written only after the Gram has
-// read K; A follows.  At C = 64 the M = 128 Gram operand's rows 64-127 read
-// whatever follows a block (still inside this CTA's shared memory; those TMEM
-// rows are not used).
+// from TMA), then A.  At C = 64, T shares its region with the K tile (T is
+// written only after the Gram has read K), and the M = 128 Gram operand's rows
+// 64-127 read whatever follows a block (still inside this CTA's shared memory;
+// those TMEM rows are not used).  At C = 128, T is built in place of A (every
+// block of A is read for the last time in the level before the one that writes
+// that block of T), which keeps the CTA at 103 KB so that two fit on an SM.
 template <int C, int DK>
 struct TsolveSmem {
+  static constexpr bool kInPlace = C == 128;
   static constexpr uint32_t kKBytes = (DK / 64) * C * 128;
   static constexpr uint32_t kTBytes = C * TsolveShape<C>::kApad * 4;
-  static constexpr uint32_t kRegion = ((kKBytes > kTBytes ? kKBytes : kTBytes) + 1023) / 1024 * 1024;
+  static constexpr uint32_t kRegion =
+      ((kInPlace || kKBytes > kTBytes ? kKBytes : kTBytes) + 1023) / 1024 * 1024;
   static constexpr uint32_t AM_OFF = kRegion;
   static constexpr uint32_t VEC_OFF = AM_OFF + kTBytes;  // beta, g, e^g, e^(m-g) (C each), 8 warp totals
   static constexpr uint32_t BAR_OFF = (VEC_OFF + (4 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
@@ -69,7 +73,7 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
 }
 
 template <int C, int DK, bool GATED>
-__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
+__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
                   const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
                   __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out, int T, int nchunks,
@@ -81,8 +85,9 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsolve_smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const uint32_t sb = warp_uniform(smem_u32(sm));
-  float* Tm = reinterpret_cast<float*>(sm);  // reuses the K tile after the Gram
   float* Am = reinterpret_cast<float*>(sm + SL::AM_OFF);
+  // T: over the K tile after the Gram (C = 64), or in place of A (C = 128)
+  float* Tm = SL::kInPlace ? Am : reinterpret_cast<float*>(sm);
   float* vb = reinterpret_cast<float*>(sm + SL::VEC_OFF);
   float* vg = vb + kC;
   float* veg = vg + kC;
@@ -240,6 +245,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 1)
 #pragma unroll
       for (int i = m + 1; i < 16; ++i) acc[i] = fmaf(Am[(o + i) * kApad + o + m], col[m], acc[i]);
     }
+    __syncwarp(0x0000FFFFu);  // every lane has read its block of A before T may overwrite it
 #pragma unroll
     for (int i = 0; i < 16; ++i) Tm[(o + i) * kApad + o + j] = col[i];
   }
