@@ -42,25 +42,27 @@ struct TsolveShape {
 };
 
 // Shared memory: the K tile (128-byte swizzled, KB blocks of C rows x 128 B,
-// from TMA), then A.  At C = 64, T shares its region with the K tile (T is
-// written only after the Gram has read K), and the M = 128 Gram operand's rows
-// 64-127 read whatever follows a block (still inside this CTA's shared memory;
-// those TMEM rows are not used).  At C = 128, T is built in place of A (every
-// block of A is read for the last time in the level before the one that writes
-// that block of T), which keeps the CTA at 103 KB so that two fit on an SM.
+// from TMA) and A, with T built in place of A (every block of A is read for
+// the last time in the level before the one that writes that block of T).
+// At C = 64, A also shares its region with the K tile (A is written only after
+// the Gram has read K), and the region extends 8 KB past the tile: the M = 128
+// Gram operand's rows 64-127 read whatever follows a block (those TMEM rows are
+// not used).  That keeps the CTA at 26 KB, eight per SM; at C = 128, K and A
+// side by side take 103 KB, two per SM.
 template <int C, int DK>
 struct TsolveSmem {
-  static constexpr bool kInPlace = C == 128;
   static constexpr uint32_t kKBytes = (DK / 64) * C * 128;
   static constexpr uint32_t kTBytes = C * TsolveShape<C>::kApad * 4;
+  static constexpr uint32_t round1k(uint32_t x) { return (x + 1023) / 1024 * 1024; }
+  static constexpr uint32_t AM_OFF = C == 64 ? 0 : round1k(kKBytes);
   static constexpr uint32_t kRegion =
-      ((kInPlace || kKBytes > kTBytes ? kKBytes : kTBytes) + 1023) / 1024 * 1024;
-  static constexpr uint32_t AM_OFF = kRegion;
-  static constexpr uint32_t VEC_OFF = AM_OFF + kTBytes;  // beta, g, e^g, e^(m-g) (C each), 8 warp totals
+      C == 64 ? round1k(kTBytes > kKBytes + 8192 ? kTBytes : kKBytes + 8192) : AM_OFF + kTBytes;
+  static constexpr uint32_t VEC_OFF = kRegion;  // beta, g, e^g, e^(m-g) (C each), 8 warp totals
   static constexpr uint32_t BAR_OFF = (VEC_OFF + (4 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
   static constexpr uint32_t BYTES = BAR_OFF + 32;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // 1024-byte alignment of the K tile
-  static_assert(C == 128 || kRegion + 8192 <= BYTES, "M = 128 operand rows past the K tile stay inside");
+  static_assert(C == 128 || kKBytes + 8192 <= BYTES, "M = 128 operand rows past the K tile stay inside");
+  static_assert(VEC_OFF % 16 == 0 && AM_OFF % 1024 == 0, "vector loads and the swizzled K tile stay aligned");
 };
 
 // tf32 operands by truncation: keep the sign, exponent and top 10 mantissa bits
@@ -73,7 +75,7 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
 }
 
 template <int C, int DK, bool GATED>
-__global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 2)
+__global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
                   const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
                   __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out, int T, int nchunks,
@@ -86,8 +88,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 6 : 2)
                                            ~uintptr_t(1023));
   const uint32_t sb = warp_uniform(smem_u32(sm));
   float* Am = reinterpret_cast<float*>(sm + SL::AM_OFF);
-  // T: over the K tile after the Gram (C = 64), or in place of A (C = 128)
-  float* Tm = SL::kInPlace ? Am : reinterpret_cast<float*>(sm);
+  float* Tm = Am;  // T is built in place of A
   float* vb = reinterpret_cast<float*>(sm + SL::VEC_OFF);
   float* vg = vb + kC;
   float* veg = vg + kC;
