@@ -8,10 +8,10 @@
 // transformers with delta rule)"); the chunk kernel then applies them with
 // tensor-core products, keeping only matrix products on its serial state chain.
 //
-// One CTA of 2C threads (one warp per 16-row block) per chunk, several CTAs per
-// SM at C = 64: the solve is a short chain
-// of dependent steps, so it is latency-bound per chunk and the grid's
-// parallelism over chunks hides that latency.
+// One CTA of 2C threads (one warp per 16-row block) per chunk, eight CTAs per
+// SM at C = 64 and two at C = 128: the solve is a short chain of dependent
+// steps, so it is latency-bound per chunk and the grid's parallelism over
+// chunks hides that latency.
 //   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
 //   2. G = K K^T by tcgen05 (bf16 operands from the swizzled K tile, float32
 //      accumulator in TMEM), read back row by row into A, masked and scaled.
