@@ -16,12 +16,12 @@
 // denominator.  Only S and z carry from chunk to chunk, and their increment
 // does not depend on them, so everything but the accumulate is pipelined ahead.
 //
-// One CTA per (b, h, 64-column slice of Dv), 10 warps:
-//   warp 8     producer: TMA of K, Q, V into a three-stage ring
-//   warp 9     MMA issuer (warp-uniform, one elected lane): Gram (c+1) and
+// One CTA per (b, h, 64-column slice of Dv), 14 warps:
+//   warp 12    producer: TMA of K, Q, V into a three-stage ring
+//   warp 13    MMA issuer (warp-uniform, one elected lane): Gram (c+1) and
 //              K'^T [V|1] (c+1) while chunk c waits for its state tile, then
 //              O (c) = Q'[S|z] + P[V|1]
-//   warps 4-7  prep: feature maps in place (rows past T zeroed)
+//   warps 4-11 prep: feature maps in place (rows past T zeroed)
 //   warps 0-3  state: [S|z] += K'^T [V|1] in float32 registers, the bf16
 //              state tile for the next chunk (double-buffered); warps 2-3 turn
 //              the Gram rows (TMEM lanes 64-127) into P; warps 0-1 drain
@@ -45,7 +45,8 @@ constexpr int kDVS = 64;
 constexpr int NST = 3;
 constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
 constexpr int kWG = 128;
-constexpr int kThreads = 2 * kWG + 64;  // state 0-3, prep 4-7, producer 8, issuer 9
+constexpr int kPrep = 256;                  // prep threads (warps 4-11)
+constexpr int kThreads = kWG + kPrep + 64;  // state 0-3, prep 4-11, producer 12, issuer 13
 constexpr int kBarState = 1, kBarLo = 2, kBarHi = 3, kBarPrep = 4;
 constexpr int kNA = 80;  // augmented width: 64 columns of V (or S) + the ones (or z) column, padded to 16
 
@@ -70,6 +71,13 @@ struct LinLayout {
   static_assert(STAGE % 1024 == 0 && P_OFF % 1024 == 0, "128-byte swizzle atoms stay aligned");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
+
+// One 32-bit column of this thread's TMEM lane (z or the denominator Q'z + P 1).
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
 
 // mbarrier slots (8 bytes each).  FULL, EMPTY and FMAP per stage; the rest per
 // chunk parity.
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -172,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = issued > NST ? issued - NST : 0; c < issued; ++c)
         (void)mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, drain);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // -------------------------------------------------------------- issuer --
     // Gram (c) = [K'; Q'] K'^T into G[c & 1] and dS (c) = K'^T V into dS[c & 1]
     auto issue_gram_ds = [&](int c) {
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < nchunks && ok; ++c) {
       const int n = min(kC, T - c * kC);
       uint8_t* stp = sm + (c % NST) * L::STAGE;
-      ok = named_bar_and(kBarPrep, kWG, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
+      ok = named_bar_and(kBarPrep, kPrep, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
       // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0) ----
       // Four 16-byte pieces per thread per round, in stages (all loads, all
@@ -256,14 +264,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // elements are in flight together.
       constexpr int kPieces = L::KB * 2 * (int)(kTile / 16);  // 16-byte pieces of the K and Q tiles
       constexpr int kNpf = 4;
-      static_assert(kPieces % (kNpf * kWG) == 0, "whole rounds of pieces per thread");
-      for (int i0 = pt; i0 < kPieces; i0 += kNpf * kWG) {
+      static_assert(kPieces % (kNpf * kPrep) == 0, "whole rounds of pieces per thread");
+      for (int i0 = pt; i0 < kPieces; i0 += kNpf * kPrep) {
         uint4 u[kNpf];
         uint8_t* ptr[kNpf];
         bool live[kNpf];
 #pragma unroll
         for (int j = 0; j < kNpf; ++j) {
-          const int i = i0 + j * kWG;
+          const int i = i0 + j * kPrep;
           const int t16 = i / (int)(kTile / 16), off = (i % (int)(kTile / 16)) * 16;
           ptr[j] = stp + (t16 >> 1) * L::KB_STRIDE + (t16 & 1) * kTile + off;
           live[j] = (off >> 7) < n;
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      named_bar_sync(kBarPrep, kWG);
+      named_bar_sync(kBarPrep, kPrep);
       if (pt == 0) mbar_arrive(bar + B_FMAP + 8 * (c % NST));
     }
   } else {
@@ -361,14 +369,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (ct < DK) {
         const uint32_t d0 = tmem + lane_base + TM_DS + kAugStride * b;
-        uint32_t ds[64], dz[32];
+        uint32_t ds[64];
         tmem_ld32(d0, *reinterpret_cast<uint32_t(*)[32]>(ds));
         tmem_ld32(d0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
-        tmem_ld32(d0 + 64, dz);
+        const uint32_t dz = tmem_ld1(d0 + 64);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 64; ++e) sreg[e] += __uint_as_float(ds[e]);
-        zreg += __uint_as_float(dz[0]);
+        zreg += __uint_as_float(dz);
       }
       tc_fence_before();
       named_bar_sync(kBarState, kWG);
@@ -389,13 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok_lo) {
           tc_fence_after();
           const uint32_t o0 = tmem + lane_base + TM_O + kAugStride * b;
-          uint32_t ov[64], od[32];
+          uint32_t ov[64];
           tmem_ld32(o0, *reinterpret_cast<uint32_t(*)[32]>(ov));
           tmem_ld32(o0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
-          tmem_ld32(o0 + 64, od);
+          const uint32_t od = tmem_ld1(o0 + 64);
           tmem_wait_ld();
           if (row < n) {
-            const float inv = 1.f / __uint_as_float(od[0]);
+            const float inv = 1.f / __uint_as_float(od);
             __nv_bfloat16* orow =
                 static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c * kC + row) * Dv + j0;
 #pragma unroll
