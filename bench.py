@@ -3,7 +3,8 @@
 
 Headline: the chunked DeltaNet forward on the prefill workload (B4 H16 T4096,
 Dk = Dv = 128, bf16 q/k/v, fp32 beta and state, C = 64, S0 = 0), tokens/s over
-all GPUs.  One step = one deltanet_chunk_fwd call over one batch (two
+all GPUs, a token being one position of one sequence with all of its heads
+(tokens/s = B * T / time; the head-token rate B * H * T / time is 16x that).  One step = one deltanet_chunk_fwd call over one batch (two
 launches: the chunk-parallel WY pre-pass and the chunk kernel).  Inputs are resident in HBM when the timed region starts;
 two input sets alternate so consecutive steps touch disjoint 274 MB working
 sets (larger than the 126 MB L2).
@@ -105,18 +106,24 @@ class ClockSampler:
         except Exception:
             self._handle = None
 
-    def _run(self):
+    def sample_now(self):
+        """Take one sample (read-only NVML queries)."""
+        if self._handle is None:
+            return
         nv, h = self._nvml, self._handle
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+            self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-                self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
-            except Exception:
-                pass
+            self.sample_now()
             self._stop.wait(0.01)
 
     def __enter__(self):
@@ -205,6 +212,8 @@ def time_region(step, K, W, world, stream, sampler=None):
         for i in range(K):
             step(i)
         end.record(stream)
+        if sampler is not None:  # the queued steps are running now: one more sample
+            sampler.sample_now()
         end.synchronize()
     torch.cuda.synchronize()
     barrier(world)
@@ -271,7 +280,7 @@ def cpu_oracle_rate(target_s=10.0, max_reps=4):
         t0 = time.perf_counter()
         oracle.deltanet(x["q"], x["k"], x["v"], x["beta"], nthreads=cores)
         secs += time.perf_counter() - t0
-        tokens += w.B * w.H * w.T
+        tokens += w.B * w.T  # tokens of all heads: B * T per pass
         reps += 1
     sample = (f"{reps} pass(es) over the full prefill workload (B4 H16 T4096 D128 bf16 inputs), "
               f"float64 per-token recurrence, {cores} threads over (b,h)")
@@ -310,10 +319,13 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     secs = time.perf_counter() - t0
-    tok = nseq * L * args.steps
+    # a token of the workload carries H heads: nseq (b, h) sequences of L
+    # positions are nseq * L / H tokens
+    tok = nseq * L * args.steps / w.H
     value = tok / secs
-    sample = (f"per step: {nseq} sequences x {L} tokens of the prefill workload "
-              f"(D128, bf16 inputs), float64 per-token recurrence, {cores} threads")
+    sample = (f"per step: {nseq} (b,h) sequences x {L} positions of the prefill workload "
+              f"(D128, bf16 inputs; {nseq * L / w.H:g} tokens of {w.H} heads), float64 per-token "
+              f"recurrence, {cores} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -358,7 +370,7 @@ def extras_measure(dn, gen, dev, stream, peaks):
     z = torch.empty(w.B, w.H, w.Dk, device=dev)
     ms = timed(lambda: dn.linear_attn_fwd(x["q"], x["k"], x["v"], C=w.C, o=o, S_out=S, z_out=z), 20)
     fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C, linear=True)
-    out["linear_attn_prefill"] = {"tokens_per_s": w.B * w.H * w.T / (ms * 1e-3), "ms": ms,
+    out["linear_attn_prefill"] = {"tokens_per_s": w.B * w.T / (ms * 1e-3), "ms": ms,
                                   "GBps": by / (ms * 1e-3) / 1e9,
                                   "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm,
                                   "TFLOPs": fl / (ms * 1e-3) / 1e12,
@@ -373,7 +385,7 @@ def extras_measure(dn, gen, dev, stream, peaks):
     ms = timed(lambda: dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C,
                                              o=o, S_out=S), 5)
     fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C, gated=True)
-    out["gated_forget"] = {"tokens_per_s": w.B * w.H * w.T / (ms * 1e-3), "ms": ms,
+    out["gated_forget"] = {"tokens_per_s": w.B * w.T / (ms * 1e-3), "ms": ms,
                            "GBps": by / (ms * 1e-3) / 1e9, "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm,
                            "TFLOPs": fl / (ms * 1e-3) / 1e12, "tc_frac": fl / (ms * 1e-3) / 1e12 / tc}
     del x, o, S
@@ -390,7 +402,7 @@ def extras_measure(dn, gen, dev, stream, peaks):
             out[f"long_C{w.C}"] = {"unavailable": str(e)}
             continue
         fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
-        out[f"long_C{w.C}"] = {"tokens_per_s": w.B * w.H * w.T / (ms * 1e-3), "ms": ms,
+        out[f"long_C{w.C}"] = {"tokens_per_s": w.B * w.T / (ms * 1e-3), "ms": ms,
                                "GBps": by / (ms * 1e-3) / 1e9,
                                "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm,
                                "TFLOPs": fl / (ms * 1e-3) / 1e12,
@@ -501,7 +513,7 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
     ms_step = ms / args.steps
-    tokens = w.B * w.H * w.T
+    tokens = w.B * w.T  # B * T tokens per step, each with all H heads
     value = whole_job_rate(world, tokens, args.steps, ms)
 
     flop, byts = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
@@ -510,6 +522,9 @@ def main():
     traffic = traffic_from_profile()
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "traffic_source": (f"ncu profile summary profiles/{PROFILE_SUMMARY} (DRAM read + write "
+                               "of one call), matched to the current kernel sources by hash")
+            if traffic is not None else "no profile of the current kernel sources",
             "peak_source": peak_src, "algorithmic_bytes_per_launch": byts,
             "tensor": {"achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                        "frac": tflops / peaks["bf16_tflops"], "algorithmic_flop_per_launch": flop}}
@@ -559,6 +574,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "Dk": w.Dk, "Dv": w.Dv,
                        "C": w.C, "state": "fp32", "per_gpu": "independent batch per GPU",
+                       "tokens_per_step": tokens, "head_tokens_per_step": tokens * w.H,
                        "parallelism": f"dp{world}",
                        "l2": "inputs larger than L2: two alternating input sets of 274 MB each"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * args.steps,

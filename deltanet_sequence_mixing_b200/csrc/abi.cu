@@ -42,7 +42,11 @@ int validate_problem(const dn::ChunkProblem& p) {
   if (p.bf16 != 0 && p.bf16 != 1) return DN_ERR_INVALID_ARG;
   if (!valid_dim(p.Dk) || !valid_dim(p.Dv)) return DN_ERR_UNSUPPORTED;
   if (p.C != 64 && p.C != 128) return DN_ERR_UNSUPPORTED;
+  // C = 128 is built for the bf16 delta rule only
+  if (p.C == 128 && (!p.bf16 || p.mode != dn::Mode::Delta)) return DN_ERR_UNSUPPORTED;
   if ((long long)p.B * p.H > INT_MAX) return DN_ERR_UNSUPPORTED;
+  // the pre-pass runs one CTA per (b, h, chunk), on a one-dimensional grid
+  if ((long long)p.B * p.H * ((p.T + (long long)p.C - 1) / p.C) > INT_MAX) return DN_ERR_UNSUPPORTED;
   // With T == 0 no token buffer is ever dereferenced (empty tensors may carry a
   // null data pointer); otherwise every token buffer is required.
   if (p.T > 0) {
@@ -103,6 +107,17 @@ int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws)
 int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStream_t st) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
   p.status = status;
+  if (p.T == 0) {  // no tokens: the final state (and normaliser) is the initial one
+    const size_t BH = (size_t)p.B * p.H;
+    auto carry = [&](float* dst, const float* src, size_t bytes) {
+      if (!dst || dst == src) return cudaSuccess;
+      return src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st)
+                 : cudaMemsetAsync(dst, 0, bytes, st);
+    };
+    cudaError_t e = carry(p.S_out, p.S0, BH * p.Dk * p.Dv * sizeof(float));
+    if (e == cudaSuccess && p.mode == dn::Mode::Linear) e = carry(p.z_out, p.z0, BH * p.Dk * sizeof(float));
+    return map_cuda(e);
+  }
   if (dn::chunk_main_supported(p) || dn::chunk128_supported(p)) {
     const dn::WyWorkspace w = dn::wy_carve(wy, p.B, p.H, p.T, p.C);
     return map_cuda(p.C == 64 ? dn::launch_chunk_main(p, w, st) : dn::launch_chunk128(p, w, st));
@@ -187,6 +202,8 @@ extern "C" {
 size_t deltanet_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
   if (B < 0 || H < 0 || T < 0 || !valid_dim(Dk) || !valid_dim(Dv)) return 0;
   if ((C != 64 && C != 128) || (dt != DN_F32 && dt != DN_BF16)) return 0;
+  if (C == 128 && dt != DN_BF16) return 0;  // C = 128 is built for bf16 only
+  if ((long long)B * H * (((long long)T + C - 1) / C) > INT_MAX) return 0;
   // bf16: room for the per-chunk WY factors of the pre-pass
   if (dt == DN_BF16 && T > 0) return kStatusBytes + dn::wy_workspace_bytes(B, H, T, C);
   return kStatusBytes;

@@ -28,7 +28,9 @@ std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  Resolved once per
-// device (the array's name is only a host-side stand-in for it in host code).
+// device (the array's name is only a host-side stand-in for it in host code) and
+// kept: a device reset after the first call would leave a stale address, which
+// the public header rules out.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -100,7 +100,8 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
 
   const int tid = threadIdx.x, lane = tid & 31;
   const int warp = (int)warp_uniform((uint32_t)tid >> 5);
-  const int chunk = blockIdx.x, bh = blockIdx.y;
+  // one-dimensional grid over (b, h, chunk), chunks of one head adjacent
+  const int chunk = (int)(blockIdx.x % (unsigned)nchunks), bh = (int)(blockIdx.x / (unsigned)nchunks);
   const int c0 = chunk * kC, n = min(kC, T - c0);
 
   // 1. K tile by TMA (rows past T read as zero), beta and the log-decay prefix g
@@ -407,7 +408,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   auto kern = tsolve_kernel<C, DK, GATED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)nchunks, (unsigned)(p.B * p.H));
+  const dim3 grid((unsigned)((size_t)nchunks * p.B * p.H));  // at most INT_MAX (checked by the caller)
   kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks,
                                                       p.status);
   return cudaGetLastError();

@@ -98,10 +98,12 @@ int deltanet_workspace_init(void *workspace, size_t ws_bytes, void *cuda_stream)
  *              overlap any input.
  *   S_out      (B,H,Dk,Dv) float32 final state, or NULL.  May equal S0
  *              (in-place carry); any other overlap is rejected.
- *   Dk, Dv     64 or 128.   C: 64 (bf16 and f32) or 128 (bf16).
+ *   Dk, Dv     64 or 128.   C: 64 (bf16 and f32) or 128 (bf16 only);
+ *              other values, and f32 with C = 128, give DN_ERR_UNSUPPORTED.
  *   T >= 0; T need not be a multiple of C (the ragged tail is handled
- *   exactly).  T == 0 copies S0 (or zeros) to S_out; q, k, v, beta, alpha
- *   and o may then be NULL.
+ *   exactly).  T == 0 copies S0 (or zeros) to S_out, for every C and dtype;
+ *   q, k, v, beta, alpha and o may then be NULL.  B * H * ceil(T / C) must
+ *   not exceed INT_MAX (DN_ERR_UNSUPPORTED otherwise).
  *   workspace  device buffer of deltanet_workspace_bytes(...) bytes.
  * bf16 runs on tcgen05 tensor cores with float32 state and accumulation;
  * f32 runs on CUDA cores in float32 throughout.
@@ -124,7 +126,11 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   q, k (B,H,Dk); v, o (B,H,Dv): element type dt, 16-byte aligned.
  *   beta (B,H) float32; alpha (B,H) float32 or NULL.
  *   S    (B,H,Dk,Dv) float32, updated in place; 16-byte aligned.
- *   Dk, Dv in {64, 128}.  No workspace.
+ *   Dk, Dv in {64, 128}.
+ * Unlike the chunked calls this one takes no workspace: each CTA reads one
+ * state, keeps it in registers between the two reductions and the write, and
+ * hands nothing to a later kernel, so there is no scratch to place and no
+ * second kernel whose bounded wait could need a status word.
  */
 int deltanet_decode_step(const void *q, const void *k, const void *v,
                          const float *beta, const float *alpha, float *S, void *o,
@@ -143,7 +149,10 @@ int deltanet_decode_step(const void *q, const void *k, const void *v,
  * (Q'z + tril(Q'K'^T) 1), S += K'^T V, z += K'^T 1.
  *   q, k raw (feature map applied inside); v unmapped.
  *   S0, z0 nullable (zero); S_out, z_out nullable.  S_out may equal S0 and
- *   z_out may equal z0.  Other arguments as deltanet_chunk_fwd (no beta, alpha).
+ *   z_out may equal z0.  C must be 64 (bf16 and f32); C = 128 gives
+ *   DN_ERR_UNSUPPORTED before anything is launched.  T == 0 copies S0 and z0
+ *   (or zeros) to S_out and z_out.  Other arguments as deltanet_chunk_fwd (no
+ *   beta, alpha).
  */
 int linear_attn_fwd(const void *q, const void *k, const void *v,
                     const float *S0, const float *z0,
@@ -188,7 +197,9 @@ int deltanet_selftest_wait_timeout(void *workspace, size_t ws_bytes, long long w
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with the caller's current device, which must be
  *     the device of the pointers and the stream); make that first call before
- *     any stream capture.
+ *     any stream capture.  The address is kept for the life of the process: a
+ *     process that resets the device (cudaDeviceReset) after that first call
+ *     must not call this entry point on that device again.
  *   - Each call clears the status word with an asynchronous memset on
  *     `cuda_stream`, then launches the kernel there.  A call rejected by
  *     validation may still have cleared that private word; it touches none of

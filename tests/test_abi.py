@@ -70,7 +70,11 @@ def test_workspace_bytes(L):
         nch = -(-T // C)
         want = 256 + 4 * 16 * nch * (2 * C * C * 2 + C * 4)
         assert L.deltanet_workspace_bytes(4, 16, T, 128, 128, C, 1) == want
-    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 128, 0) == 256  # f32: status only
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 64, 0) == 256  # f32: status only
+    assert L.deltanet_workspace_bytes(4, 16, 4096, 128, 128, 128, 0) == 0  # C = 128 is bf16 only
+    # one pre-pass CTA per (b, h, chunk) on a one-dimensional grid: at most INT_MAX of them
+    assert L.deltanet_workspace_bytes(1, 65536, 64 * 32768, 64, 64, 64, 1) == 0
+    assert L.deltanet_workspace_bytes(1, 65536, 64 * 32767, 64, 64, 64, 1) > 0
 
 
 # Fake, never dereferenced device addresses: every call below must be rejected
@@ -105,6 +109,17 @@ def test_chunk_rejects_bad_arguments(L):
     assert _chunk(L, q=A + 8) == E.DN_ERR_ALIGNMENT
     assert _chunk(L, o=A + 256 * MB + 2) == E.DN_ERR_ALIGNMENT
     assert _chunk(L, S0=A + 500 * MB + 4) == E.DN_ERR_ALIGNMENT
+    assert _chunk(L, C=128, dt=0) == E.DN_ERR_UNSUPPORTED  # C = 128 is built for bf16 only
+    assert _chunk(L, C=128, dt=0, T=0) == E.DN_ERR_UNSUPPORTED
+
+
+def test_chunk_rejects_grids_past_int_max(L):
+    """B * H * ceil(T / C) pre-pass CTAs must fit one grid dimension (INT_MAX):
+    one chunk past it is rejected before launch, not at launch."""
+    E = _lib
+    big = 1 << 40
+    assert _chunk(L, B=1, H=65536, T=64 * 32768, q=big, k=2 * big, v=3 * big, beta=4 * big,
+                  o=5 * big, S_out=None, ws=6 * big, ws_bytes=1 << 62) == E.DN_ERR_UNSUPPORTED
 
 
 def test_chunk_rejects_overlaps(L):
@@ -193,6 +208,7 @@ def test_linear_rejects_bad_arguments(L):
     assert lin(v=None) == E.DN_ERR_INVALID_ARG
     assert lin(Dk=80) == E.DN_ERR_UNSUPPORTED
     assert lin(C=96) == E.DN_ERR_UNSUPPORTED
+    assert lin(C=128) == E.DN_ERR_UNSUPPORTED  # linear attention is built for C = 64 only
     assert lin(z0=A + 300 * MB, z_out=A + 300 * MB + 4) == E.DN_ERR_ALIGNMENT
     assert lin(z0=A + 300 * MB, z_out=A + 300 * MB + 16) == E.DN_ERR_INVALID_ARG
 

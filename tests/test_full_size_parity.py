@@ -3,15 +3,17 @@ benchmark times (caller-sized workspace, preallocated outputs, one call over
 the whole batch).
 
 The CUDA path runs on every head of the workload; the float64 oracle then
-recomputes a few sampled heads in full (whole sequences, from the identical
-stored inputs) and the sampled outputs and final states are compared with
-the bf16 gate, rel-L2 <= 2e-2 per head.  Sizes:
+recomputes EVERY head (whole sequences, from the identical stored inputs, in
+batches of heads to bound host memory) and each head's outputs and final
+state are compared with the bf16 gate, rel-L2 <= 2e-2 per (b, h).  The largest
+per-head rel-L2 of each workload is printed as a diagnostic.  Sizes:
   prefill         B4 H16 T4096 D128 bf16 C64
   prefill-linear  the same shape, ELU+1 linear attention
-  long            B1 H32 T65536 D128 bf16 C64
+  long            B1 H32 T65536 D128 bf16, C64 and C128
   forget          B8 H16 T8192 D128 bf16 gated C64
   decode          256 sequences x 32 heads, D128, fp32 states from a 512-token
-                  prefill, then 1024 single-token steps with fresh inputs
+                  prefill, then 1024 single-token steps with fresh inputs:
+                  every state's final S and every step's output
 """
 import numpy as np
 import pytest
@@ -40,21 +42,30 @@ def dn():
     return m
 
 
-def _sample_heads(B, H):
-    """First, last and two interior (b, h) pairs."""
-    cand = [(0, 0), (B - 1, H - 1), (B // 2, H // 3), ((B - 1) // 3, (2 * H) // 3)]
-    out = []
-    for bh in cand:
-        if bh not in out:
-            out.append(bh)
-    return out
+def _per_head(x, ref):
+    """rel-L2 of each (b, h) slice: x, ref of shape (n, ...) -> (n,)"""
+    x = np.asarray(x, np.float64).reshape(len(x), -1)
+    ref = np.asarray(ref, np.float64).reshape(len(ref), -1)
+    return np.linalg.norm(x - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
 
 
-def _heads(t, heads):
-    """(B, H, ...) device tensor -> (1, n, ...) CPU tensor of the sampled heads."""
-    if t is None:
-        return None
-    return torch.stack([t[b, h] for b, h in heads]).unsqueeze(0).cpu()
+def _flat(t):
+    """(B, H, ...) tensor -> (B*H, ...) CPU tensor"""
+    return None if t is None else t.reshape((-1,) + tuple(t.shape[2:])).cpu()
+
+
+def _batches(n, per):
+    for a in range(0, n, per):
+        yield slice(a, min(n, a + per))
+
+
+def _report(capsys, name, errs):
+    worst = {k: (float(v.max()), int(v.argmax())) for k, v in errs.items()}
+    with capsys.disabled():
+        print(f"\nparity {name}: max per-(b,h) rel-L2 " +
+              ", ".join(f"{k}={e:.3e} (head {i})" for k, (e, i) in worst.items()))
+    for k, (e, i) in worst.items():
+        assert e <= TOL, f"{name}: {k} of flat head {i} has rel-L2 {e:.3e} > {TOL}"
 
 
 def _run_chunk_like_bench(dn, w, x):
@@ -71,22 +82,25 @@ def _run_chunk_like_bench(dn, w, x):
 
 
 @pytest.mark.parametrize("w", [gen.PREFILL, gen.FORGET, gen.LONG64, gen.LONG128], ids=lambda w: w.name)
-def test_full_size_chunk_forward_sampled_heads(dn, oracle_mod, w):
+def test_full_size_chunk_forward_all_heads(dn, oracle_mod, capsys, w):
     dev = torch.device("cuda")
     x = gen.make_workload(w, seed=11, device=dev)
     o, S = _run_chunk_like_bench(dn, w, x)
-    heads = _sample_heads(w.B, w.H)
-    sx = {k: _heads(v, heads) for k, v in x.items()}
-    o_ref, S_ref = oracle_mod.deltanet(sx["q"], sx["k"], sx["v"], sx["beta"], sx["alpha"])
-    o_s = _heads(o, heads).float().numpy()
-    S_s = _heads(S, heads).numpy()
-    assert np.isfinite(o.float().sum().item()) and np.isfinite(S.sum().item())
-    for i, bh in enumerate(heads):
-        eo, es = rel_l2(o_s[0, i], o_ref[0, i]), rel_l2(S_s[0, i], S_ref[0, i])
-        assert eo <= TOL and es <= TOL, f"{w.name} head {bh}: rel-L2 o={eo:.3e} S={es:.3e}"
+    fx = {k: _flat(v) for k, v in x.items()}
+    o_c, S_c = _flat(o).float(), _flat(S)
+    del x, o, S
+    n = w.B * w.H
+    eo, es = np.zeros(n), np.zeros(n)
+    per = max(1, (1 << 28) // (w.T * w.Dv * 8))  # oracle outputs of about 256 MB per batch
+    for sl in _batches(n, per):
+        sub = {k: (None if v is None else v[sl].unsqueeze(0)) for k, v in fx.items()}
+        o_ref, S_ref = oracle_mod.deltanet(sub["q"], sub["k"], sub["v"], sub["beta"], sub["alpha"])
+        eo[sl] = _per_head(o_c[sl].numpy(), o_ref[0])
+        es[sl] = _per_head(S_c[sl].numpy(), S_ref[0])
+    _report(capsys, w.name, {"o": eo, "S": es})
 
 
-def test_full_size_linear_attention_sampled_heads(dn, oracle_mod):
+def test_full_size_linear_attention_all_heads(dn, oracle_mod, capsys):
     w = gen.PREFILL_LINEAR
     dev = torch.device("cuda")
     x = gen.make_workload(w, seed=12, device=dev)
@@ -95,17 +109,15 @@ def test_full_size_linear_attention_sampled_heads(dn, oracle_mod):
     z = torch.empty(w.B, w.H, w.Dk, device=dev)
     dn.linear_attn_fwd(x["q"], x["k"], x["v"], C=w.C, o=o, S_out=S, z_out=z)
     torch.cuda.synchronize()
-    heads = _sample_heads(w.B, w.H)
-    sx = {k: _heads(v, heads) for k, v in x.items()}
-    o_ref, S_ref, z_ref = oracle_mod.linear_attn(sx["q"], sx["k"], sx["v"])
-    o_s, S_s, z_s = (_heads(t, heads).float().numpy() for t in (o, S, z))
-    for i, bh in enumerate(heads):
-        errs = [rel_l2(o_s[0, i], o_ref[0, i]), rel_l2(S_s[0, i], S_ref[0, i]),
-                rel_l2(z_s[0, i], z_ref[0, i])]
-        assert max(errs) <= TOL, f"head {bh}: rel-L2 o, S, z = {errs}"
+    o_ref, S_ref, z_ref = oracle_mod.linear_attn(x["q"].cpu(), x["k"].cpu(), x["v"].cpu())
+    n = w.B * w.H
+    errs = {"o": _per_head(_flat(o).float().numpy(), o_ref.reshape((n,) + o_ref.shape[2:])),
+            "S": _per_head(_flat(S).numpy(), S_ref.reshape((n,) + S_ref.shape[2:])),
+            "z": _per_head(_flat(z).numpy(), z_ref.reshape(n, -1))}
+    _report(capsys, w.name, errs)
 
 
-def test_full_size_decode_sampled_states(dn, oracle_mod):
+def test_full_size_decode_all_states(dn, oracle_mod, capsys):
     B, H, D = gen.DECODE_SEQS, gen.DECODE_HEADS, 128
     n_pre, n_steps = gen.DECODE_PREFILL, gen.DECODE_STEPS
     dev = torch.device("cuda")
@@ -114,22 +126,22 @@ def test_full_size_decode_sampled_states(dn, oracle_mod):
     steps = gen.make_inputs(B, H, n_steps, D, D, torch.bfloat16, seed=5, device=dev)
     qs, ks, vs = (steps[n].permute(2, 0, 1, 3).contiguous() for n in ("q", "k", "v"))
     bs = steps["beta"].permute(2, 0, 1).contiguous()
-    heads = _sample_heads(B, H)
-    bi = torch.tensor([b for b, _ in heads], device=dev)
-    hi = torch.tensor([h for _, h in heads], device=dev)
-    o = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
-    o_hist = torch.empty(n_steps, len(heads), D, dtype=torch.bfloat16, device=dev)
+    o_hist = torch.empty(n_steps, B, H, D, dtype=torch.bfloat16, device=dev)
     for t in range(n_steps):
-        dn.deltanet_decode_step(qs[t], ks[t], vs[t], bs[t], S, o=o)
-        o_hist[t] = o[bi, hi]
+        dn.deltanet_decode_step(qs[t], ks[t], vs[t], bs[t], S, o=o_hist[t])
     torch.cuda.synchronize()
-    # the oracle runs the plain recurrence over prefill + decode tokens
-    sx = {n: torch.cat([_heads(pre[n], heads), _heads(steps[n], heads)], dim=2)
-          for n in ("q", "k", "v", "beta")}
-    o_ref, S_ref = oracle_mod.deltanet(sx["q"], sx["k"], sx["v"], sx["beta"])
-    o_dec = o_hist.permute(1, 0, 2).float().cpu().numpy()
-    S_s = _heads(S, heads).numpy()
-    for i, bh in enumerate(heads):
-        eo = rel_l2(o_dec[i], o_ref[0, i, n_pre:])
-        es = rel_l2(S_s[0, i], S_ref[0, i])
-        assert eo <= TOL and es <= TOL, f"state {bh}: rel-L2 o={eo:.3e} S={es:.3e}"
+    del qs, ks, vs, bs
+    # the oracle runs the plain recurrence over prefill + decode tokens, per batch of states
+    o_dec = o_hist.permute(1, 2, 0, 3).reshape(B * H, n_steps, D).cpu()
+    S_c = _flat(S)
+    fp = {n: _flat(pre[n]) for n in ("q", "k", "v", "beta")}
+    fs = {n: _flat(steps[n]) for n in ("q", "k", "v", "beta")}
+    del pre, steps, o_hist, S
+    n = B * H
+    eo, es = np.zeros(n), np.zeros(n)
+    for sl in _batches(n, 256):
+        sx = {m: torch.cat([fp[m][sl], fs[m][sl]], dim=1).unsqueeze(0) for m in fp}
+        o_ref, S_ref = oracle_mod.deltanet(sx["q"], sx["k"], sx["v"], sx["beta"])
+        eo[sl] = _per_head(o_dec[sl].float().numpy(), o_ref[0, :, n_pre:])
+        es[sl] = _per_head(S_c[sl].numpy(), S_ref[0])
+    _report(capsys, "decode 256x32 D128, 1024 steps", {"o": eo, "S": es})

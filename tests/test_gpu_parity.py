@@ -174,6 +174,57 @@ def test_empty_sequence_copies_state(dn):
     assert torch.equal(S, S0)
 
 
+@pytest.mark.parametrize("dtype,C", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("with_S0", [True, False])
+def test_empty_sequence_every_chunk_size(dn, dtype, C, with_S0):
+    """T = 0 copies S0 (or zeros) to S_out for every built chunk size and dtype,
+    on the device call and on the host-buffer call."""
+    dev = torch.device("cuda")
+    q = torch.zeros(2, 3, 0, 128, dtype=dtype, device=dev)
+    S0 = torch.randn(2, 3, 128, 128, device=dev) if with_S0 else None
+    S_out = torch.full((2, 3, 128, 128), float("nan"), device=dev)
+    o, S = dn.deltanet_chunk_fwd(q, q, q, torch.zeros(2, 3, 0, device=dev), None, S0, C=C,
+                                 S_out=S_out)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 3, 0, 128)
+    assert torch.equal(S, S0 if with_S0 else torch.zeros_like(S))
+    qh = torch.zeros(2, 3, 0, 128, dtype=dtype)
+    oh, Sh = dn.deltanet_chunk_fwd_host(qh, qh, qh, torch.zeros(2, 3, 0), None,
+                                        None if S0 is None else S0.cpu(), C=C)
+    torch.cuda.synchronize()
+    assert torch.equal(Sh, S.cpu())
+
+
+def test_linear_attn_empty_sequence_copies_state(dn):
+    dev = torch.device("cuda")
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.bfloat16, device=dev)
+    S0 = torch.rand(1, 2, 64, 64, device=dev)
+    z0 = torch.rand(1, 2, 64, device=dev) + 1
+    _, S, z = dn.linear_attn_fwd(q, q, q, S0, z0)
+    _, S2, z2 = dn.linear_attn_fwd(q, q, q)
+    torch.cuda.synchronize()
+    assert torch.equal(S, S0) and torch.equal(z, z0)
+    assert not S2.any() and not z2.any()
+
+
+def test_more_heads_than_one_grid_row(dn, oracle_mod):
+    """B * H = 70,000 sequences (past the 65,535 limit of a grid's second
+    dimension), three tokens each: every head is computed; sampled heads match
+    the oracle and all heads are finite."""
+    dev = torch.device("cuda")
+    x = gen.make_inputs(1, 70000, 3, 64, 64, torch.bfloat16, gated=True, seed=17)
+    g = _to(x, dev)
+    o, S = dn.deltanet_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["alpha"])
+    torch.cuda.synchronize()
+    assert dn.deltanet_get_device_status() == 0
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+    o_ref, S_ref = oracle_mod.deltanet(x["q"], x["k"], x["v"], x["beta"], x["alpha"])
+    assert rel_l2(o.float().cpu(), o_ref) <= TOL[torch.bfloat16]
+    assert rel_l2(S.cpu(), S_ref) <= TOL[torch.bfloat16]
+    for h in (0, 65535, 65536, 69999):
+        assert rel_l2(S[0, h].cpu(), S_ref[0, h]) <= TOL[torch.bfloat16]
+
+
 def test_deterministic(dn):
     x = _to(gen.make_inputs(2, 4, 500, 128, 128, torch.bfloat16, gated=True, seed=11), "cuda")
     o1, S1 = dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"])

@@ -234,6 +234,63 @@ def test_linear_attn_matmul_closed_form(oracle_mod):
     np.testing.assert_allclose(z, Kp.sum(-2).numpy(), rtol=1e-11)
 
 
+def _elu1(x):
+    """ELU(x) + 1 in float64 (x + 1 above zero, e^x at or below)."""
+    x = np.asarray(x, np.float64)
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def test_delta_rule_without_read_is_elu1_linear_attention(oracle_mod):
+    """The delta update with its read term dropped and beta = 1 is the additive
+    update S += k^T v ("GPT-2 から Kimi K3 まで", section "DeltaNet (Fast weight
+    programmers)" against section "Linear attention").  With the ELU+1 maps on
+    q and k and a ones column appended to V, the additive state's last column
+    is the normaliser z and q'S's last entry is q'.z, so the ratio of the other
+    columns to it is ELU+1 linear attention.
+
+    Two independent routes to that reduction, both against oracle.linear_attn:
+    (1) an additive numpy loop (the delta write with the read removed);
+    (2) the delta-rule oracle itself, with the read made to vanish: key t is
+        placed in its own block of a T*Dk-dimensional key space (so every key
+        is orthogonal to all earlier ones and k_t S_{t-1} = 0 exactly) and the
+        query repeats q'_t in every block (so q S_t still sums q'_t . k'_s over
+        s <= t)."""
+    rng = np.random.default_rng(31)
+    T, Dk, Dv = 7, 4, 3
+    q = _rand((1, 1, T, Dk), rng)
+    k = _rand((1, 1, T, Dk), rng)
+    v = _rand((1, 1, T, Dv), rng)
+    o_ref, S_ref, z_ref = oracle_mod.linear_attn(q, k, v)
+    qp, kp = _elu1(q[0, 0]), _elu1(k[0, 0])
+    va = np.concatenate([v[0, 0].astype(np.float64), np.ones((T, 1))], axis=1)
+
+    # (1) additive loop on the augmented values
+    S = np.zeros((Dk, Dv + 1))
+    o1 = np.zeros((T, Dv))
+    for t in range(T):
+        S = S + np.outer(kp[t], va[t])  # write; no read term, beta = 1
+        r = qp[t] @ S
+        o1[t] = r[:Dv] / r[Dv]
+    np.testing.assert_allclose(o1, o_ref[0, 0], rtol=1e-12)
+    np.testing.assert_allclose(S[:, :Dv], S_ref[0, 0], rtol=1e-12)
+    np.testing.assert_allclose(S[:, Dv], z_ref[0, 0], rtol=1e-12)
+
+    # (2) the delta-rule oracle with block-orthogonal keys (float32 inputs)
+    kb = np.zeros((1, 1, T, T * Dk), np.float32)
+    qb = np.zeros((1, 1, T, T * Dk), np.float32)
+    for t in range(T):
+        kb[0, 0, t, t * Dk:(t + 1) * Dk] = kp[t]
+        qb[0, 0, t] = np.tile(qp[t], T)
+    beta = np.ones((1, 1, T), np.float32)
+    o2, S2 = oracle_mod.deltanet(qb, kb, va.astype(np.float32).reshape(1, 1, T, Dv + 1), beta)
+    ratio = o2[0, 0, :, :Dv] / o2[0, 0, :, Dv:]
+    # the ELU+1 values were rounded to float32 once (relative 6e-8 per entry)
+    np.testing.assert_allclose(ratio, o_ref[0, 0], rtol=1e-6, atol=1e-6)
+    S_fold = S2[0, 0].reshape(T, Dk, Dv + 1).sum(axis=0)  # sum the key blocks back up
+    np.testing.assert_allclose(S_fold[:, :Dv], S_ref[0, 0], rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(S_fold[:, Dv], z_ref[0, 0], rtol=1e-6, atol=1e-6)
+
+
 def test_bf16_inputs_widen_exactly(oracle_mod):
     """bfloat16 inputs give the same result as their exact float32 values."""
     g = torch.Generator().manual_seed(11)
