@@ -4,7 +4,9 @@ TEST INFRASTRUCTURE ONLY: only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline / reference arm of ``bench.py`` may import this package.  The
 product library never loads it, and it never loads the product library.
 
-* ``deltanet``     - the per-token delta rule (optionally gated), ``oracle.c``.
+* ``deltanet``     - the per-token delta rule (optionally gated, per-dimension
+                     gated, or behind the layer's silu / L2 / sigmoid pre-step),
+                     ``oracle.c``.
 * ``linear_attn``  - ELU+1 causal linear attention, ``oracle.c``.
 * ``chunk_form``   - the chunkwise WY form in numpy (see ``chunk_form.py``).
 
@@ -50,6 +52,8 @@ def _load():
         lib.oracle_deltanet.restype = I
         lib.oracle_linear_attn.argtypes = [vp, vp, vp, I, dp, dp, dp, dp, dp, L, L, L, L, L, I]
         lib.oracle_linear_attn.restype = I
+        lib.oracle_deltanet_ex.argtypes = [vp, vp, vp, I, fp, fp, dp, dp, dp, L, L, L, L, L, I, I]
+        lib.oracle_deltanet_ex.restype = I
         _lib = lib
     return _lib
 
@@ -106,13 +110,23 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
-def deltanet(q, k, v, beta, alpha=None, S0=None, nthreads: int = 0):
+PRESTEP, ALPHA_PER_DIM = 1, 2
+
+
+def deltanet(q, k, v, beta, alpha=None, S0=None, nthreads: int = 0, prestep: bool = False):
     """Delta rule over (B,H,T,D) sequences; returns ``(o, S_out)`` in float64.
 
     Follows the direct per-token loop of "GPT-2 から Kimi K3 まで" (news.ainew.jp),
     section "DeltaNet (Parallelizing linear transformers with delta rule)", with
     the gate of the Gated DeltaNet paragraph of "How a Baseten Engineer Traced 7
     Years of Attention Mechanism Evolution" (decay first, then the delta write).
+
+    ``alpha`` of shape (B,H,T) is the scalar gate; of shape (B,H,T,Dk) it is the
+    per-dimension gate of the same page's KDA paragraph (row i of the state
+    decays by alpha_t[i]).  ``prestep``: q and k are raw projections and beta
+    holds logits; each token first takes the DeltaNet layer's maps of the
+    section "DeltaNet (Fast weight programmers)": q, k <- normalize(silu(.)),
+    beta <- sigmoid(beta).
     """
     qa, dt = _as_stored(q)
     ka, dtk = _as_stored(k)
@@ -124,12 +138,20 @@ def deltanet(q, k, v, beta, alpha=None, S0=None, nthreads: int = 0):
     if ka.shape != (B, H, T, Dk) or va.shape != (B, H, T, Dv):
         raise ValueError("shape mismatch")
     b = _f32(beta).reshape(B, H, T)
-    a = None if alpha is None else _f32(alpha).reshape(B, H, T)
+    flags = PRESTEP if prestep else 0
+    a = None
+    if alpha is not None:
+        a = _f32(alpha)
+        if a.size == B * H * T * Dk and a.ndim == 4:
+            flags |= ALPHA_PER_DIM
+            a = a.reshape(B, H, T, Dk)
+        else:
+            a = a.reshape(B, H, T)
     s0 = None if S0 is None else _f64(S0).reshape(B, H, Dk, Dv)
     o = np.zeros((B, H, T, Dv), np.float64)
     S = np.zeros((B, H, Dk, Dv), np.float64)
-    rc = _load().oracle_deltanet(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(b), _ptr(a), _ptr(s0),
-                                 _ptr(o), _ptr(S), B, H, T, Dk, Dv, nthreads)
+    rc = _load().oracle_deltanet_ex(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(b), _ptr(a), _ptr(s0),
+                                    _ptr(o), _ptr(S), B, H, T, Dk, Dv, flags, nthreads)
     if rc != 0:
         raise RuntimeError(f"oracle_deltanet failed ({rc})")
     return o, S

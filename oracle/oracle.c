@@ -38,6 +38,17 @@
 /* Input element types understood by the oracle. */
 enum { ORC_F32 = 0, ORC_BF16 = 1 };
 
+/* Options of the delta rule.
+ *   ORC_PRESTEP: q and k are the raw projections and beta holds logits; each
+ *     token first takes the DeltaNet layer's feature maps of [P3] "DeltaNet
+ *     (Fast weight programmers)": q <- normalize(silu(q)), k <- normalize(silu(k))
+ *     (L2 over the head dimension, divisor max(norm, 1e-12) as F.normalize),
+ *     beta <- sigmoid(beta).
+ *   ORC_ALPHA_PER_DIM: alpha is (B,H,T,Dk), one decay per key dimension: row i
+ *     of the state decays by alpha_t[i] ([P1], the KDA paragraph: scalar gating
+ *     replaced by per-dimension gating). */
+enum { ORC_PRESTEP = 1, ORC_ALPHA_PER_DIM = 2 };
+
 /* Widen one stored element to double.  A bfloat16 value is the upper 16 bits
  * of the float32 with the same value, so the widening is exact. */
 static double widen(const void *p, int dtype, size_t i)
@@ -50,6 +61,30 @@ static double widen(const void *p, int dtype, size_t i)
     return (double)f;
 }
 
+/* silu(x) = x * sigmoid(x) = x / (1 + e^-x) */
+static double silu(double x)
+{
+    return x / (1.0 + exp(-x));
+}
+
+/* Read one token's Dk-vector (q or k) into out[], applying the pre-step map
+ * normalize(silu(.)) when asked. */
+static void load_key(const void *p, int dtype, size_t at, long Dk, int prestep, double *out)
+{
+    for (long i = 0; i < Dk; ++i)
+        out[i] = prestep ? silu(widen(p, dtype, at + i)) : widen(p, dtype, at + i);
+    if (prestep) {
+        double ss = 0.0;
+        for (long i = 0; i < Dk; ++i)
+            ss += out[i] * out[i];
+        double nrm = sqrt(ss);
+        if (nrm < 1e-12)
+            nrm = 1e-12;
+        for (long i = 0; i < Dk; ++i)
+            out[i] /= nrm;
+    }
+}
+
 /* Problem description shared by the worker threads. */
 typedef struct {
     const void *q, *k, *v;
@@ -59,6 +94,7 @@ typedef struct {
     double *o, *S_out, *z_out;
     long B, H, T, Dk, Dv;
     int linear; /* 0: delta rule (optionally gated); 1: ELU+1 linear attention */
+    int flags;  /* delta rule only: ORC_PRESTEP, ORC_ALPHA_PER_DIM */
     long next;  /* next (b,h) pair to process */
     pthread_mutex_t lock;
 } job_t;
@@ -71,50 +107,58 @@ typedef struct {
  * write S += k_t^T u_t, then emit o_t = q_t S with the state after the write.
  * [P1] Gated DeltaNet: S_new = alpha * S_old + k^T delta, "decay first, then
  * precise write", so the read is taken from the decayed state alpha_t S.
- * alpha == NULL means alpha_t = 1 (plain DeltaNet).
+ * alpha == NULL means alpha_t = 1 (plain DeltaNet); with ORC_ALPHA_PER_DIM the
+ * decay of row i of S is alpha_t[i].  `kv` holds 2 Dk doubles (q_t, k_t).
  */
-static void delta_sequence(const job_t *J, long bh, double *S, double *r)
+static void delta_sequence(const job_t *J, long bh, double *S, double *r, double *kv)
 {
     const long T = J->T, Dk = J->Dk, Dv = J->Dv;
     const size_t qk0 = (size_t)bh * T * Dk, v0 = (size_t)bh * T * Dv, s0 = (size_t)bh * Dk * Dv;
+    const int prestep = (J->flags & ORC_PRESTEP) != 0, per_dim = (J->flags & ORC_ALPHA_PER_DIM) != 0;
+    double *qv = kv, *kk = kv + Dk;
 
     for (long i = 0; i < Dk * Dv; ++i)
         S[i] = J->S0 ? J->S0[s0 + i] : 0.0;
 
     for (long t = 0; t < T; ++t) {
-        const double beta = (double)J->beta[(size_t)bh * T + t];
-        const double alpha = J->alpha ? (double)J->alpha[(size_t)bh * T + t] : 1.0;
+        double beta = (double)J->beta[(size_t)bh * T + t];
+        if (prestep)
+            beta = 1.0 / (1.0 + exp(-beta));
         const size_t kt = qk0 + (size_t)t * Dk, vt = v0 + (size_t)t * Dv;
+        load_key(J->q, J->dtype, kt, Dk, prestep, qv);
+        load_key(J->k, J->dtype, kt, Dk, prestep, kk);
 
         /* decay first */
-        if (J->alpha)
+        if (J->alpha && per_dim) {
+            for (long i = 0; i < Dk; ++i) {
+                const double a = (double)J->alpha[kt + i];
+                for (long j = 0; j < Dv; ++j)
+                    S[i * Dv + j] *= a;
+            }
+        } else if (J->alpha) {
+            const double alpha = (double)J->alpha[(size_t)bh * T + t];
             for (long i = 0; i < Dk * Dv; ++i)
                 S[i] *= alpha;
+        }
         /* read the value currently stored under k_t: v_old = k_t S */
         for (long j = 0; j < Dv; ++j)
             r[j] = 0.0;
-        for (long i = 0; i < Dk; ++i) {
-            const double ki = widen(J->k, J->dtype, kt + i);
+        for (long i = 0; i < Dk; ++i)
             for (long j = 0; j < Dv; ++j)
-                r[j] += ki * S[i * Dv + j];
-        }
+                r[j] += kk[i] * S[i * Dv + j];
         /* the delta u_t = beta_t (v_t - v_old), written as an outer product */
         for (long j = 0; j < Dv; ++j)
             r[j] = beta * (widen(J->v, J->dtype, vt + j) - r[j]);
-        for (long i = 0; i < Dk; ++i) {
-            const double ki = widen(J->k, J->dtype, kt + i);
+        for (long i = 0; i < Dk; ++i)
             for (long j = 0; j < Dv; ++j)
-                S[i * Dv + j] += ki * r[j];
-        }
+                S[i * Dv + j] += kk[i] * r[j];
         /* output with the updated state: o_t = q_t S */
         double *o = J->o + v0 + (size_t)t * Dv;
         for (long j = 0; j < Dv; ++j)
             o[j] = 0.0;
-        for (long i = 0; i < Dk; ++i) {
-            const double qi = widen(J->q, J->dtype, kt + i);
+        for (long i = 0; i < Dk; ++i)
             for (long j = 0; j < Dv; ++j)
-                o[j] += qi * S[i * Dv + j];
-        }
+                o[j] += qv[i] * S[i * Dv + j];
     }
     if (J->S_out)
         memcpy(J->S_out + s0, S, sizeof(double) * (size_t)(Dk * Dv));
@@ -176,7 +220,7 @@ static void *worker(void *arg)
 {
     job_t *J = (job_t *)arg;
     double *S = (double *)malloc(sizeof(double) * (size_t)(J->Dk * J->Dv));
-    double *r = (double *)malloc(sizeof(double) * (size_t)(2 * J->Dk + J->Dv));
+    double *r = (double *)malloc(sizeof(double) * (size_t)(4 * J->Dk + J->Dv));
     if (!S || !r) {
         free(S);
         free(r);
@@ -191,7 +235,7 @@ static void *worker(void *arg)
         if (J->linear)
             linear_sequence(J, bh, S, r, r + J->Dk);
         else
-            delta_sequence(J, bh, S, r);
+            delta_sequence(J, bh, S, r, r + J->Dv);
     }
     free(S);
     free(r);
@@ -246,6 +290,27 @@ int oracle_deltanet(const void *q, const void *k, const void *v, int dtype,
     J.o = o; J.S_out = S_out;
     J.B = B; J.H = H; J.T = T; J.Dk = Dk; J.Dv = Dv;
     J.linear = 0;
+    return run(&J, nthreads);
+}
+
+/*
+ * The delta rule with options (ORC_PRESTEP, ORC_ALPHA_PER_DIM; see above).
+ * Shapes as oracle_deltanet, except alpha: (B,H,T,Dk) with ORC_ALPHA_PER_DIM;
+ * with ORC_PRESTEP, q and k are the raw projections and beta the logits.
+ */
+int oracle_deltanet_ex(const void *q, const void *k, const void *v, int dtype,
+                       const float *beta, const float *alpha, const double *S0,
+                       double *o, double *S_out,
+                       long B, long H, long T, long Dk, long Dv, int flags, int nthreads)
+{
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k; J.v = v; J.dtype = dtype;
+    J.beta = beta; J.alpha = alpha; J.S0 = S0;
+    J.o = o; J.S_out = S_out;
+    J.B = B; J.H = H; J.T = T; J.Dk = Dk; J.Dv = Dv;
+    J.linear = 0;
+    J.flags = flags;
     return run(&J, nthreads);
 }
 

@@ -341,3 +341,88 @@ def test_planted_mistakes_fail_pins(oracle_mod):
     assert wrong(False, False) == pytest.approx(ref)
     assert wrong(True, False) != pytest.approx(ref)
     assert wrong(False, True) != pytest.approx(ref)
+
+
+# -- per-dimension decay (KDA) -------------------------------------------------
+
+def test_golden_kda_per_dim(oracle_mod):
+    g = _golden("kda_per_dim_worked.json")
+    a = np.asarray(g["alpha"], np.float32).reshape(1, 1, 3, 2)
+    o, S = oracle_mod.deltanet(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]),
+                               np.asarray(g["beta"], np.float32).reshape(1, 1, -1), alpha=a)
+    np.testing.assert_allclose(o[0, 0], g["o"], atol=1e-6)
+    np.testing.assert_allclose(S[0, 0], g["S"], atol=1e-6)
+
+
+def test_kda_uniform_decay_is_scalar_gating(oracle_mod):
+    """alpha_t[i] = a_t for every key dimension reduces to the scalar gate."""
+    rng = np.random.default_rng(41)
+    B, H, T, Dk, Dv = 1, 2, 19, 6, 5
+    q, v = _rand((B, H, T, Dk), rng), _rand((B, H, T, Dv), rng)
+    k = _unit_rows(_rand((B, H, T, Dk), rng))
+    beta = rng.uniform(0.1, 0.9, (B, H, T)).astype(np.float32)
+    a = rng.uniform(0.3, 1.0, (B, H, T)).astype(np.float32)
+    o1, S1 = oracle_mod.deltanet(q, k, v, beta, alpha=a)
+    o2, S2 = oracle_mod.deltanet(q, k, v, beta, alpha=np.repeat(a[..., None], Dk, axis=-1))
+    np.testing.assert_allclose(o2, o1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S2, S1, rtol=1e-13, atol=1e-13)
+
+
+def test_kda_transition_is_decayed_householder(oracle_mod):
+    """Each token maps S to (I - beta k^T k) diag(alpha) S + beta k^T v (the
+    generalised Householder transition after the per-dimension decay), and a
+    zero decay on dimension i wipes row i before the write."""
+    rng = np.random.default_rng(42)
+    Dk, Dv, T = 5, 4, 6
+    q, v = _rand((1, 1, T, Dk), rng), _rand((1, 1, T, Dv), rng)
+    k = _unit_rows(_rand((1, 1, T, Dk), rng))
+    beta = rng.uniform(0.2, 1.0, (1, 1, T)).astype(np.float32)
+    a = rng.uniform(0.0, 1.0, (1, 1, T, Dk)).astype(np.float32)
+    a[0, 0, 2, 1] = 0.0
+    S0 = rng.standard_normal((1, 1, Dk, Dv))
+    o, S_T = oracle_mod.deltanet(q, k, v, beta, alpha=a, S0=S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        kt = k[0, 0, t].astype(np.float64)
+        P = np.eye(Dk) - beta[0, 0, t] * np.outer(kt, kt)
+        S = P @ np.diag(a[0, 0, t].astype(np.float64)) @ S + beta[0, 0, t] * np.outer(kt, v[0, 0, t])
+        np.testing.assert_allclose(o[0, 0, t], q[0, 0, t].astype(np.float64) @ S, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S_T[0, 0], S, rtol=1e-11, atol=1e-12)
+
+
+# -- the layer's pre-step (silu, L2 normalise, sigmoid) ------------------------------
+
+def test_prestep_is_the_layer_feature_maps(oracle_mod):
+    """With the pre-step, q and k pass through F.normalize(F.silu(.)) and beta
+    through sigmoid ("GPT-2 から Kimi K3 まで", section "DeltaNet (Fast weight
+    programmers)", the layer's forward) before the delta rule: equal to the plain
+    oracle on inputs mapped by torch's own silu / normalize / sigmoid (rounded to
+    float32 once), gated and not."""
+    rng = np.random.default_rng(43)
+    B, H, T, Dk, Dv = 2, 2, 23, 8, 6
+    q, k, v = _rand((B, H, T, Dk), rng), _rand((B, H, T, Dk), rng), _rand((B, H, T, Dv), rng)
+    logit = _rand((B, H, T), rng)
+    a = rng.uniform(0.5, 1.0, (B, H, T)).astype(np.float32)
+    fmap = lambda x: torch.nn.functional.normalize(torch.nn.functional.silu(torch.from_numpy(x).double()),
+                                                   dim=-1).float().numpy()
+    b = torch.sigmoid(torch.from_numpy(logit).double()).float().numpy()
+    for alpha in (None, a):
+        o1, S1 = oracle_mod.deltanet(q, k, v, logit, alpha=alpha, prestep=True)
+        o2, S2 = oracle_mod.deltanet(fmap(q), fmap(k), v, b, alpha=alpha)
+        np.testing.assert_allclose(o1, o2, rtol=2e-6, atol=2e-6)
+        np.testing.assert_allclose(S1, S2, rtol=2e-6, atol=2e-6)
+
+
+def test_prestep_zero_key_writes_nothing(oracle_mod):
+    """silu(0) = 0 and the normaliser's floor keep a zero raw key at zero: that
+    token neither reads nor writes (S unchanged, o = q S)."""
+    rng = np.random.default_rng(44)
+    Dk, Dv = 4, 3
+    q, v = _rand((1, 1, 1, Dk), rng), _rand((1, 1, 1, Dv), rng)
+    k = np.zeros((1, 1, 1, Dk), np.float32)
+    S0 = rng.standard_normal((1, 1, Dk, Dv))
+    o, S = oracle_mod.deltanet(q, k, v, np.zeros((1, 1, 1), np.float32), S0=S0, prestep=True)
+    np.testing.assert_allclose(S, S0, rtol=0, atol=0)
+    qn = torch.nn.functional.normalize(torch.nn.functional.silu(torch.from_numpy(q[0, 0, 0]).double()),
+                                       dim=-1).numpy()
+    np.testing.assert_allclose(o[0, 0, 0], qn @ S0[0, 0], rtol=1e-12)
