@@ -5,8 +5,8 @@ The functions below carry the names of the C entry points in
 memory and the current stream, and every step of the computation runs in the
 library's CUDA kernels.  There is no CPU fallback.
 
-    o, S = deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C=64)
-    o    = deltanet_decode_step(q, k, v, beta, S, alpha=None)   # S updated in place
+    o, S = deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C=64, prestep=False)
+    o    = deltanet_decode_step(q, k, v, beta, S, alpha=None, prestep=False)  # S in place
     o, S, z = linear_attn_fwd(q, k, v, S0=None, z0=None, C=64)
 """
 from __future__ import annotations
@@ -69,10 +69,20 @@ def _ws_bytes(B, H, T, Dk, Dv, C, dt):
     return n
 
 
+def _options(prestep, alpha, per_dim_rank):
+    opts = _lib.DN_OPT_PRESTEP if prestep else 0
+    if alpha is not None and alpha.dim() == per_dim_rank:
+        opts |= _lib.DN_OPT_GATE_PER_DIM
+    return opts
+
+
 def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, S_out=None,
-                       workspace=None):
+                       workspace=None, prestep: bool = False):
     """Chunkwise DeltaNet forward.  q, k: (B,H,T,Dk); v: (B,H,T,Dv) (bf16 or f32);
-    beta, alpha: (B,H,T) f32; S0: (B,H,Dk,Dv) f32.  Returns (o, S_out)."""
+    beta: (B,H,T) f32; alpha: (B,H,T) f32 (one decay per token) or (B,H,T,Dk)
+    (one per key dimension); S0: (B,H,Dk,Dv) f32.  ``prestep``: q, k are raw
+    projections and beta logits (silu + L2 normalise and sigmoid run inside).
+    Returns (o, S_out)."""
     _need(q, "q")
     dev, dtype = q.device, q.dtype
     if dtype not in _DT:
@@ -93,11 +103,19 @@ def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, 
     _need(o, "o", dtype, dev)
     _need(S_out, "S_out", torch.float32, dev)
     dt = _DT[dtype]
-    nb = _ws_bytes(B, H, T, Dk, Dv, C, dt)
+    opts = _options(prestep, alpha, 4)
+    nb = lib().deltanet_workspace_bytes_ex(B, H, T, Dk, Dv, C, dt, opts)
+    if nb == 0:
+        raise DeltaNetError("deltanet_workspace_bytes_ex", _lib.DN_ERR_UNSUPPORTED)
     ws = workspace if workspace is not None else workspace_for(dev, nb)
-    check("deltanet_chunk_fwd", lib().deltanet_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
-        B, H, T, Dk, Dv, C, dt, _ptr(ws), ws.numel(), _stream(dev)))
+    if opts == 0:
+        check("deltanet_chunk_fwd", lib().deltanet_chunk_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
+            B, H, T, Dk, Dv, C, dt, _ptr(ws), ws.numel(), _stream(dev)))
+    else:
+        check("deltanet_chunk_fwd_ex", lib().deltanet_chunk_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
+            B, H, T, Dk, Dv, C, dt, opts, _ptr(ws), ws.numel(), _stream(dev)))
     return o, S_out
 
 
@@ -188,9 +206,10 @@ def linear_attn_fwd(q, k, v, S0=None, z0=None, C: int = 64, o=None, S_out=None, 
     return o, S_out, z_out
 
 
-def deltanet_decode_step(q, k, v, beta, S, alpha=None, o=None):
-    """One decode step.  q, k: (B,H,Dk); v: (B,H,Dv); beta, alpha: (B,H) f32;
-    S: (B,H,Dk,Dv) f32, updated in place.  Returns o (B,H,Dv)."""
+def deltanet_decode_step(q, k, v, beta, S, alpha=None, o=None, prestep: bool = False):
+    """One decode step.  q, k: (B,H,Dk); v: (B,H,Dv); beta: (B,H) f32; alpha:
+    (B,H) f32 or (B,H,Dk) (one decay per key dimension); S: (B,H,Dk,Dv) f32,
+    updated in place.  ``prestep``: q, k raw and beta logits.  Returns o (B,H,Dv)."""
     _need(q, "q")
     dev, dtype = q.device, q.dtype
     if dtype not in _DT:
@@ -205,9 +224,15 @@ def deltanet_decode_step(q, k, v, beta, S, alpha=None, o=None):
     Dv = v.shape[-1]
     if o is None:
         o = torch.empty(B, H, Dv, dtype=dtype, device=dev)
-    check("deltanet_decode_step", lib().deltanet_decode_step(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S), _ptr(o),
-        B, H, Dk, Dv, _DT[dtype], _stream(dev)))
+    opts = _options(prestep, alpha, 3)
+    if opts == 0:
+        check("deltanet_decode_step", lib().deltanet_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S), _ptr(o),
+            B, H, Dk, Dv, _DT[dtype], _stream(dev)))
+    else:
+        check("deltanet_decode_step_ex", lib().deltanet_decode_step_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S), _ptr(o),
+            B, H, Dk, Dv, _DT[dtype], opts, _stream(dev)))
     return o
 
 

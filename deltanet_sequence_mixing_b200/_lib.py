@@ -20,15 +20,22 @@ DN_ERR_CUDA = -4
 DN_ERR_DEVICE_TIMEOUT = -5
 DN_ERR_WORKSPACE = -6
 DN_F32, DN_BF16 = 0, 1
+DN_OPT_PRESTEP, DN_OPT_GATE_PER_DIM = 1, 2
 
 # Every symbol include/deltanet.h declares, with (restype, argtypes).
-_vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
+_vp, _sz, _i, _ll, _u = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong,
+                         ctypes.c_uint)
 SIGNATURES = {
     "deltanet_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "deltanet_workspace_init": (_i, [_vp, _sz, _vp]),
     "deltanet_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "deltanet_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "deltanet_decode_step_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _u,
+                                     _vp]),
+    "deltanet_workspace_bytes_ex": (_sz, [_i, _i, _i, _i, _i, _i, _i, _u]),
+    "deltanet_chunk_fwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _i, _i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp]),
     "linear_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "deltanet_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

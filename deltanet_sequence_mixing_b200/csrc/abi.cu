@@ -13,6 +13,7 @@
 namespace {
 
 constexpr size_t kStatusBytes = 256;  // status word + padding (keeps 256-byte alignment)
+constexpr unsigned int kKnownOptions = DN_OPT_PRESTEP | DN_OPT_GATE_PER_DIM;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -42,8 +43,10 @@ int validate_problem(const dn::ChunkProblem& p) {
   if (p.bf16 != 0 && p.bf16 != 1) return DN_ERR_INVALID_ARG;
   if (!valid_dim(p.Dk) || !valid_dim(p.Dv)) return DN_ERR_UNSUPPORTED;
   if (p.C != 64 && p.C != 128) return DN_ERR_UNSUPPORTED;
-  // C = 128 is built for the bf16 delta rule only
-  if (p.C == 128 && (!p.bf16 || p.mode != dn::Mode::Delta)) return DN_ERR_UNSUPPORTED;
+  // C = 128 is built for the bf16 delta rule only, without the options
+  if (p.C == 128 && (!p.bf16 || p.mode != dn::Mode::Delta || p.prestep || p.alpha_per_dim))
+    return DN_ERR_UNSUPPORTED;
+  if (p.alpha_per_dim && !p.alpha && p.T > 0) return DN_ERR_INVALID_ARG;
   if ((long long)p.B * p.H > INT_MAX) return DN_ERR_UNSUPPORTED;
   // the pre-pass runs one CTA per (b, h, chunk), on a one-dimensional grid
   if ((long long)p.B * p.H * ((p.T + (long long)p.C - 1) / p.C) > INT_MAX) return DN_ERR_UNSUPPORTED;
@@ -64,7 +67,7 @@ int validate_overlaps(const dn::ChunkProblem& p, const void* ws, size_t ws_bytes
   const Range q = range_of(p.q, BH * T * p.Dk * es), k = range_of(p.k, BH * T * p.Dk * es);
   const Range v = range_of(p.v, BH * T * p.Dv * es), o = range_of(p.o, BH * T * p.Dv * es);
   const Range beta = range_of(p.beta, p.beta ? BH * T * 4 : 0);
-  const Range alpha = range_of(p.alpha, p.alpha ? BH * T * 4 : 0);
+  const Range alpha = range_of(p.alpha, p.alpha ? BH * T * 4 * (p.alpha_per_dim ? p.Dk : 1) : 0);
   const Range S0 = range_of(p.S0, p.S0 ? BH * p.Dk * p.Dv * 4 : 0);
   const Range So = range_of(p.S_out, p.S_out ? BH * p.Dk * p.Dv * 4 : 0);
   const Range z0 = range_of(p.z0, p.z0 ? BH * p.Dk * 4 : 0);
@@ -87,12 +90,13 @@ int validate_overlaps(const dn::ChunkProblem& p, const void* ws, size_t ws_bytes
 }
 
 // Full validation of a chunked call on device buffers.  Returns DN_OK or an error.
-int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws) {
+int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws,
+                     unsigned int options = 0) {
   int rc = validate_problem(p);
   if (rc != DN_OK) return rc;
   if (!ws) return DN_ERR_WORKSPACE;
-  if (ws_bytes < deltanet_workspace_bytes(p.B, p.H, p.T, p.Dk, p.Dv, p.C,
-                                          p.bf16 ? DN_BF16 : DN_F32))
+  if (ws_bytes < deltanet_workspace_bytes_ex(p.B, p.H, p.T, p.Dk, p.Dv, p.C,
+                                             p.bf16 ? DN_BF16 : DN_F32, options))
     return DN_ERR_WORKSPACE;
   if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.o))
     return DN_ERR_ALIGNMENT;
@@ -104,6 +108,13 @@ int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws)
 
 // Launch the kernels of a validated chunked problem; `status` is the device
 // status word, `wy` the start of the pre-pass factor region.
+// Problems the tcgen05 chunk kernels take: the plain and scalar-gated delta rule
+// on bf16 inputs, without the pre-step; the pre-step and the per-dimension gate
+// run on the CUDA-core kernel (C = 64).
+bool tensor_core_path(const dn::ChunkProblem& p) {
+  return !p.prestep && !p.alpha_per_dim && (dn::chunk_main_supported(p) || dn::chunk128_supported(p));
+}
+
 int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStream_t st) {
   if ((size_t)p.B * p.H == 0) return DN_OK;  // nothing to compute
   p.status = status;
@@ -118,7 +129,7 @@ int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStre
     if (e == cudaSuccess && p.mode == dn::Mode::Linear) e = carry(p.z_out, p.z0, BH * p.Dk * sizeof(float));
     return map_cuda(e);
   }
-  if (dn::chunk_main_supported(p) || dn::chunk128_supported(p)) {
+  if (tensor_core_path(p)) {
     const dn::WyWorkspace w = dn::wy_carve(wy, p.B, p.H, p.T, p.C);
     return map_cuda(p.C == 64 ? dn::launch_chunk_main(p, w, st) : dn::launch_chunk128(p, w, st));
   }
@@ -199,6 +210,15 @@ cudaError_t host_queues(int dev, HostQueues** out) {
 
 extern "C" {
 
+size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                                   unsigned int options) {
+  if (options & ~kKnownOptions) return 0;
+  if (options == 0) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);
+  // the options run on the CUDA-core kernel: C = 64, status word only
+  if (C != 64 || deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt) == 0) return 0;
+  return kStatusBytes;
+}
+
 size_t deltanet_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
   if (B < 0 || H < 0 || T < 0 || !valid_dim(Dk) || !valid_dim(Dv)) return 0;
   if ((C != 64 && C != 128) || (dt != DN_F32 && dt != DN_BF16)) return 0;
@@ -215,20 +235,31 @@ int deltanet_workspace_init(void* workspace, size_t ws_bytes, void* cuda_stream)
       cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(cuda_stream)));
 }
 
-int deltanet_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
-                       const float* alpha, const float* S0, void* o, float* S_out, int B, int H,
-                       int T, int Dk, int Dv, int C, dn_dtype dt, void* workspace,
-                       size_t ws_bytes, void* cuda_stream) {
+int deltanet_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+                          const float* alpha, const float* S0, void* o, float* S_out, int B, int H,
+                          int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options,
+                          void* workspace, size_t ws_bytes, void* cuda_stream) {
   if (dt != DN_F32 && dt != DN_BF16) return DN_ERR_UNSUPPORTED;
+  if (options & ~kKnownOptions) return DN_ERR_INVALID_ARG;
   dn::ChunkProblem p{};
   p.q = q; p.k = k; p.v = v; p.beta = beta; p.alpha = alpha; p.S0 = S0;
   p.o = o; p.S_out = S_out;
   p.B = B; p.H = H; p.T = T; p.Dk = Dk; p.Dv = Dv; p.C = C;
   p.bf16 = dt == DN_BF16;
   p.mode = dn::Mode::Delta;
-  const int rc = validate_chunked(p, ws_bytes, workspace);
+  p.prestep = (options & DN_OPT_PRESTEP) != 0;
+  p.alpha_per_dim = (options & DN_OPT_GATE_PER_DIM) != 0;
+  const int rc = validate_chunked(p, ws_bytes, workspace, options);
   if (rc != DN_OK) return rc;
   return run_chunked(p, workspace, cuda_stream);
+}
+
+int deltanet_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* alpha, const float* S0, void* o, float* S_out, int B, int H,
+                       int T, int Dk, int Dv, int C, dn_dtype dt, void* workspace,
+                       size_t ws_bytes, void* cuda_stream) {
+  return deltanet_chunk_fwd_ex(q, k, v, beta, alpha, S0, o, S_out, B, H, T, Dk, Dv, C, dt, 0u,
+                               workspace, ws_bytes, cuda_stream);
 }
 
 size_t deltanet_host_workspace_bytes(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt) {
@@ -346,7 +377,16 @@ int linear_attn_fwd(const void* q, const void* k, const void* v, const float* S0
 int deltanet_decode_step(const void* q, const void* k, const void* v, const float* beta,
                          const float* alpha, float* S, void* o, int B, int H, int Dk, int Dv,
                          dn_dtype dt, void* cuda_stream) {
+  return deltanet_decode_step_ex(q, k, v, beta, alpha, S, o, B, H, Dk, Dv, dt, 0u, cuda_stream);
+}
+
+int deltanet_decode_step_ex(const void* q, const void* k, const void* v, const float* beta,
+                            const float* alpha, float* S, void* o, int B, int H, int Dk, int Dv,
+                            dn_dtype dt, unsigned int options, void* cuda_stream) {
   if (dt != DN_F32 && dt != DN_BF16) return DN_ERR_UNSUPPORTED;
+  if (options & ~kKnownOptions) return DN_ERR_INVALID_ARG;
+  const bool per_dim = (options & DN_OPT_GATE_PER_DIM) != 0;
+  if (per_dim && !alpha) return DN_ERR_INVALID_ARG;
   if (B < 0 || H < 0) return DN_ERR_INVALID_ARG;
   if (!valid_dim(Dk) || !valid_dim(Dv)) return DN_ERR_UNSUPPORTED;
   if ((long long)B * H > INT_MAX) return DN_ERR_UNSUPPORTED;
@@ -357,12 +397,13 @@ int deltanet_decode_step(const void* q, const void* k, const void* v, const floa
   const Range rs = range_of(S, BH * Dk * Dv * 4), ro = range_of(o, BH * Dv * es);
   const Range ins[] = {range_of(q, BH * Dk * es), range_of(k, BH * Dk * es),
                        range_of(v, BH * Dv * es), range_of(beta, BH * 4),
-                       range_of(alpha, alpha ? BH * 4 : 0)};
+                       range_of(alpha, alpha ? BH * 4 * (per_dim ? Dk : 1) : 0)};
   for (const Range& r : ins)
     if (overlap(rs, r) || overlap(ro, r)) return DN_ERR_INVALID_ARG;
   if (overlap(rs, ro)) return DN_ERR_INVALID_ARG;
   if (BH == 0) return DN_OK;
-  dn::DecodeProblem p{q, k, v, beta, alpha, S, o, B, H, Dk, Dv, dt == DN_BF16};
+  dn::DecodeProblem p{q, k, v, beta, alpha, S, o, B, H, Dk, Dv, dt == DN_BF16,
+                      (options & DN_OPT_PRESTEP) != 0, per_dim};
   return map_cuda(dn::launch_decode(p, static_cast<cudaStream_t>(cuda_stream)));
 }
 

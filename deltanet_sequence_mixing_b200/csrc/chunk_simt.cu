@@ -48,21 +48,52 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, size_
 // ELU(x) + 1: x + 1 for x > 0, and e^x (= (e^x - 1) + 1) otherwise.
 __device__ __forceinline__ float elu_plus_one(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
-template <int DK, int DVS, int C, bool GATED>
+__device__ __forceinline__ float silu(float x) { return x / (1.f + __expf(-x)); }
+
+// GATE: 0 none, 1 one decay per token (Gamma table), 2 one decay per token and
+// key dimension (a table of the cumulative log decay G, C x DK).
+template <int DK, int DVS, int C, int GATE>
 struct SimtSmem {
   static constexpr int KP = DK + 1, VP = DVS + 1, CP = C + 1;
   static constexpr int kFloats = 2 * C * KP      // Q, K
                                  + 2 * C * VP    // V (then X), U
                                  + DK * VP       // S slice
                                  + 2 * C * CP    // T, A / P
-                                 + (GATED ? C * CP : 0)  // Gamma
+                                 + (GATE == 1 ? C * CP : 0)  // Gamma
+                                 + (GATE == 2 ? C * KP : 0)  // G
                                  + 3 * C + DK + C;       // beta, gamma, alpha, z, den
   static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
-template <typename TI, bool LINEAR, bool GATED, int DK, int DVS, int C>
+// Stage rows [0, C) of a (T, DK) key-shaped input at token c0 into X (row
+// stride KP); rows past n are zero.  PRE maps each row to normalize(silu(row)).
+template <typename TI, bool PRE, int DK, int KP, int C>
+__device__ void stage_keys(float* X, const TI* src, size_t base, int c0, int n, bool elu) {
+  for (int idx = threadIdx.x; idx < C * DK; idx += kThreads) {
+    const int r = idx / DK, i = idx % DK;
+    float x = 0.f;
+    if (r < n) {
+      x = load_in(src, base + (size_t)(c0 + r) * DK + i);
+      if (elu) x = elu_plus_one(x);
+      if (PRE) x = silu(x);
+    }
+    X[r * KP + i] = x;
+  }
+  if (PRE) {
+    __syncthreads();
+    for (int r = threadIdx.x; r < C; r += kThreads) {
+      float ss = 0.f;
+      for (int i = 0; i < DK; ++i) ss += X[r * KP + i] * X[r * KP + i];
+      const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+      for (int i = 0; i < DK; ++i) X[r * KP + i] *= inv;
+    }
+  }
+}
+
+template <typename TI, bool LINEAR, int GATE, bool PRE, int DK, int DVS, int C>
 __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem p) {
-  using L = SimtSmem<DK, DVS, C, GATED>;
+  constexpr bool GATED = GATE == 1;
+  using L = SimtSmem<DK, DVS, C, GATE>;
   constexpr int KP = L::KP, VP = L::VP, CP = L::CP;
   extern __shared__ float sm[];
   float* Qs = sm;
@@ -72,8 +103,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
   float* Ss = Us + C * VP;
   float* Ts = Ss + DK * VP;
   float* Ps = Ts + C * CP;
-  float* Gm = Ps + C * CP;  // only meaningful when GATED
-  float* bs = Gm + (GATED ? C * CP : 0);
+  float* Gm = Ps + C * CP;  // only meaningful when GATE == 1
+  float* Gd = Gm + (GATED ? C * CP : 0);  // only meaningful when GATE == 2
+  float* bs = Gd + (GATE == 2 ? C * KP : 0);
   float* gs = bs + C;
   float* as = gs + C;
   float* zs = as + C;
@@ -102,29 +134,28 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
     const int n = min(C, T - c0);
     __syncthreads();  // previous chunk finished with every buffer
     // ---- stage the chunk (rows >= n are zero; beta 0, alpha 1) ----
-    for (int idx = tid; idx < C * DK; idx += kThreads) {
-      const int r = idx / DK, i = idx % DK;
-      float qv = 0.f, kv = 0.f;
-      if (r < n) {
-        qv = load_in(q, qk_base + (size_t)(c0 + r) * DK + i);
-        kv = load_in(k, qk_base + (size_t)(c0 + r) * DK + i);
-        if (LINEAR) {
-          qv = elu_plus_one(qv);
-          kv = elu_plus_one(kv);
-        }
-      }
-      Qs[r * KP + i] = qv;
-      Ks[r * KP + i] = kv;
-    }
+    stage_keys<TI, PRE, DK, KP, C>(Qs, q, qk_base, c0, n, LINEAR);
+    stage_keys<TI, PRE, DK, KP, C>(Ks, k, qk_base, c0, n, LINEAR);
     for (int idx = tid; idx < C * DVS; idx += kThreads) {
       const int r = idx / DVS, j = idx % DVS;
       Vs[r * VP + j] = r < n ? load_in(v, v_base + (size_t)(c0 + r) * Dv + j0 + j) : 0.f;
     }
     if (!LINEAR)
       for (int r = tid; r < C; r += kThreads) {
-        bs[r] = r < n ? p.beta[(size_t)bh * T + c0 + r] : 0.f;
+        float b = r < n ? p.beta[(size_t)bh * T + c0 + r] : 0.f;
+        if (PRE && r < n) b = 1.f / (1.f + __expf(-b));
+        bs[r] = b;
         as[r] = (GATED && r < n) ? p.alpha[(size_t)bh * T + c0 + r] : 1.f;
       }
+    if (GATE == 2) {  // G[r][i] = sum_{j <= r} max(log alpha_j[i], -87) within the chunk
+      for (int i = tid; i < DK; i += kThreads) {
+        float g = 0.f;
+        for (int r = 0; r < C; ++r) {
+          if (r < n) g += fmaxf(__logf(p.alpha[(qk_base + (size_t)(c0 + r) * DK) + i]), -87.f);
+          Gd[r * KP + i] = g;
+        }
+      }
+    }
     __syncthreads();
 
     if (LINEAR) {
@@ -186,7 +217,12 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
       const int r = idx / C, s = idx % C;
       float acc = 0.f;
       if (s < r) {
-        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
+        if (GATE == 2) {
+          for (int i = 0; i < DK; ++i)
+            acc += Ks[r * KP + i] * Ks[s * KP + i] * __expf(Gd[r * KP + i] - Gd[s * KP + i]);
+        } else {
+          for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
+        }
         acc *= bs[r];
         if (GATED) acc *= Gm[r * CP + s];
       }
@@ -208,6 +244,69 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
         }
         Ts[i * CP + j] = t;
       }
+    }
+    if constexpr (GATE == 2) {
+      // Per-dimension decay (G[r][i] = cumulative log decay of key dimension i
+      // within the chunk, non-increasing in r).  Every exponential below has a
+      // non-positive argument, so nothing overflows:
+      //   P[r][s] = sum_i Q[r][i] K[s][i] e^(G[r][i] - G[s][i])      (s <= r)
+      //   X = V - (K * e^G) S,   U = T diag(beta) X
+      //   O = (Q * e^G) S + P U
+      //   S = diag(e^G[n-1]) S + (K * e^(G[n-1] - G))^T U
+      __syncthreads();  // T is complete; A in Ps may be overwritten
+      for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, s2 = idx % C;
+        float acc = 0.f;
+        if (s2 <= r)
+          for (int i = 0; i < DK; ++i)
+            acc += Qs[r * KP + i] * Ks[s2 * KP + i] * __expf(Gd[r * KP + i] - Gd[s2 * KP + i]);
+        Ps[r * CP + s2] = acc;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DK; idx += kThreads) {  // Q, K -> Q e^G, K e^G
+        const int r = idx / DK, i = idx % DK;
+        const float e = __expf(Gd[r * KP + i]);
+        Qs[r * KP + i] *= e;
+        Ks[r * KP + i] *= e;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        const int r = idx / DVS, j = idx % DVS;
+        float acc = 0.f;
+        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ss[i * VP + j];
+        Vs[r * VP + j] -= acc;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        const int r = idx / DVS, j = idx % DVS;
+        float acc = 0.f;
+        for (int s2 = 0; s2 <= r; ++s2) acc += Ts[r * CP + s2] * bs[s2] * Vs[s2 * VP + j];
+        Us[r * VP + j] = acc;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        const int r = idx / DVS, j = idx % DVS;
+        if (r >= n) continue;
+        float acc = 0.f;
+        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ss[i * VP + j];
+        for (int s2 = 0; s2 <= r; ++s2) acc += Ps[r * CP + s2] * Us[s2 * VP + j];
+        store_out(o, v_base + (size_t)(c0 + r) * Dv + j0 + j, acc);
+      }
+      // K again, weighted for the state update: K[s][i] e^(G[n-1][i] - G[s][i])
+      stage_keys<TI, PRE, DK, KP, C>(Ks, k, qk_base, c0, n, false);
+      __syncthreads();
+      for (int idx = tid; idx < C * DK; idx += kThreads) {
+        const int r = idx / DK, i = idx % DK;
+        Ks[r * KP + i] *= __expf(Gd[(n - 1) * KP + i] - Gd[r * KP + i]);
+      }
+      __syncthreads();
+      for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+        const int i = idx / DVS, j = idx % DVS;
+        float acc = 0.f;
+        for (int s2 = 0; s2 < n; ++s2) acc += Ks[s2 * KP + i] * Us[s2 * VP + j];
+        Ss[i * VP + j] = __expf(Gd[(n - 1) * KP + i]) * Ss[i * VP + j] + acc;
+      }
+      continue;
     }
     // ---- X = V - diag(gamma) K S (in place in Vs) ----
     for (int idx = tid; idx < C * DVS; idx += kThreads) {
@@ -270,11 +369,11 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
     for (int i = tid; i < DK; i += kThreads) p.z_out[(size_t)bh * DK + i] = zs[i];
 }
 
-template <typename TI, bool LINEAR, bool GATED, int DK>
+template <typename TI, bool LINEAR, int GATE, bool PRE, int DK>
 cudaError_t launch_one(const ChunkProblem& p, cudaStream_t st) {
   constexpr int DVS = 64, C = 64;
-  using L = SimtSmem<DK, DVS, C, GATED>;
-  auto kern = chunk_simt_kernel<TI, LINEAR, GATED, DK, DVS, C>;
+  using L = SimtSmem<DK, DVS, C, GATE>;
+  auto kern = chunk_simt_kernel<TI, LINEAR, GATE, PRE, DK, DVS, C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L::kBytes);
   if (e != cudaSuccess) return e;
@@ -283,16 +382,22 @@ cudaError_t launch_one(const ChunkProblem& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <typename TI, int DK>
+cudaError_t dispatch_delta(const ChunkProblem& p, cudaStream_t st) {
+  const int gate = p.alpha == nullptr ? 0 : (p.alpha_per_dim ? 2 : 1);
+  if (p.prestep) {
+    if (gate == 0) return launch_one<TI, false, 0, true, DK>(p, st);
+    return gate == 1 ? launch_one<TI, false, 1, true, DK>(p, st) : launch_one<TI, false, 2, true, DK>(p, st);
+  }
+  if (gate == 0) return launch_one<TI, false, 0, false, DK>(p, st);
+  return gate == 1 ? launch_one<TI, false, 1, false, DK>(p, st) : launch_one<TI, false, 2, false, DK>(p, st);
+}
+
 template <typename TI>
 cudaError_t dispatch_mode(const ChunkProblem& p, cudaStream_t st) {
   const bool lin = p.mode == Mode::Linear;
-  const bool gated = !lin && p.alpha != nullptr;
-  if (p.Dk == 64) {
-    if (lin) return launch_one<TI, true, false, 64>(p, st);
-    return gated ? launch_one<TI, false, true, 64>(p, st) : launch_one<TI, false, false, 64>(p, st);
-  }
-  if (lin) return launch_one<TI, true, false, 128>(p, st);
-  return gated ? launch_one<TI, false, true, 128>(p, st) : launch_one<TI, false, false, 128>(p, st);
+  if (p.Dk == 64) return lin ? launch_one<TI, true, 0, false, 64>(p, st) : dispatch_delta<TI, 64>(p, st);
+  return lin ? launch_one<TI, true, 0, false, 128>(p, st) : dispatch_delta<TI, 128>(p, st);
 }
 
 }  // namespace

@@ -8,6 +8,8 @@
 //     u = beta (v - alpha r)
 //     o = alpha p + (q . k) u      (= q (alpha S + k^T u), the state after the write)
 //     S = alpha S + k^T u
+// With a per-dimension decay the rows of S are scaled first (S_i <- alpha_i S_i)
+// and the same formulas run with alpha = 1 on the decayed rows.
 //
 // The step is bound by HBM: each Dk x Dv float32 state is read once and written
 // once.  One CTA per head; warp w streams rows w, w + 8, ... with one 16-byte
@@ -61,12 +63,20 @@ struct Vec<2> {
   __device__ static void unpack(const T& v, float (&x)[2]) { x[0] = v.x; x[1] = v.y; }
 };
 
-template <typename TI, int DK, int DV, bool GATED>
+// Options of the step (template parameters, one instantiation each):
+//   PRE   q and k are raw projections and beta holds logits: q, k <- normalize(silu(.))
+//         (L2 over Dk, divisor max(norm, 1e-12)), beta <- sigmoid(beta): the DeltaNet
+//         layer's feature maps ("GPT-2 から Kimi K3 まで", section "DeltaNet (Fast weight
+//         programmers)"), applied here so the maps cost no extra pass over q and k.
+//   GATE  0: none; 1: one decay alpha per head; 2: one decay per key dimension,
+//         alpha (B,H,Dk), row i of S scaled by alpha[i] (the per-dimension gating of
+//         the KDA paragraph of "How a Baseten Engineer Traced 7 Years ...").
+template <typename TI, int DK, int DV, int GATE, bool PRE>
 __global__ void __launch_bounds__(kWarps * 32, 2) decode_kernel(const DecodeProblem p) {
   constexpr int CPL = DV / 32;     // state columns per lane
   constexpr int RPW = DK / kWarps; // state rows per warp
   using V = Vec<CPL>;
-  __shared__ float ks[DK], qs[DK];
+  __shared__ float ks[DK], qs[DK], as[GATE == 2 ? DK : 1];
   __shared__ float red[2][kWarps][DV];
   __shared__ float qk_s;
 
@@ -85,13 +95,31 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_kernel(const DecodeProb
   for (int i = threadIdx.x; i < DK; i += kWarps * 32) {
     qs[i] = ld1(q, i);
     ks[i] = ld1(k, i);
+    if (GATE == 2) as[i] = p.alpha[bh * DK + i];
   }
-  const float beta = p.beta[bh];
-  const float alpha = GATED ? p.alpha[bh] : 1.f;
+  float beta = p.beta[bh];
+  if (PRE) beta = 1.f / (1.f + __expf(-beta));
+  const float alpha = GATE == 1 ? p.alpha[bh] : 1.f;
   float vj[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) vj[c] = ld1(static_cast<const TI*>(p.v), bh * DV + c0 + c);
   __syncthreads();
+  if (PRE && w < 2) {  // warp 0 maps q, warp 1 maps k: silu, then L2 normalise
+    float* x = w == 0 ? qs : ks;
+    float y[DK / 32], ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < DK / 32; ++e) {
+      const float t = x[lane + 32 * e];
+      y[e] = t / (1.f + __expf(-t));
+      ss = fmaf(y[e], y[e], ss);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+    for (int e = 0; e < DK / 32; ++e) x[lane + 32 * e] = y[e] * inv;
+  }
+  if (PRE) __syncthreads();
 
   float s[RPW][CPL];
   float rk[CPL], rq[CPL];
@@ -101,6 +129,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_kernel(const DecodeProb
   for (int rr = 0; rr < RPW; ++rr) {
     V::unpack(raw[rr], s[rr]);
     const int i = rr * kWarps + w;
+    if (GATE == 2) {  // decay first: row i of the state is alpha[i] S_i
+      const float a = as[i];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) s[rr][c] *= a;
+    }
     const float ki = ks[i], qi = qs[i];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
@@ -144,14 +177,20 @@ __global__ void __launch_bounds__(kWarps * 32, 2) decode_kernel(const DecodeProb
   }
 }
 
+template <typename TI, int DK, int DV, int GATE>
+cudaError_t launch_g(const DecodeProblem& p, cudaStream_t st) {
+  const unsigned grid = (unsigned)(p.B * p.H);
+  if (p.prestep)
+    decode_kernel<TI, DK, DV, GATE, true><<<grid, kWarps * 32, 0, st>>>(p);
+  else
+    decode_kernel<TI, DK, DV, GATE, false><<<grid, kWarps * 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <typename TI, int DK, int DV>
 cudaError_t launch_t(const DecodeProblem& p, cudaStream_t st) {
-  const unsigned grid = (unsigned)(p.B * p.H);
-  if (p.alpha)
-    decode_kernel<TI, DK, DV, true><<<grid, kWarps * 32, 0, st>>>(p);
-  else
-    decode_kernel<TI, DK, DV, false><<<grid, kWarps * 32, 0, st>>>(p);
-  return cudaGetLastError();
+  if (!p.alpha) return launch_g<TI, DK, DV, 0>(p, st);
+  return p.alpha_per_dim ? launch_g<TI, DK, DV, 2>(p, st) : launch_g<TI, DK, DV, 1>(p, st);
 }
 
 template <typename TI>

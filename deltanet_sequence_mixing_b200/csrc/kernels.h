@@ -31,6 +31,8 @@ struct ChunkProblem {
   int B, H, T, Dk, Dv, C;
   int bf16;            // 1: q/k/v/o are bfloat16, 0: float32
   Mode mode;
+  int prestep;         // Delta only: q, k raw and beta logits (silu + L2 normalise, sigmoid inside)
+  int alpha_per_dim;   // Delta only: alpha is (B,H,T,Dk), one decay per key dimension
   unsigned int* status;  // device status word (workspace)
 };
 
@@ -54,6 +56,8 @@ struct DecodeProblem {
   void* o;
   int B, H, Dk, Dv;
   int bf16;
+  int prestep;        // q, k raw and beta logits: silu + L2 normalise, sigmoid inside
+  int alpha_per_dim;  // alpha is (B,H,Dk): one decay per key dimension
 };
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t st);
 

@@ -9,6 +9,9 @@ Recipe (draw order fixed: q, k, v, beta, alpha):
   k     ~ N(0, 1), then L2-normalised per (token, head) in float32
   beta  = sigmoid(N(0, 1))                 float32, one per (b, h, t)
   alpha = exp(-softplus(N(0, 1)))          float32 in (0, 1), one per (b, h, t)
+                                           (per-dimension gate: one per (b, h, t, i))
+Inputs of the calls that apply the layer's pre-step themselves ("raw"): k is
+left unnormalised and beta is the N(0, 1) logit itself.
 q, k, v are stored in ``dtype`` (float32 or bfloat16) after the float32 draw.
 """
 from __future__ import annotations
@@ -54,20 +57,28 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
-def make_inputs(B, H, T, Dk, Dv, dtype=torch.bfloat16, gated=False, seed=0, device="cpu"):
+def make_inputs(B, H, T, Dk, Dv, dtype=torch.bfloat16, gated=False, seed=0, device="cpu",
+                raw=False, gate_per_dim=False):
     """Return dict(q, k, v, beta, alpha) drawn with the recipe above.
 
-    ``alpha`` is None unless ``gated``.  All tensors are contiguous on ``device``.
+    ``alpha`` is None unless ``gated``; with ``gate_per_dim`` it has one decay
+    per key dimension, shape (B,H,T,Dk), drawn the same way.  ``raw`` leaves k
+    unnormalised and beta as its N(0,1) logit (the inputs of the call that
+    applies the layer's maps itself).  All tensors are contiguous on ``device``.
     """
     g = _gen(seed, device)
     q = torch.randn(B, H, T, Dk, generator=g, device=device, dtype=torch.float32)
     k = torch.randn(B, H, T, Dk, generator=g, device=device, dtype=torch.float32)
-    k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+    if not raw:
+        k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-30)
     v = torch.randn(B, H, T, Dv, generator=g, device=device, dtype=torch.float32)
-    beta = torch.sigmoid(torch.randn(B, H, T, generator=g, device=device, dtype=torch.float32))
+    beta = torch.randn(B, H, T, generator=g, device=device, dtype=torch.float32)
+    if not raw:
+        beta = torch.sigmoid(beta)
     alpha = None
     if gated:
-        x = torch.randn(B, H, T, generator=g, device=device, dtype=torch.float32)
+        shape = (B, H, T, Dk) if gate_per_dim else (B, H, T)
+        x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
         alpha = torch.exp(-torch.nn.functional.softplus(x))
     return dict(q=q.to(dtype).contiguous(), k=k.to(dtype).contiguous(),
                 v=v.to(dtype).contiguous(), beta=beta.contiguous(),
@@ -79,8 +90,9 @@ def make_workload(w: Workload, seed=0, device="cpu"):
 
 
 def make_decode_step_inputs(B, H, Dk, Dv, dtype=torch.bfloat16, gated=False, seed=0,
-                            device="cpu"):
-    """One decode step's q, k, v (B,H,D), beta (B,H) and optional alpha (B,H)."""
-    d = make_inputs(B, H, 1, Dk, Dv, dtype, gated, seed, device)
+                            device="cpu", raw=False, gate_per_dim=False):
+    """One decode step's q, k, v (B,H,D), beta (B,H) and optional alpha (B,H)
+    (or (B,H,Dk) with ``gate_per_dim``)."""
+    d = make_inputs(B, H, 1, Dk, Dv, dtype, gated, seed, device, raw, gate_per_dim)
     return {n: (None if t is None else t.reshape(t.shape[:2] + t.shape[3:]).contiguous())
             for n, t in d.items()}

@@ -115,6 +115,50 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
                        void *workspace, size_t ws_bytes, void *cuda_stream);
 
 /*
+ * Options of the *_ex entry points (bit flags, OR-ed together; 0 gives the
+ * plain call).
+ *
+ * DN_OPT_PRESTEP: the DeltaNet layer's feature maps run inside the call ([P3]
+ *   "DeltaNet (Fast weight programmers)", the layer's forward: q and k go
+ *   through silu and an L2 normalisation over the head dimension, beta through
+ *   a sigmoid).  q and k are then the raw projections and beta holds logits;
+ *   per token  q <- silu(q) / max(||silu(q)||_2, 1e-12),  likewise k,
+ *   beta <- 1 / (1 + exp(-beta)).  This saves the separate elementwise pass
+ *   (and its HBM round trip) over q, k and beta.
+ * DN_OPT_GATE_PER_DIM: alpha holds one decay per key dimension, (B,H,T,Dk)
+ *   for the chunked call and (B,H,Dk) for the decode step: row i of the state
+ *   decays by alpha_t[i] before the delta write ([P1], the KDA paragraph:
+ *   scalar gating replaced by per-dimension gating).  alpha must not be NULL.
+ *
+ * Paths: with either option the chunked call runs on the CUDA-core kernel
+ * (float32 arithmetic, bf16 or f32 inputs, C = 64 only; C = 128 gives
+ * DN_ERR_UNSUPPORTED) and needs only the 256-byte status word as workspace;
+ * the decode step takes both options on its usual kernel.  Unknown bits give
+ * DN_ERR_INVALID_ARG.
+ */
+enum {
+    DN_OPT_PRESTEP = 1,
+    DN_OPT_GATE_PER_DIM = 2
+};
+
+/* deltanet_workspace_bytes for a deltanet_chunk_fwd_ex call with `options`. */
+size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                                   unsigned int options);
+
+/*
+ * deltanet_chunk_fwd with options (see above).  Arguments, layout, ownership,
+ * aliasing and status codes as deltanet_chunk_fwd, except: with
+ * DN_OPT_PRESTEP q and k are raw projections and beta holds logits; with
+ * DN_OPT_GATE_PER_DIM alpha is (B,H,T,Dk) float32 in [0,1].
+ */
+int deltanet_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                          const float *beta, const float *alpha, const float *S0,
+                          void *o, float *S_out,
+                          int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                          unsigned int options,
+                          void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
  * One recurrent decode step for a batch of B x H states, updated in place.
  *
  * The case t = 1 of the recurrence above ([P3] "DeltaNet (Fast weight
@@ -135,6 +179,18 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
 int deltanet_decode_step(const void *q, const void *k, const void *v,
                          const float *beta, const float *alpha, float *S, void *o,
                          int B, int H, int Dk, int Dv, dn_dtype dt, void *cuda_stream);
+
+/*
+ * deltanet_decode_step with options (see above): with DN_OPT_PRESTEP q and k
+ * are raw projections and beta logits (the maps run in the kernel); with
+ * DN_OPT_GATE_PER_DIM alpha is (B,H,Dk): row i of S is scaled by alpha[i]
+ * before the read, then u = beta (v - k S'), o = q S' + (q . k) u,
+ * S <- S' + k^T u.  Each state is still read once and written once.
+ */
+int deltanet_decode_step_ex(const void *q, const void *k, const void *v,
+                            const float *beta, const float *alpha, float *S, void *o,
+                            int B, int H, int Dk, int Dv, dn_dtype dt, unsigned int options,
+                            void *cuda_stream);
 
 /*
  * Causal linear attention with the ELU+1 feature map (the additive special

@@ -221,3 +221,36 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 1, 4, 64)
     with pytest.raises(ValueError, match="CUDA"):
         dn.deltanet_chunk_fwd(x, x, x, torch.zeros(1, 1, 4))
+
+
+def test_option_flags_are_validated_on_the_host(L):
+    """The *_ex calls: unknown option bits, a per-dimension gate without alpha,
+    and the options with C = 128 are rejected before any CUDA call."""
+    E = _lib
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def ex(opts, alpha=None, C=64, T=100):
+        return L.deltanet_chunk_fwd_ex(vp(A), vp(A + 64 * MB), vp(A + 128 * MB), vp(A + 192 * MB),
+                                       vp(alpha), None, vp(A + 256 * MB), vp(A + 320 * MB),
+                                       2, 2, T, 64, 64, C, 1, opts, vp(A + 400 * MB), 1 << 20, None)
+
+    assert ex(4) == E.DN_ERR_INVALID_ARG
+    assert ex(E.DN_OPT_GATE_PER_DIM) == E.DN_ERR_INVALID_ARG  # per-dimension gate needs alpha
+    assert ex(E.DN_OPT_PRESTEP, C=128) == E.DN_ERR_UNSUPPORTED
+    assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 500 * MB, C=128) == E.DN_ERR_UNSUPPORTED
+    # the per-dimension alpha covers B*H*T*Dk floats: an alpha that ends inside o overlaps it
+    assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 256 * MB - 2 * 2 * 100 * 64 * 4 + 64) == E.DN_ERR_INVALID_ARG
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 1) == 256
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 128, 1, 1) == 0
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 8) == 0
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 0) == \
+        L.deltanet_workspace_bytes(2, 2, 100, 64, 64, 64, 1)
+
+    def dec(opts, alpha=None):
+        return L.deltanet_decode_step_ex(vp(A), vp(A + MB), vp(A + 2 * MB), vp(A + 3 * MB), vp(alpha),
+                                         vp(A + 8 * MB), vp(A + 4 * MB), 4, 2, 128, 128, 1, opts, None)
+
+    assert dec(4) == E.DN_ERR_INVALID_ARG
+    assert dec(E.DN_OPT_GATE_PER_DIM) == E.DN_ERR_INVALID_ARG
+    # a (B,H,Dk) alpha of 4*2*128 floats starting 1 KB before S overlaps S
+    assert dec(E.DN_OPT_GATE_PER_DIM, alpha=A + 8 * MB - 1024) == E.DN_ERR_INVALID_ARG
