@@ -7,6 +7,7 @@ product library never loads it, and it never loads the product library.
 * ``deltanet``     - the per-token delta rule (optionally gated, per-dimension
                      gated, or behind the layer's silu / L2 / sigmoid pre-step),
                      ``oracle.c``.
+* ``deltanet_bwd`` - its gradient, the reverse sweep of the per-token loop, ``oracle.c``.
 * ``linear_attn``  - ELU+1 causal linear attention, ``oracle.c``.
 * ``chunk_form``   - the chunkwise WY form in numpy (see ``chunk_form.py``).
 
@@ -28,7 +29,7 @@ _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-F32, BF16 = 0, 1
+F32, BF16, F64 = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -54,6 +55,9 @@ def _load():
         lib.oracle_linear_attn.restype = I
         lib.oracle_deltanet_ex.argtypes = [vp, vp, vp, I, fp, fp, dp, dp, dp, L, L, L, L, L, I, I]
         lib.oracle_deltanet_ex.restype = I
+        lib.oracle_deltanet_bwd.argtypes = [vp, vp, vp, I, fp, fp, dp, dp, dp,
+                                            dp, dp, dp, dp, dp, dp, L, L, L, L, L, I]
+        lib.oracle_deltanet_bwd.restype = I
         _lib = lib
     return _lib
 
@@ -69,10 +73,14 @@ def _as_stored(x):
                 return x.view(torch.int16).numpy().view(np.uint16), BF16
             if x.dtype == torch.float32:
                 return x.numpy(), F32
+            if x.dtype == torch.float64:
+                return x.numpy(), F64
             raise TypeError(f"oracle inputs must be float32 or bfloat16, got {x.dtype}")
     except ImportError:  # pragma: no cover
         pass
     x = np.ascontiguousarray(x)
+    if x.dtype == np.float64:
+        return x, F64
     if x.dtype == np.float32:
         return x, F32
     if x.dtype == np.uint16:
@@ -155,6 +163,38 @@ def deltanet(q, k, v, beta, alpha=None, S0=None, nthreads: int = 0, prestep: boo
     if rc != 0:
         raise RuntimeError(f"oracle_deltanet failed ({rc})")
     return o, S
+
+
+def deltanet_bwd(q, k, v, beta, dO, alpha=None, S0=None, dS_T=None, nthreads: int = 0):
+    """Gradient of the delta rule: the reverse sweep of the per-token loop (see
+    ``oracle_deltanet_bwd`` in ``oracle.c``), in float64.
+
+    The loss is ``sum(dO * o) + sum(dS_T * S_T)``.  Returns a dict with dq, dk
+    (B,H,T,Dk), dv (B,H,T,Dv), dbeta (B,H,T), dalpha (B,H,T, or None when
+    ungated) and dS0 (B,H,Dk,Dv).  q, k, v may be float64, float32 or bfloat16.
+    """
+    qa, dt = _as_stored(q)
+    ka, dtk = _as_stored(k)
+    va, dtv = _as_stored(v)
+    if not (dt == dtk == dtv):
+        raise TypeError("q, k, v must share one dtype")
+    B, H, T, Dk = qa.shape
+    Dv = va.shape[-1]
+    b = _f32(beta).reshape(B, H, T)
+    a = None if alpha is None else _f32(alpha).reshape(B, H, T)
+    s0 = None if S0 is None else _f64(S0).reshape(B, H, Dk, Dv)
+    do = _f64(dO).reshape(B, H, T, Dv)
+    dst = None if dS_T is None else _f64(dS_T).reshape(B, H, Dk, Dv)
+    out = dict(dq=np.zeros((B, H, T, Dk)), dk=np.zeros((B, H, T, Dk)), dv=np.zeros((B, H, T, Dv)),
+               dbeta=np.zeros((B, H, T)), dalpha=None if a is None else np.zeros((B, H, T)),
+               dS0=np.zeros((B, H, Dk, Dv)))
+    rc = _load().oracle_deltanet_bwd(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(b), _ptr(a), _ptr(s0),
+                                     _ptr(do), _ptr(dst), _ptr(out["dq"]), _ptr(out["dk"]),
+                                     _ptr(out["dv"]), _ptr(out["dbeta"]), _ptr(out["dalpha"]),
+                                     _ptr(out["dS0"]), B, H, T, Dk, Dv, nthreads)
+    if rc != 0:
+        raise RuntimeError(f"oracle_deltanet_bwd failed ({rc})")
+    return out
 
 
 def linear_attn(q, k, v, S0=None, z0=None, nthreads: int = 0):

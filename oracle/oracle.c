@@ -36,7 +36,7 @@
 #include <unistd.h>
 
 /* Input element types understood by the oracle. */
-enum { ORC_F32 = 0, ORC_BF16 = 1 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_F64 = 2 };
 
 /* Options of the delta rule.
  *   ORC_PRESTEP: q and k are the raw projections and beta holds logits; each
@@ -53,6 +53,8 @@ enum { ORC_PRESTEP = 1, ORC_ALPHA_PER_DIM = 2 };
  * of the float32 with the same value, so the widening is exact. */
 static double widen(const void *p, int dtype, size_t i)
 {
+    if (dtype == ORC_F64)
+        return ((const double *)p)[i];
     if (dtype == ORC_F32)
         return (double)((const float *)p)[i];
     uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
@@ -331,4 +333,207 @@ int oracle_linear_attn(const void *q, const void *k, const void *v, int dtype,
     J.B = B; J.H = H; J.T = T; J.Dk = Dk; J.Dv = Dv;
     J.linear = 1;
     return run(&J, nthreads);
+}
+
+
+/* ------------------------------------------------------------------------ */
+/* Gradient of the delta rule (reverse mode of the per-token loop).
+ *
+ * [P3] "DeltaNet (Parallelizing linear transformers with delta rule)" presents
+ * the chunked form as what makes linear-time training hardware-efficient; the
+ * training step needs the gradient of the same recurrence.  This is the plain
+ * reverse sweep of the per-token loop above (gated as [P1]'s Gated DeltaNet),
+ * written from the chain rule, one token at a time from the last:
+ *
+ *   forward   S'_t = a_t S_{t-1};  r_t = k_t S'_t;  u_t = b_t (v_t - r_t);
+ *             S_t = S'_t + k_t^T u_t;  o_t = q_t S_t
+ *   backward  G  <- G + q_t^T dO_t                  (G = dL/dS_t)
+ *             dq_t = dO_t S_t^T
+ *             du   = k_t G;     dk_t  = G u_t^T
+ *             db_t = du . (v_t - r_t);   dv_t = b_t du;   dr = -b_t du
+ *             dk_t += dr S'_t^T;  G' = G + k_t^T dr  (= dL/dS'_t)
+ *             da_t = <G', S_{t-1}>;   G <- a_t G'     (= dL/dS_{t-1})
+ *   dS0 = G after token 0.  The loss is sum(dO * o) + sum(dS_T * S_T).
+ *
+ * The forward states are kept for the sweep ((T+1) Dk Dv doubles per
+ * sequence).  Inputs as oracle_deltanet (q, k, v may also be float64, dtype
+ * 2); alpha is per token (or NULL); dO (B,H,T,Dv) and dS_T (B,H,Dk,Dv, nullable)
+ * are float64; outputs dq, dk (B,H,T,Dk), dv (B,H,T,Dv), dbeta (B,H,T), dalpha
+ * (B,H,T, nullable) and dS0 (B,H,Dk,Dv) are float64.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    int dtype;
+    const float *beta, *alpha;
+    const double *S0, *dO, *dST;
+    double *dq, *dk, *dv, *dbeta, *dalpha, *dS0;
+    long B, H, T, Dk, Dv;
+    long next;
+    pthread_mutex_t lock;
+} bjob_t;
+
+static void delta_sequence_bwd(const bjob_t *J, long bh, double *Ss, double *G, double *w)
+{
+    const long T = J->T, Dk = J->Dk, Dv = J->Dv, DD = Dk * Dv;
+    const size_t qk0 = (size_t)bh * T * Dk, v0 = (size_t)bh * T * Dv, s0 = (size_t)bh * DD;
+    double *kk = w, *qq = w + Dk, *r = w + 2 * Dk, *u = r + Dv, *du = u + Dv, *dr = du + Dv;
+
+    /* forward sweep: Ss holds S_{-1} = S0, S_0, ..., S_{T-1} */
+    for (long i = 0; i < DD; ++i)
+        Ss[i] = J->S0 ? J->S0[s0 + i] : 0.0;
+    for (long t = 0; t < T; ++t) {
+        const double *Sp = Ss + (size_t)t * DD;
+        double *Sn = Ss + (size_t)(t + 1) * DD;
+        const double beta = (double)J->beta[(size_t)bh * T + t];
+        const double alpha = J->alpha ? (double)J->alpha[(size_t)bh * T + t] : 1.0;
+        for (long i = 0; i < Dk; ++i)
+            kk[i] = widen(J->k, J->dtype, qk0 + (size_t)t * Dk + i);
+        for (long i = 0; i < DD; ++i)
+            Sn[i] = alpha * Sp[i];
+        for (long j = 0; j < Dv; ++j) {
+            r[j] = 0.0;
+            for (long i = 0; i < Dk; ++i)
+                r[j] += kk[i] * Sn[i * Dv + j];
+            u[j] = beta * (widen(J->v, J->dtype, v0 + (size_t)t * Dv + j) - r[j]);
+        }
+        for (long i = 0; i < Dk; ++i)
+            for (long j = 0; j < Dv; ++j)
+                Sn[i * Dv + j] += kk[i] * u[j];
+    }
+    /* reverse sweep */
+    for (long i = 0; i < DD; ++i)
+        G[i] = J->dST ? J->dST[s0 + i] : 0.0;
+    for (long t = T - 1; t >= 0; --t) {
+        const double *Sprev = Ss + (size_t)t * DD, *St = Ss + (size_t)(t + 1) * DD;
+        const double beta = (double)J->beta[(size_t)bh * T + t];
+        const double alpha = J->alpha ? (double)J->alpha[(size_t)bh * T + t] : 1.0;
+        const double *dO = J->dO + v0 + (size_t)t * Dv;
+        for (long i = 0; i < Dk; ++i) {
+            kk[i] = widen(J->k, J->dtype, qk0 + (size_t)t * Dk + i);
+            qq[i] = widen(J->q, J->dtype, qk0 + (size_t)t * Dk + i);
+        }
+        /* o_t = q_t S_t */
+        for (long i = 0; i < Dk; ++i)
+            for (long j = 0; j < Dv; ++j)
+                G[i * Dv + j] += qq[i] * dO[j];
+        double *dq = J->dq + qk0 + (size_t)t * Dk, *dk = J->dk + qk0 + (size_t)t * Dk;
+        for (long i = 0; i < Dk; ++i) {
+            double acc = 0.0;
+            for (long j = 0; j < Dv; ++j)
+                acc += dO[j] * St[i * Dv + j];
+            dq[i] = acc;
+        }
+        /* recompute r_t, u_t from S'_t = alpha S_{t-1} */
+        for (long j = 0; j < Dv; ++j) {
+            r[j] = 0.0;
+            for (long i = 0; i < Dk; ++i)
+                r[j] += kk[i] * alpha * Sprev[i * Dv + j];
+            u[j] = beta * (widen(J->v, J->dtype, v0 + (size_t)t * Dv + j) - r[j]);
+        }
+        /* S_t = S'_t + k_t^T u_t */
+        for (long j = 0; j < Dv; ++j) {
+            du[j] = 0.0;
+            for (long i = 0; i < Dk; ++i)
+                du[j] += kk[i] * G[i * Dv + j];
+        }
+        for (long i = 0; i < Dk; ++i) {
+            double acc = 0.0;
+            for (long j = 0; j < Dv; ++j)
+                acc += G[i * Dv + j] * u[j];
+            dk[i] = acc;
+        }
+        /* u_t = beta_t (v_t - r_t) */
+        double db = 0.0;
+        double *dv = J->dv + v0 + (size_t)t * Dv;
+        for (long j = 0; j < Dv; ++j) {
+            db += du[j] * (widen(J->v, J->dtype, v0 + (size_t)t * Dv + j) - r[j]);
+            dv[j] = beta * du[j];
+            dr[j] = -beta * du[j];
+        }
+        J->dbeta[(size_t)bh * T + t] = db;
+        /* r_t = k_t S'_t */
+        for (long i = 0; i < Dk; ++i) {
+            double acc = 0.0;
+            for (long j = 0; j < Dv; ++j)
+                acc += dr[j] * alpha * Sprev[i * Dv + j];
+            dk[i] += acc;
+        }
+        for (long i = 0; i < Dk; ++i)
+            for (long j = 0; j < Dv; ++j)
+                G[i * Dv + j] += kk[i] * dr[j];
+        /* S'_t = alpha_t S_{t-1} */
+        if (J->dalpha) {
+            double da = 0.0;
+            for (long i = 0; i < DD; ++i)
+                da += G[i] * Sprev[i];
+            J->dalpha[(size_t)bh * T + t] = da;
+        }
+        for (long i = 0; i < DD; ++i)
+            G[i] *= alpha;
+    }
+    memcpy(J->dS0 + s0, G, sizeof(double) * (size_t)DD);
+}
+
+static void *bwd_worker(void *arg)
+{
+    bjob_t *J = (bjob_t *)arg;
+    const size_t DD = (size_t)(J->Dk * J->Dv);
+    double *Ss = (double *)malloc(sizeof(double) * DD * (size_t)(J->T + 1));
+    double *G = (double *)malloc(sizeof(double) * DD);
+    double *w = (double *)malloc(sizeof(double) * (size_t)(2 * J->Dk + 4 * J->Dv));
+    void *rc = NULL;
+    if (!Ss || !G || !w) {
+        rc = (void *)1;
+    } else {
+        for (;;) {
+            pthread_mutex_lock(&J->lock);
+            const long bh = J->next++;
+            pthread_mutex_unlock(&J->lock);
+            if (bh >= J->B * J->H)
+                break;
+            delta_sequence_bwd(J, bh, Ss, G, w);
+        }
+    }
+    free(Ss);
+    free(G);
+    free(w);
+    return rc;
+}
+
+int oracle_deltanet_bwd(const void *q, const void *k, const void *v, int dtype,
+                        const float *beta, const float *alpha, const double *S0,
+                        const double *dO, const double *dST,
+                        double *dq, double *dk, double *dv, double *dbeta, double *dalpha,
+                        double *dS0, long B, long H, long T, long Dk, long Dv, int nthreads)
+{
+    if (B < 0 || H < 0 || T < 0 || Dk <= 0 || Dv <= 0)
+        return -1;
+    bjob_t J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k; J.v = v; J.dtype = dtype;
+    J.beta = beta; J.alpha = alpha; J.S0 = S0; J.dO = dO; J.dST = dST;
+    J.dq = dq; J.dk = dk; J.dv = dv; J.dbeta = dbeta; J.dalpha = dalpha; J.dS0 = dS0;
+    J.B = B; J.H = H; J.T = T; J.Dk = Dk; J.Dv = Dv;
+    if (nthreads <= 0)
+        nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > B * H)
+        nthreads = (int)(B * H > 0 ? B * H : 1);
+    pthread_mutex_init(&J.lock, NULL);
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!th)
+        return -2;
+    int rc = 0;
+    for (int i = 0; i < nthreads; ++i)
+        pthread_create(&th[i], NULL, bwd_worker, &J);
+    for (int i = 0; i < nthreads; ++i) {
+        void *ret = NULL;
+        pthread_join(th[i], &ret);
+        if (ret)
+            rc = -2;
+    }
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return rc;
 }

@@ -426,3 +426,82 @@ def test_prestep_zero_key_writes_nothing(oracle_mod):
     qn = torch.nn.functional.normalize(torch.nn.functional.silu(torch.from_numpy(q[0, 0, 0]).double()),
                                        dim=-1).numpy()
     np.testing.assert_allclose(o[0, 0, 0], qn @ S0[0, 0], rtol=1e-12)
+
+
+# -- the gradient (reverse sweep) ------------------------------------------------------
+
+def _fd_check(oracle_mod, gated):
+    """Every gradient entry of oracle.deltanet_bwd against a central finite
+    difference of the forward oracle's loss sum(dO * o) + sum(dS_T * S_T),
+    Richardson-extrapolated (error O(h^4)).  q, k, v, S0 are perturbed in
+    float64; beta and alpha (float32 inputs of the oracle) sit on a 2^-14 grid
+    and are perturbed by 2^-9 and 2^-8, which float32 holds exactly."""
+    rng = np.random.default_rng(61 + gated)
+    B, H, T, Dk, Dv = 1, 2, 6, 3, 2
+    q = rng.standard_normal((B, H, T, Dk))
+    k = rng.standard_normal((B, H, T, Dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, H, T, Dv))
+    grid = lambda x: (np.round(x * 2 ** 14) / 2 ** 14).astype(np.float32)
+    beta = grid(rng.uniform(0.2, 0.8, (B, H, T)))
+    alpha = grid(rng.uniform(0.5, 0.95, (B, H, T))) if gated else None
+    S0 = rng.standard_normal((B, H, Dk, Dv)) * 0.5
+    dO = rng.standard_normal((B, H, T, Dv))
+    dST = rng.standard_normal((B, H, Dk, Dv))
+    g = oracle_mod.deltanet_bwd(q, k, v, beta, dO, alpha, S0, dST)
+
+    def loss(q_, k_, v_, b_, a_, s_):
+        o, S = oracle_mod.deltanet(q_, k_, v_, b_, a_, s_)
+        return float((o * dO).sum() + (S * dST).sum())
+
+    def fd(name, x, h, cast=lambda y: y):
+        grad = np.zeros(x.shape)
+        for idx in np.ndindex(x.shape):
+            def at(step):
+                y = x.astype(np.float64).copy()
+                y[idx] += step
+                args = dict(q_=q, k_=k, v_=v, b_=beta, a_=alpha, s_=S0)
+                args[name] = cast(y)
+                return loss(**args)
+            d1 = (at(h) - at(-h)) / (2 * h)
+            d2 = (at(2 * h) - at(-2 * h)) / (4 * h)
+            grad[idx] = (4 * d1 - d2) / 3
+        return grad
+
+    f32 = lambda y: y.astype(np.float32)
+    checks = [("dq", fd("q_", q, 1e-4)), ("dk", fd("k_", k, 1e-4)), ("dv", fd("v_", v, 1e-4)),
+              ("dS0", fd("s_", S0, 1e-4)), ("dbeta", fd("b_", beta, 2.0 ** -9, f32))]
+    if gated:
+        checks.append(("dalpha", fd("a_", alpha, 2.0 ** -9, f32)))
+    for name, ref in checks:
+        np.testing.assert_allclose(g[name], ref, rtol=1e-7, atol=1e-8, err_msg=name)
+    if not gated:
+        assert g["dalpha"] is None
+
+
+def test_gradient_matches_finite_differences(oracle_mod):
+    _fd_check(oracle_mod, gated=False)
+
+
+def test_gradient_matches_finite_differences_gated(oracle_mod):
+    _fd_check(oracle_mod, gated=True)
+
+
+def test_gradient_of_a_single_write(oracle_mod):
+    """One token from S0 = 0 (worked by hand): S = b k^T v, o = b (q.k) v, so
+    dL/dv = b (q.k) dO + b dS^T k, dL/db = (q.k) (v.dO) + k dS v^T,
+    dL/dq = b (v.dO) k, dL/dS0 = q^T dO + dS - b k^T (k (q^T dO + dS))."""
+    q = np.array([[[[1.0, 2.0]]]])
+    k = np.array([[[[0.6, 0.8]]]])
+    v = np.array([[[[3.0, -1.0]]]])
+    b = np.array([[[0.5]]], np.float32)
+    dO = np.array([[[[1.0, 2.0]]]])
+    dS = np.array([[[[0.5, 0.0], [0.0, -1.0]]]])
+    g = oracle_mod.deltanet_bwd(q, k, v, b, dO, dS_T=dS)
+    qk, vdo = 0.6 + 1.6, 3.0 - 2.0
+    kdSv = k[0, 0, 0] @ dS[0, 0] @ v[0, 0, 0]
+    np.testing.assert_allclose(g["dv"][0, 0, 0], 0.5 * qk * dO[0, 0, 0] + 0.5 * dS[0, 0].T @ k[0, 0, 0])
+    np.testing.assert_allclose(g["dbeta"][0, 0, 0], qk * vdo + kdSv)
+    np.testing.assert_allclose(g["dq"][0, 0, 0], 0.5 * vdo * k[0, 0, 0])
+    Gt = np.outer(q[0, 0, 0], dO[0, 0, 0]) + dS[0, 0]
+    np.testing.assert_allclose(g["dS0"][0, 0], Gt - 0.5 * np.outer(k[0, 0, 0], k[0, 0, 0] @ Gt))
