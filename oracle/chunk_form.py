@@ -104,3 +104,102 @@ def linear_attn_chunked(q, k, v, S0=None, z0=None, C: int = 64):
                 z = z + K.sum(axis=0)
             S_all[b, h], z_all[b, h] = S, z
     return o, S_all, z_all
+
+
+def deltanet_chunked_bwd(q, k, v, beta, dO, alpha=None, S0=None, dS_T=None, C: int = 64):
+    """Gradient of the chunk form above, chunk by chunk from the last (numpy
+    float64, test-side math).  The loss is sum(dO * o) + sum(dS_T * S_T).
+    Returns dict(dq, dk, dv, dbeta, dlogalpha, dS0); dlogalpha (the gradient with
+    respect to log alpha, = alpha * dL/dalpha) is None when ungated.
+
+    With g the within-chunk cumulative log decay, Gamma = exp(g_r - g_s) and
+    gamma = exp(g), every quantity of the forward is a product of matrices, so
+    the reverse pass runs the same products transposed:
+      dU  = (tril(Q K^T) * Gamma)^T dO + K_out dS+          K_out = diag(gamma_n / gamma) K
+      dS  = (diag(gamma) Q)^T dO + gamma_n dS+ - W^T dU     W = T diag(beta gamma) K
+      dP  = tril(dO U^T)  (scores),  dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T
+      dA  = -strict_lower(T^T dT T^T)
+    and the chain rule through Gamma / gamma gives the gradient of g, whose
+    reverse cumulative sum within the chunk is the gradient of log alpha.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    beta = np.asarray(beta, np.float64)
+    dO = np.asarray(dO, np.float64)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    gated = alpha is not None
+    la = np.zeros((B, H, T)) if alpha is None else np.log(np.asarray(alpha, np.float64))
+    out = dict(dq=np.zeros((B, H, T, Dk)), dk=np.zeros((B, H, T, Dk)), dv=np.zeros((B, H, T, Dv)),
+               dbeta=np.zeros((B, H, T)), dlogalpha=np.zeros((B, H, T)) if gated else None,
+               dS0=np.zeros((B, H, Dk, Dv)))
+    for b in range(B):
+        for h in range(H):
+            chunks = [slice(c0, min(c0 + C, T)) for c0 in range(0, T, C)]
+            # forward: entry state of every chunk
+            S = np.zeros((Dk, Dv)) if S0 is None else np.array(S0[b, h], np.float64)
+            entry = []
+            for sl in chunks:
+                entry.append(S.copy())
+                Q, K, V, bt = q[b, h, sl], k[b, h, sl], v[b, h, sl], beta[b, h, sl]
+                n = Q.shape[0]
+                g = np.cumsum(la[b, h, sl])
+                Gam = np.tril(np.exp(g[:, None] - g[None, :]))
+                gam = np.exp(g)
+                Tm = np.linalg.inv(np.eye(n) + np.tril(bt[:, None] * (K @ K.T) * Gam, -1))
+                U = Tm @ (bt[:, None] * (V - gam[:, None] * (K @ S)))
+                S = gam[-1] * S + (np.exp(g[-1] - g)[:, None] * K).T @ U
+            dSp = np.zeros((Dk, Dv)) if dS_T is None else np.array(dS_T[b, h], np.float64)
+            for ci in range(len(chunks) - 1, -1, -1):
+                sl, S = chunks[ci], entry[ci]
+                Q, K, V, bt = q[b, h, sl], k[b, h, sl], v[b, h, sl], beta[b, h, sl]
+                dOc = dO[b, h, sl]
+                n = Q.shape[0]
+                g = np.cumsum(la[b, h, sl])
+                Gam = np.tril(np.exp(g[:, None] - g[None, :]))
+                gam = np.exp(g)
+                e_out = np.exp(g[-1] - g)
+                MA = (K @ K.T) * Gam
+                A = np.tril(bt[:, None] * MA, -1)
+                Tm = np.linalg.inv(np.eye(n) + A)
+                BK = (bt * gam)[:, None] * K
+                BV = bt[:, None] * V
+                W, Uh = Tm @ BK, Tm @ BV
+                U = Uh - W @ S
+                MP = np.tril((Q @ K.T) * Gam)
+                Kout = e_out[:, None] * K
+                # reverse
+                dU = MP.T @ dOc + Kout @ dSp
+                dS = (gam[:, None] * Q).T @ dOc + gam[-1] * dSp - W.T @ dU
+                dMP = np.tril(dOc @ U.T)
+                dQ = gam[:, None] * (dOc @ S.T) + (dMP * Gam) @ K
+                dK = (dMP * Gam).T @ Q + e_out[:, None] * (U @ dSp.T)
+                dg = gam * np.sum(dOc * (Q @ S), axis=1)
+                EP = dMP * MP
+                dg += EP.sum(1) - EP.sum(0)
+                c_out = e_out * np.sum(K * (U @ dSp.T), axis=1)
+                dg[-1] += gam[-1] * np.sum(dSp * S) + c_out.sum()
+                dg -= c_out
+                dW = -dU @ S.T
+                dT = dW @ BK.T + dU @ BV.T
+                dBK, dBV = Tm.T @ dW, Tm.T @ dU
+                dV = bt[:, None] * dBV
+                dK += (bt * gam)[:, None] * dBK
+                dbt = gam * np.sum(dBK * K, axis=1) + np.sum(dBV * V, axis=1)
+                dg += bt * gam * np.sum(dBK * K, axis=1)
+                dA = -np.tril(Tm.T @ dT @ Tm.T, -1)
+                dbt += np.sum(dA * MA, axis=1)
+                dMA = bt[:, None] * dA
+                dK += (dMA * Gam) @ K + (dMA * Gam).T @ K
+                EA = dMA * MA
+                dg += EA.sum(1) - EA.sum(0)
+                out["dq"][b, h, sl] = dQ
+                out["dk"][b, h, sl] = dK
+                out["dv"][b, h, sl] = dV
+                out["dbeta"][b, h, sl] = dbt
+                if gated:
+                    out["dlogalpha"][b, h, sl] = np.cumsum(dg[::-1])[::-1]
+                dSp = dS
+            out["dS0"][b, h] = dSp
+    return out

@@ -57,3 +57,30 @@ def test_linear_chunk_form_matches_recurrence(oracle_mod, C):
     np.testing.assert_allclose(o, o_ref, rtol=1e-11)
     np.testing.assert_allclose(S, S_ref, rtol=1e-11)
     np.testing.assert_allclose(z, z_ref, rtol=1e-11)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("C", [1, 5, 16, 64])
+def test_chunked_gradient_equals_reverse_sweep(oracle_mod, gated, C):
+    """The chunk-form gradient equals the oracle's per-token reverse sweep for
+    every chunk size (alpha * dL/dalpha for the log-decay gradient)."""
+    from oracle import chunk_form
+
+    rng = np.random.default_rng(70 + C + gated)
+    B, H, T, Dk, Dv = 1, 2, 37, 6, 5
+    q = rng.standard_normal((B, H, T, Dk))
+    k = rng.standard_normal((B, H, T, Dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, H, T, Dv))
+    beta = rng.uniform(0.1, 0.9, (B, H, T)).astype(np.float32)
+    alpha = rng.uniform(0.4, 1.0, (B, H, T)).astype(np.float32) if gated else None
+    S0 = rng.standard_normal((B, H, Dk, Dv)) * 0.3
+    dO = rng.standard_normal((B, H, T, Dv))
+    dST = rng.standard_normal((B, H, Dk, Dv))
+    ref = oracle_mod.deltanet_bwd(q, k, v, beta, dO, alpha, S0, dST)
+    got = chunk_form.deltanet_chunked_bwd(q, k, v, beta, dO, alpha, S0, dST, C=C)
+    for name in ("dq", "dk", "dv", "dbeta", "dS0"):
+        np.testing.assert_allclose(got[name], ref[name], rtol=1e-9, atol=1e-10, err_msg=name)
+    if gated:
+        np.testing.assert_allclose(got["dlogalpha"], alpha.astype(np.float64) * ref["dalpha"],
+                                   rtol=1e-9, atol=1e-10)
