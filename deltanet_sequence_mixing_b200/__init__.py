@@ -20,6 +20,7 @@ from ._lib import DeltaNetError, check, lib, status_string  # noqa: F401
 
 __all__ = [
     "deltanet_chunk_fwd", "deltanet_chunk_fwd_host", "deltanet_decode_step", "linear_attn_fwd",
+    "deltanet_chunk_bwd",
     "workspace_for", "host_workspace_for",
     "deltanet_get_device_status", "deltanet_selftest_wait_timeout", "DeltaNetError",
 ]
@@ -117,6 +118,39 @@ def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, 
             _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
             B, H, T, Dk, Dv, C, dt, opts, _ptr(ws), ws.numel(), _stream(dev)))
     return o, S_out
+
+
+def deltanet_chunk_bwd(q, k, v, beta, dO, alpha=None, S0=None, dS_T=None, workspace=None):
+    """Gradient of deltanet_chunk_fwd for the loss sum(dO * o) + sum(dS_T * S_T).
+    Returns dict(dq, dk, dv, dbeta, dlog_alpha, dS0), float32 tensors
+    (dlog_alpha is None when ungated)."""
+    _need(q, "q")
+    dev, dtype = q.device, q.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for t, n in ((k, "k"), (v, "v"), (dO, "dO")):
+        _need(t, n, dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
+    for t, n in ((alpha, "alpha"), (S0, "S0"), (dS_T, "dS_T")):
+        if t is not None:
+            _need(t, n, torch.float32, dev)
+    B, H, T, Dk = q.shape
+    Dv = v.shape[-1]
+    f = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty(B, H, T, Dk, **f), dk=torch.empty(B, H, T, Dk, **f),
+               dv=torch.empty(B, H, T, Dv, **f), dbeta=torch.empty(B, H, T, **f),
+               dlog_alpha=None if alpha is None else torch.empty(B, H, T, **f),
+               dS0=torch.empty(B, H, Dk, Dv, **f))
+    nb = lib().deltanet_chunk_bwd_workspace_bytes(B, H, T, Dk, Dv, _DT[dtype])
+    if nb == 0:
+        raise DeltaNetError("deltanet_chunk_bwd_workspace_bytes", _lib.DN_ERR_UNSUPPORTED)
+    ws = workspace if workspace is not None else torch.empty(nb, dtype=torch.uint8, device=dev)
+    check("deltanet_chunk_bwd", lib().deltanet_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(dO), _ptr(dS_T),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dbeta"]),
+        _ptr(out["dlog_alpha"]), _ptr(out["dS0"]), B, H, T, Dk, Dv, _DT[dtype], _ptr(ws), ws.numel(),
+        _stream(dev)))
+    return out
 
 
 def _need_host(t, name, dtype=None):

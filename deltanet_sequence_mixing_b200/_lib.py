@@ -43,6 +43,10 @@ SIGNATURES = {
     "deltanet_host_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "deltanet_chunk_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "deltanet_chunk_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "deltanet_chunk_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp, _vp, _vp, _vp, _vp, _vp,
+                                _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "deltanet_get_device_status": (_i, [_vp, _vp]),
     "deltanet_selftest_wait_timeout": (_i, [_vp, _sz, _ll, _vp]),
     "deltanet_status_string": (ctypes.c_char_p, [_i]),

@@ -407,6 +407,63 @@ int deltanet_decode_step_ex(const void* q, const void* k, const void* v, const f
   return map_cuda(dn::launch_decode(p, static_cast<cudaStream_t>(cuda_stream)));
 }
 
+size_t deltanet_chunk_bwd_workspace_bytes(int B, int H, int T, int Dk, int Dv, dn_dtype dt) {
+  if (B < 0 || H < 0 || T < 0 || !valid_dim(Dk) || !valid_dim(Dv)) return 0;
+  if (dt != DN_F32 && dt != DN_BF16) return 0;
+  if ((long long)B * H > INT_MAX) return 0;
+  return kStatusBytes + dn::chunk_bwd_state_bytes(B, H, T, Dk, Dv);
+}
+
+int deltanet_chunk_bwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* alpha, const float* S0, const void* dO, const float* dS_T,
+                       float* dq, float* dk, float* dv, float* dbeta, float* dlog_alpha, float* dS0,
+                       int B, int H, int T, int Dk, int Dv, dn_dtype dt, void* workspace,
+                       size_t ws_bytes, void* cuda_stream) {
+  if (dt != DN_F32 && dt != DN_BF16) return DN_ERR_UNSUPPORTED;
+  if (B < 0 || H < 0 || T < 0) return DN_ERR_INVALID_ARG;
+  if (!valid_dim(Dk) || !valid_dim(Dv)) return DN_ERR_UNSUPPORTED;
+  if ((long long)B * H > INT_MAX) return DN_ERR_UNSUPPORTED;
+  if (T > 0 && (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta))
+    return DN_ERR_INVALID_ARG;
+  if (dlog_alpha && !alpha) return DN_ERR_INVALID_ARG;
+  if (!workspace) return DN_ERR_WORKSPACE;
+  if (ws_bytes < deltanet_chunk_bwd_workspace_bytes(B, H, T, Dk, Dv, dt)) return DN_ERR_WORKSPACE;
+  const void* f32s[] = {beta, alpha, S0, dS_T, dq, dk, dv, dbeta, dlog_alpha, dS0, workspace};
+  for (const void* x : f32s)
+    if (x && (reinterpret_cast<uintptr_t>(x) & 3u)) return DN_ERR_ALIGNMENT;
+  if (!aligned16(workspace)) return DN_ERR_ALIGNMENT;
+  const size_t es = dt == DN_BF16 ? 2 : 4, BH = (size_t)B * H, TT = (size_t)T;
+  const Range ins[] = {range_of(q, BH * TT * Dk * es), range_of(k, BH * TT * Dk * es),
+                       range_of(v, BH * TT * Dv * es), range_of(beta, BH * TT * 4),
+                       range_of(alpha, alpha ? BH * TT * 4 : 0), range_of(S0, S0 ? BH * Dk * Dv * 4 : 0),
+                       range_of(dO, BH * TT * Dv * es), range_of(dS_T, dS_T ? BH * Dk * Dv * 4 : 0)};
+  const Range outs[] = {range_of(dq, BH * TT * Dk * 4), range_of(dk, BH * TT * Dk * 4),
+                        range_of(dv, BH * TT * Dv * 4), range_of(dbeta, BH * TT * 4),
+                        range_of(dlog_alpha, dlog_alpha ? BH * TT * 4 : 0),
+                        range_of(dS0, dS0 ? BH * Dk * Dv * 4 : 0), range_of(workspace, ws_bytes)};
+  for (size_t a = 0; a < sizeof outs / sizeof outs[0]; ++a) {
+    for (const Range& r : ins)
+      if (overlap(outs[a], r)) return DN_ERR_INVALID_ARG;
+    for (size_t b = a + 1; b < sizeof outs / sizeof outs[0]; ++b)
+      if (overlap(outs[a], outs[b])) return DN_ERR_INVALID_ARG;
+  }
+  if (BH == 0) return DN_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (T == 0) {  // no tokens: dL/dS0 is dL/dS_T
+    if (!dS0) return DN_OK;
+    const size_t nb = BH * Dk * Dv * 4;
+    return map_cuda(dS_T ? cudaMemcpyAsync(dS0, dS_T, nb, cudaMemcpyDeviceToDevice, st)
+                         : cudaMemsetAsync(dS0, 0, nb, st));
+  }
+  dn::BwdProblem p{};
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.alpha = alpha; p.S0 = S0; p.dO = dO; p.dS_T = dS_T;
+  p.dq = dq; p.dk = dk; p.dv = dv; p.dbeta = dbeta; p.dlog_alpha = dlog_alpha; p.dS0 = dS0;
+  p.states = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+  p.B = B; p.H = H; p.T = T; p.Dk = Dk; p.Dv = Dv;
+  p.bf16 = dt == DN_BF16;
+  return map_cuda(dn::launch_chunk_bwd(p, st));
+}
+
 int deltanet_get_device_status(const void* workspace, void* cuda_stream) {
   if (!workspace) return DN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);

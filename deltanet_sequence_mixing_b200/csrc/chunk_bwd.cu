@@ -1,0 +1,476 @@
+// Gradient of the chunked delta rule (the training backward), float32 on CUDA
+// cores.
+//
+// The pages present the chunkwise form as what makes linear-time TRAINING
+// hardware-efficient ("GPT-2 から Kimi K3 まで", news.ainew.jp, section "DeltaNet
+// (Parallelizing linear transformers with delta rule)"); this kernel runs the
+// reverse of that form.  Per chunk of C rows entered with state S (g = the
+// chunk's cumulative log decay, Gamma_rs = e^(g_r - g_s), gamma = e^g, n = last
+// row; ungated g = 0):
+//   forward   A = strict_lower(diag(beta) (K K^T * Gamma)),  T = (I + A)^-1
+//             X = diag(beta) (V - diag(gamma) K S),  U = T X
+//             P = tril(Q K^T) * Gamma,  O = diag(gamma) Q S + P U
+//             S+ = gamma_n S + (diag(e^(g_n - g)) K)^T U
+//   reverse   dU  = P^T dO + diag(e^(g_n - g)) K dS+
+//             dP  = tril(dO U^T)                       dBV = T^T dU
+//             dT  = dU X^T,  dA = -strict_lower(T^T dT T^T)
+//             dq  = diag(gamma) dO S^T + (dP * Gamma) K
+//             dk  = (dP * Gamma)^T Q + diag(e^(g_n - g)) U dS+^T - diag(beta gamma) dBV S^T
+//                   + (dMA * Gamma) K + (dMA * Gamma)^T K,    dMA = diag(beta) dA
+//             dv  = diag(beta) dBV
+//             dbeta = rowsum(dBV * V) - gamma * rowsum(dBV * KS) + rowsum(dA * MA)
+//             dS  = (diag(gamma) Q)^T dO + gamma_n dS+ - K^T diag(beta gamma) dBV
+//   and the gradient of g (rows and columns of every Gamma-weighted product,
+//   gamma_r on the read of S, the S+ carry) summed from the last row gives the
+//   gradient of log alpha.
+//
+// One CTA per (b, h, 64-column slice of Dv), 256 threads, C = 32 (the
+// backward's own chunk; the result does not depend on it).  A forward sweep
+// stores every chunk's entry state (float32) in the workspace, then the reverse
+// sweep walks the chunks from the last.  The forward and the dv, dS0 outputs
+// are separable over the columns of v; dq, dk, dbeta and dlog_alpha are sums
+// over all columns, so each slice adds its part with one atomicAdd per element
+// onto outputs cleared first: with at most two slices (Dv <= 128) the sum is
+// the same in either order, so the result is deterministic.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+
+namespace dn {
+namespace {
+
+constexpr int kThreads = 256, kWarps = kThreads / 32;
+constexpr int C = 32, DVS = 64, VP = DVS + 1, CP = C + 1;
+
+template <typename TI>
+__device__ __forceinline__ float ld(const TI* p, size_t i);
+template <>
+__device__ __forceinline__ float ld<float>(const float* p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+template <int DK>
+struct BwdSmem {
+  static constexpr int KP = DK + 1;
+  static constexpr int kFloats = 2 * C * KP      // Q, K
+                                 + 2 * DK * VP   // S, dS
+                                 + 7 * C * VP    // V, dO, KS, X, U, dU, dBV
+                                 + 3 * C * CP    // T, M1, M2
+                                 + 8 * C;        // beta, g, gamma, e_out, dg, dbeta, red, spare
+  static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <typename TI, bool GATED, int DK>
+__global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p) {
+  using L = BwdSmem<DK>;
+  constexpr int KP = L::KP;
+  extern __shared__ float sm[];
+  float* Qs = sm;
+  float* Ks = Qs + C * KP;
+  float* Ss = Ks + C * KP;
+  float* dSs = Ss + DK * VP;
+  float* Vs = dSs + DK * VP;
+  float* dOs = Vs + C * VP;
+  float* KSs = dOs + C * VP;
+  float* Xs = KSs + C * VP;
+  float* Us = Xs + C * VP;
+  float* dUs = Us + C * VP;
+  float* dBVs = dUs + C * VP;
+  float* Ts = dBVs + C * VP;
+  float* M1 = Ts + C * CP;
+  float* M2 = M1 + C * CP;
+  float* bs = M2 + C * CP;
+  float* gs = bs + C;
+  float* gam = gs + C;
+  float* eo = gam + C;
+  float* dg = eo + C;
+  float* db = dg + C;
+  float* red = db + C;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x, slice = blockIdx.y, j0 = slice * DVS;
+  const int T = p.T, Dv = p.Dv, nch = (T + C - 1) / C;
+  const TI* q = static_cast<const TI*>(p.q);
+  const TI* k = static_cast<const TI*>(p.k);
+  const TI* v = static_cast<const TI*>(p.v);
+  const TI* dO = static_cast<const TI*>(p.dO);
+  const size_t qk_base = (size_t)bh * T * DK, v_base = (size_t)bh * T * Dv;
+  const size_t s_base = (size_t)bh * DK * Dv;
+  // entry states of this (b, h, slice): nch x DK x DVS floats
+  float* states = p.states + ((size_t)bh * gridDim.y + slice) * (size_t)nch * DK * DVS;
+
+  auto gamma_rs = [&](int r, int s) { return GATED ? __expf(gs[r] - gs[s]) : 1.f; };
+
+  // Stage chunk c: Q, K, V (slice), dO (slice), beta, g (rows past n: zero
+  // inputs, beta 0, log alpha 0 so g stays flat), gamma, e^(g_last - g).
+  auto stage = [&](int c, bool with_q) {
+    const int c0 = c * C, n = min(C, T - c0);
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      const size_t at = qk_base + (size_t)(c0 + r) * DK + i;
+      Ks[r * KP + i] = r < n ? ld(k, at) : 0.f;
+      if (with_q) Qs[r * KP + i] = r < n ? ld(q, at) : 0.f;
+    }
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      const size_t at = v_base + (size_t)(c0 + r) * Dv + j0 + j;
+      Vs[r * VP + j] = r < n ? ld(v, at) : 0.f;
+      if (with_q) dOs[r * VP + j] = r < n ? ld(dO, at) : 0.f;
+    }
+    if (warp == 0) {  // one lane per row: beta and the inclusive scan of log alpha
+      const int r = lane;
+      bs[r] = r < n ? p.beta[(size_t)bh * T + c0 + r] : 0.f;
+      float la = 0.f;
+      if (GATED && r < n) la = fmaxf(__logf(p.alpha[(size_t)bh * T + c0 + r]), -87.f);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, la, off);
+        if (lane >= off) la += y;
+      }
+      gs[r] = la;
+      const float glast = __shfl_sync(0xffffffffu, la, 31);
+      gam[r] = GATED ? __expf(la) : 1.f;
+      eo[r] = GATED ? __expf(glast - la) : 1.f;
+    }
+  };
+
+  // T = (I + A)^-1 with A = strict_lower(diag(beta) (K K^T * Gamma)): A into
+  // M1, then forward substitution, one column per thread of warp 0.
+  auto solve_T = [&]() {
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s < r) {
+        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
+        acc *= bs[r] * gamma_rs(r, s);
+      }
+      M1[r * CP + s] = acc;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int j = lane;
+      for (int i = 0; i < C; ++i) {
+        float t;
+        if (i < j) {
+          t = 0.f;
+        } else if (i == j) {
+          t = 1.f;
+        } else {
+          float acc = 0.f;
+          for (int m = j; m < i; ++m) acc += M1[i * CP + m] * Ts[m * CP + j];
+          t = -acc;
+        }
+        Ts[i * CP + j] = t;
+      }
+    }
+    __syncthreads();
+  };
+
+  // KS = K S, X = diag(beta) (V - diag(gamma) K S), U = T X
+  auto forward_u = [&]() {
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ss[i * VP + j];
+      KSs[r * VP + j] = acc;
+      Xs[r * VP + j] = bs[r] * (Vs[r * VP + j] - gam[r] * acc);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int s = 0; s <= r; ++s) acc += Ts[r * CP + s] * Xs[s * VP + j];
+      Us[r * VP + j] = acc;
+    }
+    __syncthreads();
+  };
+
+  // ---------------------------------------------------------- forward sweep --
+  for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+    const int i = idx / DVS, j = idx % DVS;
+    Ss[i * VP + j] = p.S0 ? p.S0[s_base + (size_t)i * Dv + j0 + j] : 0.f;
+  }
+  for (int c = 0; c < nch; ++c) {
+    __syncthreads();
+    stage(c, false);
+    for (int idx = tid; idx < DK * DVS; idx += kThreads)
+      states[(size_t)c * DK * DVS + idx] = Ss[(idx / DVS) * VP + idx % DVS];
+    __syncthreads();
+    solve_T();
+    forward_u();
+    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+      const int i = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int s = 0; s < C; ++s) acc += eo[s] * Ks[s * KP + i] * Us[s * VP + j];
+      Ss[i * VP + j] = gam[C - 1] * Ss[i * VP + j] + acc;
+    }
+  }
+
+  // ---------------------------------------------------------- reverse sweep --
+  __syncthreads();
+  for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+    const int i = idx / DVS, j = idx % DVS;
+    dSs[i * VP + j] = p.dS_T ? p.dS_T[s_base + (size_t)i * Dv + j0 + j] : 0.f;
+  }
+  for (int c = nch - 1; c >= 0; --c) {
+    const int c0 = c * C, n = min(C, T - c0);
+    __syncthreads();
+    stage(c, true);
+    for (int idx = tid; idx < DK * DVS; idx += kThreads)
+      Ss[(idx / DVS) * VP + idx % DVS] = states[(size_t)c * DK * DVS + idx];
+    __syncthreads();
+    solve_T();
+    forward_u();
+    // P = tril(Q K^T) * Gamma into M1
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s <= r) {
+        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ks[s * KP + i];
+        acc *= gamma_rs(r, s);
+      }
+      M1[r * CP + s] = acc;
+    }
+    __syncthreads();
+    // dU = P^T dO + diag(e_out) K dS+
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int t = r; t < C; ++t) acc += M1[t * CP + r] * dOs[t * VP + j];
+      float ks = 0.f;
+      for (int i = 0; i < DK; ++i) ks += Ks[r * KP + i] * dSs[i * VP + j];
+      dUs[r * VP + j] = acc + eo[r] * ks;
+    }
+    __syncthreads();
+    // dP = tril(dO U^T) into M2;  dBV = T^T dU
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s <= r)
+        for (int j = 0; j < DVS; ++j) acc += dOs[r * VP + j] * Us[s * VP + j];
+      M2[r * CP + s] = acc;
+    }
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      float acc = 0.f;
+      for (int a = r; a < C; ++a) acc += Ts[a * CP + r] * dUs[a * VP + j];
+      dBVs[r * VP + j] = acc;
+    }
+    __syncthreads();
+    // Per-row sums, one warp per row (lanes over the slice's columns):
+    //   dg_r  = gamma_r sum_j dO (Q S) - beta_r gamma_r sum_j dBV KS - c_out_r
+    //   db_r  = sum_j dBV V - gamma_r sum_j dBV KS
+    //   c_out_r = e_out_r sum_j U (K dS+)        (the S+ carry's decay)
+    for (int r = warp; r < C; r += kWarps) {
+      float t_qs = 0.f, t_bk = 0.f, t_bv = 0.f, t_co = 0.f;
+      for (int j = lane; j < DVS; j += 32) {
+        float qs = 0.f, kd = 0.f;
+        for (int i = 0; i < DK; ++i) {
+          qs += Qs[r * KP + i] * Ss[i * VP + j];
+          kd += Ks[r * KP + i] * dSs[i * VP + j];
+        }
+        t_qs += dOs[r * VP + j] * qs;
+        t_bk += dBVs[r * VP + j] * KSs[r * VP + j];
+        t_bv += dBVs[r * VP + j] * Vs[r * VP + j];
+        t_co += Us[r * VP + j] * kd;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        t_qs += __shfl_xor_sync(0xffffffffu, t_qs, off);
+        t_bk += __shfl_xor_sync(0xffffffffu, t_bk, off);
+        t_bv += __shfl_xor_sync(0xffffffffu, t_bv, off);
+        t_co += __shfl_xor_sync(0xffffffffu, t_co, off);
+      }
+      if (lane == 0) {
+        const float co = eo[r] * t_co;
+        dg[r] = gam[r] * t_qs - bs[r] * gam[r] * t_bk - co;
+        db[r] = t_bv - gam[r] * t_bk;
+        red[r] = co;
+      }
+    }
+    // the carry gamma_n S: sum over the slice of dS+ * S (block reduction)
+    {
+      float acc = 0.f;
+      for (int idx = tid; idx < DK * DVS; idx += kThreads)
+        acc += dSs[(idx / DVS) * VP + idx % DVS] * Ss[(idx / DVS) * VP + idx % DVS];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      __syncthreads();  // red[] of the row sums is written
+      __shared__ float wsum[kWarps];
+      if (lane == 0) wsum[warp] = acc;
+      __syncthreads();
+      if (tid == 0) {
+        float tot = 0.f, co = 0.f;
+        for (int w = 0; w < kWarps; ++w) tot += wsum[w];
+        for (int r = 0; r < C; ++r) co += red[r];
+        dg[C - 1] += gam[C - 1] * tot + co;
+      }
+    }
+    __syncthreads();
+    // the rows and columns of P's decay: dg += rowsum(dP * P) - colsum(dP * P)
+    if (GATED && tid < C) {
+      const int r = tid;
+      float acc = 0.f;
+      for (int s = 0; s < C; ++s) acc += M2[r * CP + s] * M1[r * CP + s] - M2[s * CP + r] * M1[s * CP + r];
+      dg[r] += acc;
+    }
+    // dq = diag(gamma) dO S^T + (dP * Gamma) K
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      if (r >= n) continue;
+      float a = 0.f, b = 0.f;
+      for (int j = 0; j < DVS; ++j) a += dOs[r * VP + j] * Ss[i * VP + j];
+      for (int s = 0; s <= r; ++s) b += M2[r * CP + s] * gamma_rs(r, s) * Ks[s * KP + i];
+      atomicAdd(p.dq + qk_base + (size_t)(c0 + r) * DK + i, gam[r] * a + b);
+    }
+    __syncthreads();
+    // dT = dU X^T (strictly lower part: only it reaches dA), into M1
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float acc = 0.f;
+      if (s < r)
+        for (int j = 0; j < DVS; ++j) acc += dUs[r * VP + j] * Xs[s * VP + j];
+      M1[r * CP + s] = acc;
+    }
+    __syncthreads();
+    // Y = dT T^T, row by row in place (row a of Y needs only row a of dT)
+    for (int a = warp; a < C; a += kWarps) {
+      const float d = M1[a * CP + lane];
+      __syncwarp();
+      float y = 0.f;
+      for (int b = 0; b < C; ++b) y += __shfl_sync(0xffffffffu, d, b) * Ts[lane * CP + b];
+      M1[a * CP + lane] = y;
+    }
+    __syncthreads();
+    // dA = -strict_lower(T^T Y), column by column in place (column s of dA
+    // needs only column s of Y)
+    for (int s = warp; s < C; s += kWarps) {
+      const float y = M1[lane * CP + s];
+      __syncwarp();
+      float acc = 0.f;
+      for (int a = 0; a < C; ++a) acc += Ts[a * CP + lane] * __shfl_sync(0xffffffffu, y, a);
+      M1[lane * CP + s] = lane > s ? -acc : 0.f;
+    }
+    __syncthreads();
+    // E = dA * MA into Ts (T is no longer needed), MA = K K^T * Gamma
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      float e = 0.f;
+      if (s < r) {
+        float kk = 0.f;
+        for (int i = 0; i < DK; ++i) kk += Ks[r * KP + i] * Ks[s * KP + i];
+        e = M1[r * CP + s] * kk * gamma_rs(r, s);
+      }
+      Ts[r * CP + s] = e;
+    }
+    __syncthreads();
+    // dbeta += rowsum(dA * MA);  dg += beta_r rowsum(E) - sum_t beta_t E[t][r];
+    // then dMA = diag(beta) dA in place
+    if (tid < C) {
+      const int r = tid;
+      float rs = 0.f, cs = 0.f;
+      for (int s = 0; s < C; ++s) {
+        rs += Ts[r * CP + s];
+        cs += bs[s] * Ts[s * CP + r];
+      }
+      db[r] += rs;
+      if (GATED) dg[r] += bs[r] * rs - cs;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s = idx % C;
+      M1[r * CP + s] *= bs[r];
+    }
+    __syncthreads();
+    // dk = (dP * Gamma)^T Q + diag(e_out) U dS+^T - diag(beta gamma) dBV S^T
+    //      + (dMA * Gamma) K + (dMA * Gamma)^T K
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int s = idx / DK, i = idx % DK;
+      if (s >= n) continue;
+      float a = 0.f, u = 0.f, bv = 0.f, m = 0.f;
+      for (int r = s; r < C; ++r) a += M2[r * CP + s] * gamma_rs(r, s) * Qs[r * KP + i];
+      for (int j = 0; j < DVS; ++j) {
+        u += Us[s * VP + j] * dSs[i * VP + j];
+        bv += dBVs[s * VP + j] * Ss[i * VP + j];
+      }
+      for (int t = 0; t < s; ++t) m += M1[s * CP + t] * gamma_rs(s, t) * Ks[t * KP + i];
+      for (int r = s + 1; r < C; ++r) m += M1[r * CP + s] * gamma_rs(r, s) * Ks[r * KP + i];
+      atomicAdd(p.dk + qk_base + (size_t)(c0 + s) * DK + i,
+                a + eo[s] * u - bs[s] * gam[s] * bv + m);
+    }
+    // dv = diag(beta) dBV (this slice's columns: a plain store)
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      if (r < n) p.dv[v_base + (size_t)(c0 + r) * Dv + j0 + j] = bs[r] * dBVs[r * VP + j];
+    }
+    // dbeta and d(log alpha) = sum of dg over rows >= r within the chunk
+    if (warp == 0) {
+      const int r = lane;
+      float x = GATED ? dg[C - 1 - r] : 0.f;  // reverse inclusive scan
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      const int row = C - 1 - r;
+      if (row < n) {
+        atomicAdd(p.dbeta + (size_t)bh * T + c0 + row, db[row]);
+        if (GATED && p.dlog_alpha) atomicAdd(p.dlog_alpha + (size_t)bh * T + c0 + row, x);
+      }
+    }
+    __syncthreads();
+    // dS = (diag(gamma) Q)^T dO + gamma_n dS+ - K^T diag(beta gamma) dBV, in place
+    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+      const int i = idx / DVS, j = idx % DVS;
+      float acc = gam[C - 1] * dSs[i * VP + j];
+      for (int r = 0; r < C; ++r)
+        acc += gam[r] * (Qs[r * KP + i] * dOs[r * VP + j] - bs[r] * Ks[r * KP + i] * dBVs[r * VP + j]);
+      dSs[i * VP + j] = acc;
+    }
+  }
+  __syncthreads();
+  if (p.dS0)
+    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
+      const int i = idx / DVS, j = idx % DVS;
+      p.dS0[s_base + (size_t)i * Dv + j0 + j] = dSs[i * VP + j];
+    }
+}
+
+template <typename TI, bool GATED, int DK>
+cudaError_t launch_one(const BwdProblem& p, cudaStream_t st) {
+  using L = BwdSmem<DK>;
+  auto kern = chunk_bwd_kernel<TI, GATED, DK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((unsigned)(p.B * p.H), (unsigned)(p.Dv / DVS)), kThreads, L::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t launch_dt(const BwdProblem& p, cudaStream_t st) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_one<TI, true, 128>(p, st) : launch_one<TI, false, 128>(p, st);
+  return gated ? launch_one<TI, true, 64>(p, st) : launch_one<TI, false, 64>(p, st);
+}
+
+}  // namespace
+
+size_t chunk_bwd_state_bytes(int B, int H, int T, int Dk, int Dv) {
+  const size_t nch = ((size_t)T + C - 1) / C;
+  return (size_t)B * H * nch * Dk * Dv * sizeof(float);
+}
+
+cudaError_t launch_chunk_bwd(const BwdProblem& p, cudaStream_t st) {
+  const size_t BH = (size_t)p.B * p.H, T = (size_t)p.T;
+  // the slices add their parts of these onto zeros
+  cudaError_t e = cudaMemsetAsync(p.dq, 0, BH * T * p.Dk * sizeof(float), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p.dk, 0, BH * T * p.Dk * sizeof(float), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p.dbeta, 0, BH * T * sizeof(float), st);
+  if (e == cudaSuccess && p.dlog_alpha) e = cudaMemsetAsync(p.dlog_alpha, 0, BH * T * sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  return p.bf16 ? launch_dt<__nv_bfloat16>(p, st) : launch_dt<float>(p, st);
+}
+
+}  // namespace dn

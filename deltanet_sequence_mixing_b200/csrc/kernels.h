@@ -84,6 +84,29 @@ cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaS
 bool chunk128_supported(const ChunkProblem& p);
 cudaError_t launch_chunk128(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 
+// Gradient of the chunked delta rule (float32 arithmetic on CUDA cores).
+struct BwdProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  const float* alpha;   // nullable (ungated)
+  const float* S0;      // nullable
+  const void* dO;       // (B,H,T,Dv), element type of q
+  const float* dS_T;    // nullable
+  float* dq;            // (B,H,T,Dk)
+  float* dk;
+  float* dv;            // (B,H,T,Dv)
+  float* dbeta;         // (B,H,T)
+  float* dlog_alpha;    // (B,H,T), nullable
+  float* dS0;           // (B,H,Dk,Dv), nullable
+  float* states;        // workspace: entry state of every 32-token chunk
+  int B, H, T, Dk, Dv;
+  int bf16;
+};
+size_t chunk_bwd_state_bytes(int B, int H, int T, int Dk, int Dv);
+cudaError_t launch_chunk_bwd(const BwdProblem& p, cudaStream_t st);
+
 // Bounded-wait self test.
 cudaError_t launch_wait_selftest(unsigned int* status, long long wait_ns, cudaStream_t st);
 

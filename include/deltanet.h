@@ -217,6 +217,42 @@ int linear_attn_fwd(const void *q, const void *k, const void *v,
                     void *workspace, size_t ws_bytes, void *cuda_stream);
 
 /*
+ * Bytes of device workspace deltanet_chunk_bwd needs: the 256-byte status word
+ * plus the float32 entry state of every 32-token chunk of every (b, h)
+ * (B * H * ceil(T / 32) * Dk * Dv * 4 bytes).  0 for sizes it rejects.
+ */
+size_t deltanet_chunk_bwd_workspace_bytes(int B, int H, int T, int Dk, int Dv, dn_dtype dt);
+
+/*
+ * Gradient of deltanet_chunk_fwd (the backward of a training step).
+ *
+ * [P3] "DeltaNet (Parallelizing linear transformers with delta rule)" gives
+ * the chunkwise form as what makes linear-time training hardware-efficient;
+ * this call runs the reverse of that form.  For the loss
+ *     L = sum(dO * o) + sum(dS_T * S_T)
+ * of the forward with the same q, k, v, beta, alpha, S0, it writes
+ *     dq, dk  (B,H,T,Dk) float32      dv (B,H,T,Dv) float32
+ *     dbeta   (B,H,T) float32         dlog_alpha (B,H,T) float32 = alpha * dL/dalpha
+ *     dS0     (B,H,Dk,Dv) float32 (nullable)
+ * dO has the shape and element type of o; dS_T is (B,H,Dk,Dv) float32 or NULL
+ * (zero).  dlog_alpha may be NULL; it must be NULL when alpha is NULL.  The
+ * decay enters through log(max(alpha, e^-87)), as in the forward.
+ * Inputs as deltanet_chunk_fwd (Dk, Dv in {64, 128}, bf16 or f32, any T >= 0;
+ * T = 0 copies dS_T, or zeros, to dS0); the float32 buffers need 4-byte
+ * alignment; no output may overlap an input or another output.  Arithmetic is
+ * float32 on CUDA cores: a forward sweep stores the chunk entry states in the
+ * workspace, then a reverse sweep forms the gradients chunk by chunk.  The
+ * result is deterministic.
+ */
+int deltanet_chunk_bwd(const void *q, const void *k, const void *v,
+                       const float *beta, const float *alpha, const float *S0,
+                       const void *dO, const float *dS_T,
+                       float *dq, float *dk, float *dv, float *dbeta, float *dlog_alpha,
+                       float *dS0,
+                       int B, int H, int T, int Dk, int Dv, dn_dtype dt,
+                       void *workspace, size_t ws_bytes, void *cuda_stream);
+
+/*
  * Synchronise `cuda_stream` and read the sticky device status word of
  * `workspace`: DN_OK, or DN_ERR_DEVICE_TIMEOUT if any earlier kernel given
  * this workspace ran out of a bounded wait (results of that call are then
