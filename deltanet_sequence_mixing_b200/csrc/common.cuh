@@ -182,6 +182,19 @@ __device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t ades
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] x B[smem] (the A operand in tensor memory: row m of A on
+// TMEM lane m, 32-bit column c holding elements 2c (low half) and 2c + 1 (high
+// half); one K = 16 step spans 8 columns), issued by one elected lane.  Only B
+// is read from shared memory, which halves (N = 128) or thirds (N = 64) the
+// shared-memory traffic of the product.
+__device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred e, p; .reg .b32 x; elect.sync x|e, 0xffffffff; setp.ne.b32 p, %4, 0;"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Commit from one elected lane of a warp-uniform issuer (see mma_bf16_ss_elect).
 __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
   asm volatile(
