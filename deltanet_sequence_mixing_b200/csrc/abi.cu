@@ -109,10 +109,11 @@ int validate_chunked(const dn::ChunkProblem& p, size_t ws_bytes, const void* ws,
 // Launch the kernels of a validated chunked problem; `status` is the device
 // status word, `wy` the start of the pre-pass factor region.
 // Problems the tcgen05 chunk kernels take: the plain and scalar-gated delta rule
-// on bf16 inputs, without the pre-step; the pre-step and the per-dimension gate
-// run on the CUDA-core kernel (C = 64).
+// on bf16 inputs, with the layer's pre-step at C = 64; the per-dimension gate
+// (and float32 inputs) run on the CUDA-core kernel (C = 64).
 bool tensor_core_path(const dn::ChunkProblem& p) {
-  return !p.prestep && !p.alpha_per_dim && (dn::chunk_main_supported(p) || dn::chunk128_supported(p));
+  if (p.alpha_per_dim) return false;
+  return dn::chunk_main_supported(p) || (!p.prestep && dn::chunk128_supported(p));
 }
 
 int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStream_t st) {
@@ -214,8 +215,11 @@ size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, d
                                    unsigned int options) {
   if (options & ~kKnownOptions) return 0;
   if (options == 0) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);
-  // the options run on the CUDA-core kernel: C = 64, status word only
   if (C != 64 || deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt) == 0) return 0;
+  // the pre-step alone runs on the tcgen05 path for bf16 (the per-chunk factors
+  // of the pre-pass); the per-dimension gate runs on the CUDA-core kernel
+  // (status word only)
+  if (options == DN_OPT_PRESTEP) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);
   return kStatusBytes;
 }
 

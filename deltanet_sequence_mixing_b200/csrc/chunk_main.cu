@@ -100,7 +100,7 @@ struct MainLayout {
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
                    B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168,
-                   B_QREADY = 176;
+                   B_QREADY = 176, B_LANDED = 192;  // LANDED: one per ring stage (pre-step only)
 
 // Pack 32 floats into 16 32-bit words of bf16 pairs (element 2i in the low half).
 __device__ __forceinline__ void pack16(const float* x, uint32_t* w) {
@@ -131,7 +131,7 @@ __device__ __forceinline__ void u_epilogue_half(uint32_t ws_addr, uint32_t uh_ad
   }
 }
 
-template <int DK, bool GATED>
+template <int DK, bool GATED, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
@@ -157,8 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
-      mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's arrival (after the g rows)
+      // TMA bytes + the producer's arrival (after the g rows); with the pre-step
+      // the bytes land on LANDED and the producer arrives once K is mapped
+      mbar_init(bar + B_FULL + 8 * i, PRE ? 1 : 2);
       mbar_init(bar + B_EMPTY + 8 * i, 1);
+      if (PRE) mbar_init(bar + B_LANDED + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + B_OFREE + 8 * i, 1);
@@ -201,7 +204,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Tb, Tbg and g come from the pre-pass launched just before this kernel
     grid_dependency_wait();
-    int issued = 0;
+    int issued = 0, finished = 0;
+    // Pre-step: once chunk c's tiles have landed, map K in place (two lanes per
+    // row, the pre-pass's split, so both kernels see identical bf16 keys) and
+    // release the stage to the consumers.
+    auto finish = [&](int c) {
+      const int s = c % NST;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar + B_LANDED + 8 * s, (c / NST) & 1, wc))) return false;
+      uint8_t* kt = sm + s * L::STAGE + L::K_OFF;
+#pragma unroll 1
+      for (int rr = 0; rr < kC / 16; ++rr) prestep_row_sw128<DK>(kt, L::KB_STRIDE, rr * 16 + (lane >> 1), lane & 1);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + B_FULL + 8 * s);
+      finished = c + 1;
+      return true;
+    };
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % NST, use = c / NST;
       const int c0 = c * kC, n = min(kC, T - c0);
@@ -209,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && use > 0) ok = mbar_wait(bar + B_EMPTY + 8 * s, (use - 1) & 1, wc);
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
       const uint32_t st = sb + s * L::STAGE;
-      const uint32_t full = bar + B_FULL + 8 * s;
+      const uint32_t full = bar + (PRE ? B_LANDED : B_FULL) + 8 * s;
       if (lane == 0) {
         mbar_expect_tx(full, tile_bytes);
 #pragma unroll
@@ -228,8 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       (void)n;
       __syncwarp();
+      if (!PRE && lane == 0) mbar_arrive(full);
+      if (PRE && c > 0 && !finish(c - 1)) {
+        issued = c + 1;
+        break;
+      }
       if (lane == 0) {
-        mbar_arrive(full);
         if (c + 2 < nchunks) {  // warm L2 for the chunk after next
           const int cn = c0 + 2 * kC;
 #pragma unroll
@@ -249,11 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       issued = c + 1;
     }
+    if (PRE && issued == nchunks && finished == nchunks - 1) (void)finish(nchunks - 1);
     if (lane == 0) {  // never leave with copies in flight
       int zero = 0;
       const WaitCtl drain{&zero, p.status, kWaitLimitNs};
       for (int c = issued > NST ? issued - NST : 0; c < issued; ++c)
-        (void)mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, drain);
+        (void)mbar_wait(bar + (PRE ? B_LANDED : B_FULL) + 8 * (c % NST), (c / NST) & 1, drain);
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- issuer --
@@ -452,13 +475,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (c == 0 || mbar_wait(bar + B_CMMA3, (c - 1) & 1, wc)));
       if (!ok) break;
       tc_fence_after();
+      float qinv = 1.f;
+      if (PRE) {  // the layer's pre-step on q: silu, then 1 / max(||silu(q)||, 1e-12)
+        float ss = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            float x[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(stp + kb * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16)), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float y = silu_f(x[e]);
+              ss = fmaf(y, y, ss);
+            }
+          }
+        qinv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+      }
 #pragma unroll
       for (int kb = 0; kb < DK / 64; ++kb) {
         const uint8_t* qt = stp + kb * L::KB_STRIDE + L::Q_OFF;
         uint32_t pk[32];
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {
-          const uint4 u = *reinterpret_cast<const uint4*>(qt + sw128_off(row, c16));
+          uint4 u = *reinterpret_cast<const uint4*>(qt + sw128_off(row, c16));
+          if (PRE) {
+            float x[8];
+            unpack_bf16x8(u, x);
+            u.x = pack2_bf16(silu_f(x[0]) * qinv, silu_f(x[1]) * qinv);
+            u.y = pack2_bf16(silu_f(x[2]) * qinv, silu_f(x[3]) * qinv);
+            u.z = pack2_bf16(silu_f(x[4]) * qinv, silu_f(x[5]) * qinv);
+            u.w = pack2_bf16(silu_f(x[6]) * qinv, silu_f(x[7]) * qinv);
+          }
           pk[4 * c16] = u.x;
           pk[4 * c16 + 1] = u.y;
           pk[4 * c16 + 2] = u.z;
@@ -647,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, bool GATED>
+template <int DK, bool GATED, bool PRE>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   using L = MainLayout<DK, GATED>;
   const int BH = p.B * p.H;
@@ -660,7 +708,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
       !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
       !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))
     return cudaErrorInvalidValue;
-  auto kern = chunk_main_kernel<DK, GATED>;
+  auto kern = chunk_main_kernel<DK, GATED, PRE>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
@@ -686,10 +734,15 @@ bool chunk_main_supported(const ChunkProblem& p) {
          (p.Dv == 64 || p.Dv == 128);
 }
 
-cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+template <bool PRE>
+cudaError_t launch_pre(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   const bool gated = p.alpha != nullptr;
-  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
-  return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
+  if (p.Dk == 128) return gated ? launch_t<128, true, PRE>(p, w, st) : launch_t<128, false, PRE>(p, w, st);
+  return gated ? launch_t<64, true, PRE>(p, w, st) : launch_t<64, false, PRE>(p, w, st);
+}
+
+cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  return p.prestep ? launch_pre<true>(p, w, st) : launch_pre<false>(p, w, st);
 }
 
 }  // namespace dn

@@ -322,4 +322,55 @@ __device__ __forceinline__ void st_bf16x8(void* dst, const float* x) {
   *reinterpret_cast<uint4*>(dst) = u;
 }
 
+// ------------------------------------------------- the layer's pre-step --
+// silu(x) = x sigmoid(x)
+__device__ __forceinline__ float silu_f(float x) { return x / (1.f + __expf(-x)); }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* x) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// The DeltaNet layer's map x <- silu(x) / max(||silu(x)||_2, 1e-12) on one row
+// of a K-major, 128-byte-swizzled bf16 tile in shared memory (DK columns in
+// 64-column blocks `blk_stride` bytes apart), in place.  Two adjacent lanes
+// share a row: lane parity `part` takes the 16-byte chunks [part * DK/16,
+// (part + 1) * DK/16) and the two partial sums of squares are combined with
+// one shuffle, so every kernel that maps the same row gets bit-identical bf16
+// values (the sum is always (first half) + (second half)).  All 32 lanes of
+// the warp must call it.
+template <int DK>
+__device__ __forceinline__ void prestep_row_sw128(uint8_t* tile, uint32_t blk_stride, int row, int part) {
+  constexpr int NCH = DK / 16;  // 16-byte chunks per thread
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    const int cg = part * NCH + j, blk = cg >> 3, c16 = cg & 7;
+    float x[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(tile + blk * blk_stride + sw128_off(row, c16)), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float y = silu_f(x[e]);
+      ss = fmaf(y, y, ss);
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, ss, 1);
+  const float tot = part == 0 ? ss + other : other + ss;
+  const float inv = 1.f / fmaxf(sqrtf(tot), 1e-12f);
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    const int cg = part * NCH + j, blk = cg >> 3, c16 = cg & 7;
+    uint4* at = reinterpret_cast<uint4*>(tile + blk * blk_stride + sw128_off(row, c16));
+    float x[8];
+    unpack_bf16x8(*at, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = silu_f(x[e]) * inv;
+    st_bf16x8(at, x);
+  }
+}
+
 }  // namespace dn

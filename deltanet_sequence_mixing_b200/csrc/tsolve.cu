@@ -74,7 +74,7 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
   for (int t = 0; t < f.num_elements; ++t) f.x[t] = __uint_as_float(__float_as_uint(f.x[t]) & 0xFFFFE000u);
 }
 
-template <int C, int DK, bool GATED>
+template <int C, int DK, bool GATED, bool PRE>
 __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
                   const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
   float glog = 0.f;
   if (tid < kC) {
     const size_t tb = (size_t)bh * T + c0;
-    vb[tid] = tid < n ? beta[tb + tid] : 0.f;
+    float b = tid < n ? beta[tb + tid] : 0.f;
+    if (PRE && tid < n) b = 1.f / (1.f + __expf(-b));  // beta holds logits
+    vb[tid] = b;
     if (GATED) {  // inclusive scan of max(log alpha, -87) within each warp
       glog = tid < n ? fmaxf(__logf(alpha[tb + tid]), -87.f) : 0.f;
 #pragma unroll
@@ -143,11 +145,19 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
       if (lane == 31) wsum[warp] = glog;
     }
   }
+  bool ok = true;
+  if (PRE) {
+    // The layer's pre-step on K in shared memory (two threads per row, the
+    // same split as the chunk kernel's, so both see identical bf16 keys).
+    ok = __all_sync(0xffffffffu, mbar_wait(bar_full, 0, wc));  // warp-uniform for the shuffles
+    if (ok) prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, tid >> 1, tid & 1);
+    fence_proxy_async_smem();
+    ok = __syncthreads_and(ok);
+  }
   // 2. G = K K^T on the tensor cores (M = 128, N = C, into TMEM), issued by one
   //    elected lane of warp 0 once the tile has landed.
-  bool ok = true;
   if (warp == 0) {
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_full, 0, wc));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_full, 0, wc));
     if (!ok && lane == 0) {  // never leave with the copy in flight
       int zero = 0;
       const WaitCtl drain{&zero, status, kWaitLimitNs};
@@ -405,7 +415,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   constexpr size_t smem = TsolveSmem<C, DK>::ALLOC;
   CUtensorMap mk;
   if (!make_tmap_3d_bf16(&mk, p.k, DK, p.T, p.B * p.H)) return cudaErrorInvalidValue;
-  auto kern = tsolve_kernel<C, DK, GATED>;
+  auto kern = p.prestep ? tsolve_kernel<C, DK, GATED, true> : tsolve_kernel<C, DK, GATED, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((size_t)nchunks * p.B * p.H));  // at most INT_MAX (checked by the caller)

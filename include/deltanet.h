@@ -130,10 +130,14 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   decays by alpha_t[i] before the delta write ([P1], the KDA paragraph:
  *   scalar gating replaced by per-dimension gating).  alpha must not be NULL.
  *
- * Paths: with either option the chunked call runs on the CUDA-core kernel
- * (float32 arithmetic, bf16 or f32 inputs, C = 64 only; C = 128 gives
- * DN_ERR_UNSUPPORTED) and needs only the 256-byte status word as workspace;
- * the decode step takes both options on its usual kernel.  Unknown bits give
+ * Paths: the options are built for C = 64 (C = 128 gives DN_ERR_UNSUPPORTED).
+ * DN_OPT_PRESTEP alone on bf16 inputs runs on the tcgen05 path (the maps are
+ * applied to the q and k tiles in shared memory, K identically in the pre-pass
+ * and the chunk kernel) with the workspace of deltanet_workspace_bytes; every
+ * other combination (per-dimension decay, float32 inputs) runs on the
+ * CUDA-core kernel (float32 arithmetic) and needs only the 256-byte status
+ * word.  deltanet_workspace_bytes_ex gives the size for each case.  The
+ * decode step takes both options on its usual kernel.  Unknown bits give
  * DN_ERR_INVALID_ARG.
  */
 enum {

@@ -240,7 +240,12 @@ def test_option_flags_are_validated_on_the_host(L):
     assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 500 * MB, C=128) == E.DN_ERR_UNSUPPORTED
     # the per-dimension alpha covers B*H*T*Dk floats: an alpha that ends inside o overlaps it
     assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 256 * MB - 2 * 2 * 100 * 64 * 4 + 64) == E.DN_ERR_INVALID_ARG
-    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 1) == 256
+    # the pre-step alone on bf16 runs on the tcgen05 path: the full workspace
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 1) == \
+        L.deltanet_workspace_bytes(2, 2, 100, 64, 64, 64, 1)
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 0, 1) == 256
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 2) == 256
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 3) == 256
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 128, 1, 1) == 0
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 8) == 0
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 0) == \
