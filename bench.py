@@ -409,6 +409,43 @@ def extras_measure(dn, gen, dev, stream, peaks):
                                "tc_frac": fl / (ms * 1e-3) / 1e12 / tc}
         del x, o, S
 
+    # the options and the backward on the prefill shape (B4 H16 T4096 D128 bf16)
+    w = gen.PREFILL
+    fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
+    x = gen.make_inputs(w.B, w.H, w.T, w.Dk, w.Dv, w.dtype, gated=False, seed=6, device=dev, raw=True)
+    o = torch.empty_like(x["v"])
+    S = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev)
+    ms = timed(lambda: dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], C=w.C, o=o, S_out=S,
+                                             prestep=True), 20)
+    out["prestep_prefill"] = {"path": "tcgen05 (layer pre-step inside the call)", "ms": ms,
+                              "tokens_per_s": w.B * w.T / (ms * 1e-3), "GBps": by / (ms * 1e-3) / 1e9,
+                              "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm}
+    del x
+    x = gen.make_inputs(w.B, w.H, w.T, w.Dk, w.Dv, w.dtype, gated=True, seed=7, device=dev,
+                        gate_per_dim=True)
+    ms = timed(lambda: dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C,
+                                             o=o, S_out=S), 3, 1)
+    by_kda = by + w.B * w.H * w.T * w.Dk * 4  # plus the per-dimension decays
+    out["kda_prefill"] = {"path": "CUDA cores, float32 (per-dimension decay)", "ms": ms,
+                          "tokens_per_s": w.B * w.T / (ms * 1e-3), "GBps": by_kda / (ms * 1e-3) / 1e9,
+                          "hbm_frac": by_kda / (ms * 1e-3) / 1e9 / hbm,
+                          "TFLOPs_fp32": fl / (ms * 1e-3) / 1e12}
+    del x
+    x = gen.make_workload(w, seed=8, device=dev)
+    dO = torch.randn(w.B, w.H, w.T, w.Dv, device=dev).to(w.dtype)
+    nb = dn.lib().deltanet_chunk_bwd_workspace_bytes(w.B, w.H, w.T, w.Dk, w.Dv, 1)
+    bws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    ms = timed(lambda: dn.deltanet_chunk_bwd(x["q"], x["k"], x["v"], x["beta"], dO, workspace=bws), 2, 1)
+    ht = w.B * w.H * w.T
+    # inputs q, k, v, dO, beta read; dq, dk, dv (float32), dbeta written; state checkpoints
+    # written and read once
+    by_bwd = ht * (3 * w.Dk + w.Dv) * 2 + ht * 4 + ht * (2 * w.Dk + w.Dv) * 4 + ht * 4 + 2 * (nb - 256)
+    out["backward_prefill"] = {"path": "CUDA cores, float32", "ms": ms,
+                               "tokens_per_s": w.B * w.T / (ms * 1e-3),
+                               "GBps": by_bwd / (ms * 1e-3) / 1e9, "hbm_frac": by_bwd / (ms * 1e-3) / 1e9 / hbm,
+                               "bytes": by_bwd}
+    del x, dO, bws, o, S
+
     # batched decode: 256 x 32 states from a 512-token prefill, then 1024 steps
     B, H, D = gen.DECODE_SEQS, gen.DECODE_HEADS, 128
     pre = gen.make_inputs(B, H, gen.DECODE_PREFILL, D, D, torch.bfloat16, seed=4, device=dev)
@@ -435,6 +472,17 @@ def extras_measure(dn, gen, dev, stream, peaks):
     out["decode"] = {"steps_per_s": 1e3 / ms, "us_per_step": ms * 1e3,
                      "GBps": by / (ms * 1e-3) / 1e9, "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm,
                      "bytes_per_step": by, "states": B * H, "steps": n}
+    # the same steps with the pre-step and a per-dimension decay (alpha (B,H,Dk) read as well)
+    a = torch.rand(B, H, D, device=dev) * 0.1 + 0.9
+    s.record(stream)
+    for t in range(n):
+        dn.deltanet_decode_step(qs[t], ks[t], vs[t], bs[t], S, alpha=a, o=o, prestep=True)
+    e.record(stream)
+    e.synchronize()
+    ms = s.elapsed_time(e) / n
+    by2 = by + B * H * D * 4
+    out["decode_prestep_kda"] = {"steps_per_s": 1e3 / ms, "us_per_step": ms * 1e3,
+                                 "GBps": by2 / (ms * 1e-3) / 1e9, "hbm_frac": by2 / (ms * 1e-3) / 1e9 / hbm}
     return out
 
 
