@@ -219,7 +219,11 @@ size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, d
   // the pre-step alone runs on the tcgen05 path for bf16 (the per-chunk factors
   // of the pre-pass); the per-dimension gate runs on the CUDA-core kernel
   // (status word only)
-  if (options == DN_OPT_PRESTEP) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);
+  if (options == DN_OPT_PRESTEP) {
+    if (dt != DN_BF16 || T == 0) return kStatusBytes;  // the CUDA-core kernel
+    const size_t wy = dn::wy_workspace_bytes(B, H, T, C);
+    return kStatusBytes + (wy + 255) / 256 * 256 + dn::wy_khat_bytes(B, H, T, Dk);  // + the mapped keys
+  }
   return kStatusBytes;
 }
 

@@ -100,7 +100,7 @@ struct MainLayout {
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
                    B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168,
-                   B_QREADY = 176, B_LANDED = 192;  // LANDED: one per ring stage (pre-step only)
+                   B_QREADY = 176;
 
 // Pack 32 floats into 16 32-bit words of bf16 pairs (element 2i in the low half).
 __device__ __forceinline__ void pack16(const float* x, uint32_t* w) {
@@ -157,11 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
-      // TMA bytes + the producer's arrival (after the g rows); with the pre-step
-      // the bytes land on LANDED and the producer arrives once K is mapped
-      mbar_init(bar + B_FULL + 8 * i, PRE ? 1 : 2);
+      mbar_init(bar + B_FULL + 8 * i, 2);  // TMA bytes + the producer's arrival (after the g rows)
       mbar_init(bar + B_EMPTY + 8 * i, 1);
-      if (PRE) mbar_init(bar + B_LANDED + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + B_OFREE + 8 * i, 1);
@@ -204,22 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Tb, Tbg and g come from the pre-pass launched just before this kernel
     grid_dependency_wait();
-    int issued = 0, finished = 0;
-    // Pre-step: once chunk c's tiles have landed, map K in place (two lanes per
-    // row, the pre-pass's split, so both kernels see identical bf16 keys) and
-    // release the stage to the consumers.
-    auto finish = [&](int c) {
-      const int s = c % NST;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar + B_LANDED + 8 * s, (c / NST) & 1, wc))) return false;
-      uint8_t* kt = sm + s * L::STAGE + L::K_OFF;
-#pragma unroll 1
-      for (int rr = 0; rr < kC / 16; ++rr) prestep_row_sw128<DK>(kt, L::KB_STRIDE, rr * 16 + (lane >> 1), lane & 1);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar + B_FULL + 8 * s);
-      finished = c + 1;
-      return true;
-    };
+    int issued = 0;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % NST, use = c / NST;
       const int c0 = c * kC, n = min(kC, T - c0);
@@ -227,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && use > 0) ok = mbar_wait(bar + B_EMPTY + 8 * s, (use - 1) & 1, wc);
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
       const uint32_t st = sb + s * L::STAGE;
-      const uint32_t full = bar + (PRE ? B_LANDED : B_FULL) + 8 * s;
+      const uint32_t full = bar + B_FULL + 8 * s;
       if (lane == 0) {
         mbar_expect_tx(full, tile_bytes);
 #pragma unroll
@@ -246,12 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       (void)n;
       __syncwarp();
-      if (!PRE && lane == 0) mbar_arrive(full);
-      if (PRE && c > 0 && !finish(c - 1)) {
-        issued = c + 1;
-        break;
-      }
       if (lane == 0) {
+        mbar_arrive(full);
         if (c + 2 < nchunks) {  // warm L2 for the chunk after next
           const int cn = c0 + 2 * kC;
 #pragma unroll
@@ -271,12 +249,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       issued = c + 1;
     }
-    if (PRE && issued == nchunks && finished == nchunks - 1) (void)finish(nchunks - 1);
     if (lane == 0) {  // never leave with copies in flight
       int zero = 0;
       const WaitCtl drain{&zero, p.status, kWaitLimitNs};
       for (int c = issued > NST ? issued - NST : 0; c < issued; ++c)
-        (void)mbar_wait(bar + (PRE ? B_LANDED : B_FULL) + 8 * (c % NST), (c / NST) & 1, drain);
+        (void)mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, drain);
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- issuer --
@@ -703,7 +680,8 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   cudaError_t e = launch_tsolve(p, w, st);
   if (e != cudaSuccess) return e;
   CUtensorMap mq, mk, mv, mtb, mtbg;
-  if (!make_tmap_3d_bf16(&mq, p.q, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, p.k, DK, p.T, BH) ||
+  // with the pre-step the keys come mapped from the pre-pass (workspace)
+  if (!make_tmap_3d_bf16(&mq, p.q, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, PRE ? w.khat : p.k, DK, p.T, BH) ||
       !make_tmap_3d_bf16(&mv, p.v, p.Dv, p.T, BH) ||
       !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
       !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))

@@ -71,8 +71,11 @@ struct WyWorkspace {
   __nv_bfloat16* tb;   // [B*H][chunks][C][C]  T diag(beta)
   __nv_bfloat16* tbg;  // [B*H][chunks][C][C]  T diag(beta) diag(exp(g))   (gated)
   float* g;            // [B*H][chunks][C]     cumulative log decay        (gated)
+  __nv_bfloat16* khat; // [B*H][T][Dk]          keys after the layer's pre-step (pre-step only)
 };
 size_t wy_workspace_bytes(int B, int H, int T, int C);
+// Bytes of the mapped keys the pre-step adds after the factors (256-byte aligned start).
+size_t wy_khat_bytes(int B, int H, int T, int Dk);
 WyWorkspace wy_carve(void* base, int B, int H, int T, int C);
 cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 

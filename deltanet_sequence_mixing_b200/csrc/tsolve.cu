@@ -78,8 +78,8 @@ template <int C, int DK, bool GATED, bool PRE>
 __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
                   const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
-                  __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out, int T, int nchunks,
-                  unsigned int* status) {
+                  __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out,
+                  __nv_bfloat16* __restrict__ khat, int T, int nchunks, unsigned int* status) {
   using Sh = TsolveShape<C>;
   using SL = TsolveSmem<C, DK>;
   constexpr int kC = C, kApad = Sh::kApad;
@@ -147,10 +147,13 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
   }
   bool ok = true;
   if (PRE) {
-    // The layer's pre-step on K in shared memory (two threads per row, the
-    // same split as the chunk kernel's, so both see identical bf16 keys).
+    // The layer's pre-step on K in shared memory (two threads per row); the
+    // mapped rows also go to the workspace, where the chunk kernel reads them.
     ok = __all_sync(0xffffffffu, mbar_wait(bar_full, 0, wc));  // warp-uniform for the shuffles
-    if (ok) prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, tid >> 1, tid & 1);
+    const int r = tid >> 1;
+    if (ok)
+      prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, r, tid & 1,
+                            r < n ? khat + ((size_t)bh * T + c0 + r) * DK : nullptr);
     fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
   }
@@ -419,8 +422,8 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((size_t)nchunks * p.B * p.H));  // at most INT_MAX (checked by the caller)
-  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, p.T, nchunks,
-                                                      p.status);
+  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, w.khat, p.T,
+                                                      nchunks, p.status);
   return cudaGetLastError();
 }
 
@@ -446,6 +449,8 @@ size_t wy_workspace_bytes(int B, int H, int T, int C) {
   return tiles * (2 * (size_t)C * C * 2 + (size_t)C * 4);  // Tb, Tbg (bf16) and g (f32)
 }
 
+size_t wy_khat_bytes(int B, int H, int T, int Dk) { return (size_t)B * H * T * Dk * 2; }
+
 WyWorkspace wy_carve(void* base, int B, int H, int T, int C) {
   const size_t nch = ((size_t)T + C - 1) / C;
   const size_t tiles = (size_t)B * H * nch;
@@ -454,6 +459,8 @@ WyWorkspace wy_carve(void* base, int B, int H, int T, int C) {
   w.tb = reinterpret_cast<__nv_bfloat16*>(q);
   w.tbg = reinterpret_cast<__nv_bfloat16*>(q + tiles * C * C * 2);
   w.g = reinterpret_cast<float*>(q + 2 * tiles * C * C * 2);
+  // mapped keys (pre-step only): after the factors, on a 256-byte boundary
+  w.khat = reinterpret_cast<__nv_bfloat16*>(q + (wy_workspace_bytes(B, H, T, C) + 255) / 256 * 256);
   return w;
 }
 
