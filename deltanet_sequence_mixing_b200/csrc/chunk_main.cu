@@ -18,24 +18,25 @@
 //   warp 9     MMA issuer (warp-uniform, one elected lane issues): every
 //              tcgen05.mma of the CTA, in a fixed order that keeps the state
 //              chain fed:
-//                [Q;W]S (c), W/Uh (c+1), PU (c-1), K^T U (c), QK^T (c+1)
-//              W/Uh (c+1) and PU (c-1) run while the U epilogue of chunk c
-//              drains, QK^T (c+1) while the state update does: the in-order
-//              tensor pipe then never holds the next state-chain product
-//              behind more work than fits in the epilogue before it (Uh, U and
-//              P are double-buffered).
+//                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
+//              W/Uh (c+1) runs while the U epilogue of chunk c drains (Uh is
+//              double-buffered in TMEM); PU (c) and QK^T (c+1) run during the
+//              state update.
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
 //              a three-stage ring, L2 prefetch two chunks ahead
 //   warps 6-7  W rows to bf16 into tensor memory (state-independent, one chunk
 //              ahead), then columns 32-63 of the U epilogue
-//   warps 4-5  Q rows into tensor memory; P rows to bf16 (gated: with the decay Gamma)
+//   warps 4-5  Q rows into tensor memory; P rows (gated: with the decay Gamma)
 //   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
 //   warps 0-1  gated: QS rows times gamma in TMEM while the U epilogue runs;
 //              drain the output tile O = diag(gamma) QS + PU
 // Operands and shared-memory traffic: every product whose A operand is built
-// inside the CTA for both QK^T and [Q;W]S takes it from tensor memory ([Q; W]),
-// so those MMAs read only their B operand from shared memory: Q is copied into
-// tensor memory once per chunk and W never passes through shared memory.
+// inside the CTA takes it from tensor memory ([Q; W] for QK^T and [Q;W]S, P for
+// PU), so those MMAs read only their B operand from shared memory.  The SS
+// form re-reads the 128-row A tile (4 KB) for every K = 16 step, which made the
+// N = 64 products shared-memory bound and slowed the epilogues' own shared
+// accesses; Q is copied into tensor memory once per chunk instead, and W and P
+// never pass through shared memory.
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
 // signal back; the issuer waits on their signals.  Every mbarrier completes
 // once per chunk (or per use of a parity), so parity waits are unambiguous.
@@ -59,7 +60,8 @@ constexpr int kWG = 128;
 constexpr int kThreads = 2 * kWG + 64;  // chain 0-3, prep 4-7, producer 8, issuer 9
 constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kBarPrepW = 5;
 
-// TMEM columns: G (QK^T scores), W (float32, Dk columns), Uh[0], QW[2] (lanes 0-63: O, lanes 64-127:
+// TMEM columns: G (QK^T scores, then P as bf16 A operand in its first
+// columns), W (float32, Dk columns), Uh[0], QW[2] (lanes 0-63: O, lanes 64-127:
 // WS), Uh[1], AQW (the bf16 A operand [Q; W]: Q on lanes 0-63, W on lanes
 // 64-127, Dk / 2 columns).  Uh[0] sits right after W (at TM_W + Dk) so that,
 // ungated and for even chunks, one N = Dk + 64 product writes both.  The
@@ -68,15 +70,13 @@ constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kB
 constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_UH1 = 384, TM_AQW = 448;
 
 // Shared memory.  A stage holds one chunk's TMA tiles [K | Q] per 64 columns
-// of Dk, V, Tb (gated also Tbg and the g rows).  Three stages ungated (the
-// chunk after next streams in while one chunk is on the state chain and the
-// next is being prepared), two gated (Tbg, the g rows and the decay-weighted
-// U~ leave no room for a third).  U, U~ and P are double-buffered: PU (c-1)
-// reads them while the epilogues of chunk c write the other buffers.
+// of Dk, V, Tb (gated also Tbg and the g rows).  Three stages: the chunk after
+// next streams in while one chunk is on the state chain and the next is being
+// prepared.
 template <int DK, bool GATED>
 struct MainLayout {
   static constexpr int KB = DK / 64;
-  static constexpr int NST = GATED ? 2 : 3;           // ring stages
+  static constexpr int NST = 3;                       // ring stages
   static constexpr uint32_t KB_STRIDE = 2 * kTile;    // [K | Q] per 64 columns of Dk
   static constexpr uint32_t K_OFF = 0, Q_OFF = kTile;
   static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | (Tbg | beta, g)
@@ -84,10 +84,9 @@ struct MainLayout {
   static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
   static constexpr uint32_t VEC_OFF = TBG_OFF + kTile;
   static constexpr uint32_t STAGE = GATED ? VEC_OFF + 1024 : TBG_OFF;
-  static constexpr uint32_t U_OFF = NST * STAGE;                    // U[2]
-  static constexpr uint32_t UT_OFF = U_OFF + 2 * kTile;             // gated: U~[2]
-  static constexpr uint32_t P_OFF = UT_OFF + (GATED ? 2 : 0) * kTile;  // P[2]
-  static constexpr uint32_t S_OFF = P_OFF + 2 * kTile;              // bf16 state, DK rows x 128 B
+  static constexpr uint32_t U_OFF = NST * STAGE;      // U | (U~)
+  static constexpr uint32_t UT_OFF = U_OFF + kTile;
+  static constexpr uint32_t S_OFF = U_OFF + (GATED ? 2 : 1) * kTile;  // bf16 state, DK rows x 128 B
   static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // gated: chain copy of g per parity, [2][64]
   static constexpr uint32_t BAR_OFF = CV_OFF + (GATED ? 2 * 64 * 4 : 0);
   static constexpr uint32_t BYTES = BAR_OFF + 256;
@@ -97,11 +96,11 @@ struct MainLayout {
 };
 
 // mbarrier slots (8 bytes each).  FULL and EMPTY: one per ring stage;
-// OFREE, CMMA5, PREADY and QSCALED: one per chunk parity.
+// OFREE, CMMA5 and PREADY: one per chunk parity.
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
                    B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168,
-                   B_QREADY = 184;
+                   B_QREADY = 176;
 
 // Pack 32 floats into 16 32-bit words of bf16 pairs (element 2i in the low half).
 __device__ __forceinline__ void pack16(const float* x, uint32_t* w) {
@@ -165,7 +164,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar + B_OFREE + 8 * i, 1);
       mbar_init(bar + B_CMMA5 + 8 * i, 1);
       mbar_init(bar + B_PREADY + 8 * i, 1);
-      mbar_init(bar + B_QSCALED + 8 * i, 1);  // gated: the QS rows of TM_QW[parity] scaled by gamma
     }
     mbar_init(bar + B_CMMA3, 1);
     mbar_init(bar + B_CMMA4, 1);
@@ -174,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
     mbar_init(bar + B_WREADY, 1);
+    mbar_init(bar + B_QSCALED, 1);  // gated: the QS rows of TM_QW scaled by gamma
     mbar_init(bar + B_QREADY, 1);   // Q of the chunk in the A operand region AQW
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
@@ -310,33 +309,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dS = K^T U~ into Uh[c & 1] (drained by the U epilogue of chunk c)
     auto issue_ds = [&](int c) {
       const uint32_t st = stage(c);
-      const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF) + (c & 1) * kTile;
+      const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
       constexpr uint32_t id = idesc_bf16(128, 64, true, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         mma_bf16_ss_elect(tmem + ((c & 1) ? TM_UH1 : TM_UH0), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
                           desc_mn(ut + ks * 2048, kTile), id, ks > 0);
     };
-    // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1];
-    // A rows 64-127 read the tile after P[c & 1] and land on the consumed WS rows)
+    // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1]);
+    // A = P, bf16 in the first columns of TM_G
     auto issue_pu = [&](int c) {
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
-      const uint32_t pa = sb + L::P_OFF + (c & 1) * kTile, ub = sb + L::U_OFF + (c & 1) * kTile;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32), desc_mn(ub + ks * 2048, kTile), id,
-                          1);
-    };
-    // PU (c) once its P rows are written (and, gated, its QS rows scaled);
-    // gated, the P rows were the last reader of stage c's g rows
-    auto pu_step = [&](int c) {
-      const bool r = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * (c & 1), (c >> 1) & 1, wc) &&
-                                                 (!GATED || mbar_wait(bar + B_QSCALED + 8 * (c & 1), (c >> 1) & 1, wc)));
-      if (!r) return false;
-      tc_fence_after();
-      issue_pu(c);
-      mma_commit_elect(bar + B_CMMA5 + 8 * (c & 1));
-      return true;
+        mma_bf16_ts_elect(tmem + TM_QW + 64 * (c & 1), tmem + TM_G + ks * 8,
+                          desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
     };
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL, 0, wc));
     if (ok) {
@@ -368,21 +355,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_wu(c + 1);
         mma_commit_elect(bar + B_PMMA2);
       }
-      if (c > 0 && !(ok = pu_step(c - 1))) break;
       ok = __all_sync(0xffffffffu, mbar_wait(bar + B_UREADY, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
       issue_ds(c);
       mma_commit_elect(bar + B_CMMA4);
-      // K^T U (c) is the last MMA that reads stage c (Q went to TMEM before
-      // Q_READY; PU reads U and P outside the ring).  Gated, the P rows of
-      // chunk c also read its g rows: the stage goes once they are done.
+      // K^T U (c) is the last MMA that reads stage c.  Ungated the stage is
+      // free now (Q went to TMEM before Q_READY); gated the P rows of chunk c
+      // still read its g rows, so it goes once they are done.
       if (!GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
-      // QK^T (c+1) overwrites TM_G once the P rows of chunk c have left it
-      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc) &&
+                                       (!GATED || mbar_wait(bar + B_QSCALED, c & 1, wc)));
       if (!ok) break;
+      tc_fence_after();
       if (GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
-      if (nxt) {  // [Q; W] (c+1) is in TMEM
+      issue_pu(c);
+      mma_commit_elect(bar + B_CMMA5 + 8 * b);
+      if (nxt) {  // after PU (c): TM_G is free once PMMA1 fires; [Q; W] (c+1) is in TMEM
         ok = __all_sync(0xffffffffu, mbar_wait(bar + B_QREADY, (c + 1) & 1, wc) &&
                                          mbar_wait(bar + B_WREADY, (c + 1) & 1, wc));
         if (!ok) break;
@@ -391,7 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_elect(bar + B_PMMA1);
       }
     }
-    if (ok && nchunks > 0) ok = pu_step(nchunks - 1);
     tc_fence_after();  // no MMA may outlive TMEM
     mma_commit_elect(bar + B_FIN);
     int zero = 0;
@@ -441,8 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* vb = cvec + (c & 1) * 64;
         const float wl = GATED ? __expf(vb[n - 1] - vb[row]) : 1.f;
         u_epilogue_half<GATED>(tmem + lane_base + TM_QW + 64 * (c & 1),
-                               tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0), 32, row, wl,
-                               sm + L::U_OFF + (c & 1) * kTile, sm + L::UT_OFF + (c & 1) * kTile);
+                               tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0), 32, row, wl, sm + L::U_OFF,
+                               sm + L::UT_OFF);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -552,12 +540,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int sc = 0; sc < 64; ++sc) pv[sc] = sc <= row ? pv[sc] * __expf(gr - vs[64 + sc]) : 0.f;
         }
-        // P as the bf16 A operand of PU (K-major, P[c & 1])
-        uint8_t* ptile = sm + L::P_OFF + b * kTile;
+        // P as the bf16 A operand of PU: the first 32 columns of TM_G (packed
+        // in place: word i takes elements 2i and 2i + 1, read before it is written)
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(ptile + sw128_off(row, c16), pv + c16 * 8);
+        for (int i = 0; i < 32; ++i) g[i] = pack2_bf16(pv[2 * i], pv[2 * i + 1]);
+        tmem_st32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrepP, 64);
       if (row == 0) mbar_arrive(bar + B_PREADY + 8 * b);
@@ -596,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float wl = GATED ? __expf(vb[n - 1] - vb[row]) : 1.f;
           // columns 0-31 here, 32-63 in the W warps (same TMEM lanes)
           u_epilogue_half<GATED>(qw + lane_base, tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0), 0, row, wl,
-                                 sm + L::U_OFF + (c & 1) * kTile, sm + L::UT_OFF + (c & 1) * kTile);
+                                 sm + L::U_OFF, sm + L::UT_OFF);
           fence_proxy_async_smem();
           tc_fence_before();
           named_bar_sync(kBarChainHi, 64);
@@ -621,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
           tc_fence_before();
           named_bar_sync(kBarChainLo, 64);
-          if (ct == 0) mbar_arrive(bar + B_QSCALED + 8 * b);
+          if (ct == 0) mbar_arrive(bar + B_QSCALED);
         }
       }
       ok = named_bar_and(kBarChain, kWG, ok_hi && ok_lo && mbar_wait(bar + B_CMMA4, c & 1, wc));
