@@ -131,7 +131,7 @@ int run_chunked_at(dn::ChunkProblem& p, unsigned int* status, void* wy, cudaStre
     return map_cuda(e);
   }
   if (tensor_core_path(p)) {
-    const dn::WyWorkspace w = dn::wy_carve(wy, p.B, p.H, p.T, p.C);
+    const dn::WyWorkspace w = dn::wy_carve(wy, p.B, p.H, p.T, p.C, p.Dk);
     return map_cuda(p.C == 64 ? dn::launch_chunk_main(p, w, st) : dn::launch_chunk128(p, w, st));
   }
   if (dn::linear_tc_supported(p)) return map_cuda(dn::launch_linear_tc(p, st));
@@ -222,7 +222,7 @@ size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, d
   if (options == DN_OPT_PRESTEP) {
     if (dt != DN_BF16 || T == 0) return kStatusBytes;  // the CUDA-core kernel
     const size_t wy = dn::wy_workspace_bytes(B, H, T, C);
-    return kStatusBytes + (wy + 255) / 256 * 256 + dn::wy_khat_bytes(B, H, T, Dk);  // + the mapped keys
+    return kStatusBytes + (wy + 255) / 256 * 256 + dn::wy_khat_bytes(B, H, T, Dk);  // + mapped k and q
   }
   return kStatusBytes;
 }

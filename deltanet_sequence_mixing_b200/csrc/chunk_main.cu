@@ -21,29 +21,23 @@
 //                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
 //              W/Uh (c+1) runs while the U epilogue of chunk c drains (Uh is
 //              double-buffered in TMEM); PU (c) and QK^T (c+1) run during the
-//              state update.
+//              state update.  The single P tile is rewritten only after PU (c)
+//              has completed (QK^T (c+1) is committed after it).
 //   warp 8     producer: TMA of K, Q, V, Tb (gated: Tbg and the g rows) into
-//              a three-stage ring, L2 prefetch two chunks ahead
-//   warps 6-7  W rows to bf16 into tensor memory (state-independent, one chunk
-//              ahead), then columns 32-63 of the U epilogue
-//   warps 4-5  Q rows into tensor memory; P rows (gated: with the decay Gamma)
+//              a three-stage ring (gated: two), L2 prefetch two chunks ahead
+//   warps 6-7  W rows to bf16 next to Q (state-independent, one chunk ahead),
+//              then columns 32-63 of the U epilogue
+//   warps 4-5  P rows to bf16 (gated: with the decay Gamma)
 //   warps 2-3  U = Uh - WS (columns 0-31);   warps 0-3 the state update;
 //   warps 0-1  gated: QS rows times gamma in TMEM while the U epilogue runs;
 //              drain the output tile O = diag(gamma) QS + PU
-// Operands and shared-memory traffic: every product whose A operand is built
-// inside the CTA takes it from tensor memory ([Q; W] for QK^T and [Q;W]S, P for
-// PU), so those MMAs read only their B operand from shared memory.  The SS
-// form re-reads the 128-row A tile (4 KB) for every K = 16 step, which made the
-// N = 64 products shared-memory bound and slowed the epilogues' own shared
-// accesses; Q is copied into tensor memory once per chunk instead, and W and P
-// never pass through shared memory.
 // Epilogue warps only wait on mbarriers signalled by tcgen05.commit and
 // signal back; the issuer waits on their signals.  Every mbarrier completes
 // once per chunk (or per use of a parity), so parity waits are unambiguous.
-// Accumulators live in TMEM (512 columns), shared-memory operands in the
-// 128-byte-swizzled canonical layout, the running state in float32 registers.
-// All waits are bounded; a wait that runs out sets the workspace status word
-// and the CTA winds down (copies drained, TMEM freed) without trapping.
+// Accumulators live in TMEM (512 columns), every operand in the 128-byte-
+// swizzled canonical layout, the running state in float32 registers.  All
+// waits are bounded; a wait that runs out sets the workspace status word and
+// the CTA winds down (copies drained, TMEM freed) without trapping.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -60,31 +54,30 @@ constexpr int kWG = 128;
 constexpr int kThreads = 2 * kWG + 64;  // chain 0-3, prep 4-7, producer 8, issuer 9
 constexpr int kBarChain = 1, kBarChainHi = 2, kBarChainLo = 3, kBarPrepP = 4, kBarPrepW = 5;
 
-// TMEM columns: G (QK^T scores, then P as bf16 A operand in its first
-// columns), W (float32, Dk columns), Uh[0], QW[2] (lanes 0-63: O, lanes 64-127:
-// WS), Uh[1], AQW (the bf16 A operand [Q; W]: Q on lanes 0-63, W on lanes
-// 64-127, Dk / 2 columns).  Uh[0] sits right after W (at TM_W + Dk) so that,
-// ungated and for even chunks, one N = Dk + 64 product writes both.  The
-// state update K^T U of chunk c lands in Uh[c & 1], which the U epilogue of
-// chunk c has just drained.
-constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_UH1 = 384, TM_AQW = 448;
+// TMEM columns: G (P scores), W, Uh[0], QW[2] (lanes 0-63: O, lanes 64-127: WS),
+// dS, Uh[1].  Uh[0] sits right after W (at TM_W + Dk) so that, ungated and for
+// even chunks, one N = Dk + 64 product writes both.
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_QW = 256, TM_DS = 384, TM_UH1 = 448;
 
-// Shared memory.  A stage holds one chunk's TMA tiles [K | Q] per 64 columns
-// of Dk, V, Tb (gated also Tbg and the g rows).  Three stages: the chunk after
-// next streams in while one chunk is on the state chain and the next is being
-// prepared.
+// Shared memory.  A stage holds one chunk's TMA tiles [K | Q | W] per 64
+// columns of Dk, V, Tb (gated also Tbg and the g rows); W is written there
+// by the W warps, right after Q, so that [Q; W] is one M = 128 operand.
+// Ungated runs a three-stage ring (the chunk after next streams in while one
+// chunk is on the state chain and the next is being prepared); gated needs
+// the Tbg tile, the decay-weighted U and the g rows, and fits two stages.
 template <int DK, bool GATED>
 struct MainLayout {
   static constexpr int KB = DK / 64;
-  static constexpr int NST = 3;                       // ring stages
-  static constexpr uint32_t KB_STRIDE = 2 * kTile;    // [K | Q] per 64 columns of Dk
-  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile;
+  static constexpr int NST = GATED ? 2 : 3;           // ring stages
+  static constexpr uint32_t KB_STRIDE = 3 * kTile;    // [K | Q | W] per 64 columns of Dk
+  static constexpr uint32_t K_OFF = 0, Q_OFF = kTile, W_OFF = 2 * kTile;
   static constexpr uint32_t V_OFF = KB * KB_STRIDE;   // V | Tb | (Tbg | beta, g)
   static constexpr uint32_t TB_OFF = V_OFF + kTile;
   static constexpr uint32_t TBG_OFF = TB_OFF + kTile;
   static constexpr uint32_t VEC_OFF = TBG_OFF + kTile;
   static constexpr uint32_t STAGE = GATED ? VEC_OFF + 1024 : TBG_OFF;
-  static constexpr uint32_t U_OFF = NST * STAGE;      // U | (U~)
+  static constexpr uint32_t P_OFF = NST * STAGE;      // P | U | (UT)
+  static constexpr uint32_t U_OFF = P_OFF + kTile;
   static constexpr uint32_t UT_OFF = U_OFF + kTile;
   static constexpr uint32_t S_OFF = U_OFF + (GATED ? 2 : 1) * kTile;  // bf16 state, DK rows x 128 B
   static constexpr uint32_t CV_OFF = S_OFF + DK * 128;  // gated: chain copy of g per parity, [2][64]
@@ -99,14 +92,7 @@ struct MainLayout {
 // OFREE, CMMA5 and PREADY: one per chunk parity.
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_OFREE = 48, B_CMMA5 = 64, B_PREADY = 80,
                    B_CMMA3 = 96, B_CMMA4 = 104, B_PMMA1 = 112, B_PMMA2 = 120, B_UREADY = 128,
-                   B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168,
-                   B_QREADY = 176;
-
-// Pack 32 floats into 16 32-bit words of bf16 pairs (element 2i in the low half).
-__device__ __forceinline__ void pack16(const float* x, uint32_t* w) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = pack2_bf16(x[2 * i], x[2 * i + 1]);
-}
+                   B_SREADY = 136, B_WREADY = 144, B_FIN = 152, B_TMEM = 160, B_ABORT = 164, B_QSCALED = 168;
 
 // One half (32 columns, [col0, col0 + 32)) of the U epilogue for the row on
 // this thread's TMEM lane: U = Uh - WS to bf16 (gated also U~ = U e^(g_last - g_row)).
@@ -131,7 +117,7 @@ __device__ __forceinline__ void u_epilogue_half(uint32_t ws_addr, uint32_t uh_ad
   }
 }
 
-template <int DK, bool GATED, bool PRE>
+template <int DK, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
@@ -173,7 +159,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_SREADY, 1);
     mbar_init(bar + B_WREADY, 1);
     mbar_init(bar + B_QSCALED, 1);  // gated: the QS rows of TM_QW scaled by gamma
-    mbar_init(bar + B_QREADY, 1);   // Q of the chunk in the A operand region AQW
     mbar_init(bar + B_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -261,14 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // each MMA and commit is issued by one elected lane.  Wait results are
     // combined over the warp so every lane takes the same path.
     auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
-    // P scores = Q K^T of chunk c (lanes 0-63 of TM_G); A = [Q; W] from TMEM
+    // P scores = Q K^T of chunk c (lanes 0-63 of TM_G)
     auto issue_qkt = [&](int c) {
       const uint32_t st = stage(c);
       constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
         const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
-        mma_bf16_ts_elect(tmem + TM_G, tmem + TM_AQW + ks * 8, desc_k(st + L::K_OFF + off), id, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
       }
     };
     // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of Uh[c & 1]).
@@ -298,31 +283,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    // [Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1]); A = [Q; W] from TMEM
+    // [Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
     auto issue_qw = [&](int c) {
+      const uint32_t st = stage(c);
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks)
-        mma_bf16_ts_elect(tmem + TM_QW + 64 * (c & 1), tmem + TM_AQW + ks * 8,
-                          desc_mn(sb + L::S_OFF + ks * 2048, kTile), id, ks > 0);
+      for (int ks = 0; ks < DK / 16; ++ks) {
+        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
+                          id, ks > 0);
+      }
     };
-    // dS = K^T U~ into Uh[c & 1] (drained by the U epilogue of chunk c)
+    // dS = K^T U~
     auto issue_ds = [&](int c) {
       const uint32_t st = stage(c);
       const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
       constexpr uint32_t id = idesc_bf16(128, 64, true, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + ((c & 1) ? TM_UH1 : TM_UH0), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
+        mma_bf16_ss_elect(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
                           desc_mn(ut + ks * 2048, kTile), id, ks > 0);
     };
-    // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1]);
-    // A = P, bf16 in the first columns of TM_G
+    // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
     auto issue_pu = [&](int c) {
+      const uint32_t pa = sb + L::P_OFF;
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ts_elect(tmem + TM_QW + 64 * (c & 1), tmem + TM_G + ks * 8,
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32),
                           desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
     };
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL, 0, wc));
@@ -330,10 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       issue_wu(0);
       mma_commit_elect(bar + B_PMMA2);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar + B_QREADY, 0, wc) && mbar_wait(bar + B_WREADY, 0, wc));
-    }
-    if (ok) {
-      tc_fence_after();
       issue_qkt(0);
       mma_commit_elect(bar + B_PMMA1);
     }
@@ -341,14 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = c & 1;
       const bool nxt = c + 1 < nchunks;
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar + B_WREADY, c & 1, wc) && mbar_wait(bar + B_QREADY, c & 1, wc) &&
-                          mbar_wait(bar + B_SREADY, c & 1, wc) &&
+                      mbar_wait(bar + B_WREADY, c & 1, wc) && mbar_wait(bar + B_SREADY, c & 1, wc) &&
                           (c < 2 || mbar_wait(bar + B_OFREE + 8 * b, ((c >> 1) - 1) & 1, wc)));
       if (!ok) break;
       tc_fence_after();
       issue_qw(c);
       mma_commit_elect(bar + B_CMMA3);
-      if (nxt) {  // Uh[(c+1) & 1] was drained by chunk c-1 and its dS read by the state update
+      if (nxt) {  // W (c) is already in shared memory and Uh[(c+1) & 1] was consumed by chunk c-1
         ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc));
         if (!ok) break;
         tc_fence_after();
@@ -361,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_ds(c);
       mma_commit_elect(bar + B_CMMA4);
       // K^T U (c) is the last MMA that reads stage c.  Ungated the stage is
-      // free now (Q went to TMEM before Q_READY); gated the P rows of chunk c
-      // still read its g rows, so it goes once they are done.
+      // free now (its W / Q epilogues came before W_READY); gated the P rows
+      // of chunk c still read its g rows, so it goes once they are done.
       if (!GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
       ok = __all_sync(0xffffffffu, mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc) &&
                                        (!GATED || mbar_wait(bar + B_QSCALED, c & 1, wc)));
@@ -371,11 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (GATED) mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));
       issue_pu(c);
       mma_commit_elect(bar + B_CMMA5 + 8 * b);
-      if (nxt) {  // after PU (c): TM_G is free once PMMA1 fires; [Q; W] (c+1) is in TMEM
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_QREADY, (c + 1) & 1, wc) &&
-                                         mbar_wait(bar + B_WREADY, (c + 1) & 1, wc));
-        if (!ok) break;
-        tc_fence_after();
+      if (nxt) {  // after PU (c): the single P tile is free once PMMA1 fires
         issue_qkt(c + 1);
         mma_commit_elect(bar + B_PMMA1);
       }
@@ -397,25 +376,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                              mbar_wait(bar + B_PMMA2, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      // W (float32, lanes 64-127 of TM_W) -> bf16 A operand rows 64-127 of AQW.
-      // [Q;W]S (c-1) and QK^T (c-1), the last readers of AQW's W rows, ran before
-      // W/Uh (c) on the in-order tensor pipe.
 #pragma unroll
-      for (int h = 0; h < DK / 64; ++h) {
-        uint32_t w[32], pk[32];
+      for (int q = 0; q < DK / 32; ++q) {
+        uint32_t w[32];
+        tmem_ld32(tmem + lane_base + TM_W + q * 32, w);
+        tmem_wait_ld();
+        uint8_t* wt = stp + (q >> 1) * L::KB_STRIDE + L::W_OFF;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld32(tmem + lane_base + TM_W + h * 64 + half * 32, w);
-          tmem_wait_ld();
-          pack16(reinterpret_cast<const float*>(w), pk + 16 * half);
-        }
-        tmem_st32(tmem + lane_base + TM_AQW + h * 32, pk);
+        for (int cc = 0; cc < 4; ++cc)
+          st_bf16x8(wt + sw128_off(row, (q & 1) * 4 + cc), reinterpret_cast<const float*>(w) + cc * 8);
       }
-      tmem_wait_st();
       if (GATED) {  // the chain's copy of g (the stage is released before the chain is done)
         const float* vs = reinterpret_cast<const float*>(stp + L::VEC_OFF);
         cvec[(c & 1) * 64 + row] = vs[64 + row];
       }
+      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrepW, 64);
       if (tid == 192) mbar_arrive(bar + B_WREADY);
@@ -445,56 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = c & 1;
       uint8_t* stp = sm + (c % NST) * L::STAGE;
       float* vs = reinterpret_cast<float*>(stp + L::VEC_OFF);  // gated only: g at [64, 128)
-      // Q (c) -> bf16 A operand rows 0-63 of AQW, once [Q;W]S (c-1) (the last
-      // reader of Q (c-1)) has completed
-      ok = named_bar_and(kBarPrepP, 64,
-                         mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc) &&
-                             (c == 0 || mbar_wait(bar + B_CMMA3, (c - 1) & 1, wc)));
+      ok = named_bar_and(kBarPrepP, 64, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
-      tc_fence_after();
-      float qinv = 1.f;
-      if (PRE) {  // the layer's pre-step on q: silu, then 1 / max(||silu(q)||, 1e-12)
-        float ss = 0.f;
-#pragma unroll
-        for (int kb = 0; kb < DK / 64; ++kb)
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(stp + kb * L::KB_STRIDE + L::Q_OFF + sw128_off(row, c16)), x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float y = silu_f(x[e]);
-              ss = fmaf(y, y, ss);
-            }
-          }
-        qinv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
-      }
-#pragma unroll
-      for (int kb = 0; kb < DK / 64; ++kb) {
-        const uint8_t* qt = stp + kb * L::KB_STRIDE + L::Q_OFF;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint4 u = *reinterpret_cast<const uint4*>(qt + sw128_off(row, c16));
-          if (PRE) {
-            float x[8];
-            unpack_bf16x8(u, x);
-            u.x = pack2_bf16(silu_f(x[0]) * qinv, silu_f(x[1]) * qinv);
-            u.y = pack2_bf16(silu_f(x[2]) * qinv, silu_f(x[3]) * qinv);
-            u.z = pack2_bf16(silu_f(x[4]) * qinv, silu_f(x[5]) * qinv);
-            u.w = pack2_bf16(silu_f(x[6]) * qinv, silu_f(x[7]) * qinv);
-          }
-          pk[4 * c16] = u.x;
-          pk[4 * c16 + 1] = u.y;
-          pk[4 * c16 + 2] = u.z;
-          pk[4 * c16 + 3] = u.w;
-        }
-        tmem_st32(tmem + lane_base + TM_AQW + kb * 32, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      named_bar_sync(kBarPrepP, 64);
-      if (row == 0) mbar_arrive(bar + B_QREADY);
       // Gated: Gamma_rs = e^(g_r - g_s) (s <= r) as a_r b_s, a_r = e^(g_r - m),
       // b_s = e^(m - g_s) with m the midpoint of the chunk's g range (g is
       // non-increasing, rows past T flat).  Both factors stay within e^(+-80)
@@ -517,8 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
         tmem_ld32(tmem + lane_base + TM_G + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
         tmem_wait_ld();
+        uint8_t* ptile = sm + L::P_OFF;
         // every value of the row in registers (the shared-memory reads of the
-        // decay factors all come before any use)
+        // decay factors all come before the first store of the P tile)
         float* pv = reinterpret_cast<float*>(g);
         if (!GATED || fact) {
 #pragma unroll
@@ -540,13 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int sc = 0; sc < 64; ++sc) pv[sc] = sc <= row ? pv[sc] * __expf(gr - vs[64 + sc]) : 0.f;
         }
-        // P as the bf16 A operand of PU: the first 32 columns of TM_G (packed
-        // in place: word i takes elements 2i and 2i + 1, read before it is written)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) g[i] = pack2_bf16(pv[2 * i], pv[2 * i + 1]);
-        tmem_st32(tmem + lane_base + TM_G, *reinterpret_cast<uint32_t(*)[32]>(g));
-        tmem_wait_st();
+        for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(ptile + sw128_off(row, c16), pv + c16 * 8);
       }
+      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(kBarPrepP, 64);
       if (row == 0) mbar_arrive(bar + B_PREADY + 8 * b);
@@ -621,9 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ct < DK) {
         const float carry = GATED ? __expf(vb[n - 1]) : 1.f;
         uint32_t ds[64];
-        const uint32_t dsa = tmem + lane_base + ((c & 1) ? TM_UH1 : TM_UH0);
-        tmem_ld32(dsa, *reinterpret_cast<uint32_t(*)[32]>(ds));
-        tmem_ld32(dsa + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
+        tmem_ld32(tmem + lane_base + TM_DS, *reinterpret_cast<uint32_t(*)[32]>(ds));
+        tmem_ld32(tmem + lane_base + TM_DS + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 64; ++e) sreg[e] = fmaf(carry, sreg[e], __uint_as_float(ds[e]));
@@ -672,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, bool GATED, bool PRE>
+template <int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   using L = MainLayout<DK, GATED>;
   const int BH = p.B * p.H;
@@ -680,13 +604,15 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   cudaError_t e = launch_tsolve(p, w, st);
   if (e != cudaSuccess) return e;
   CUtensorMap mq, mk, mv, mtb, mtbg;
-  // with the pre-step the keys come mapped from the pre-pass (workspace)
-  if (!make_tmap_3d_bf16(&mq, p.q, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, PRE ? w.khat : p.k, DK, p.T, BH) ||
+  // with the layer's pre-step, q and k come mapped from the pre-pass (workspace)
+  const void* qsrc = p.prestep ? static_cast<const void*>(w.qhat) : p.q;
+  const void* ksrc = p.prestep ? static_cast<const void*>(w.khat) : p.k;
+  if (!make_tmap_3d_bf16(&mq, qsrc, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, ksrc, DK, p.T, BH) ||
       !make_tmap_3d_bf16(&mv, p.v, p.Dv, p.T, BH) ||
       !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
       !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))
     return cudaErrorInvalidValue;
-  auto kern = chunk_main_kernel<DK, GATED, PRE>;
+  auto kern = chunk_main_kernel<DK, GATED>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
@@ -712,15 +638,10 @@ bool chunk_main_supported(const ChunkProblem& p) {
          (p.Dv == 64 || p.Dv == 128);
 }
 
-template <bool PRE>
-cudaError_t launch_pre(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  const bool gated = p.alpha != nullptr;
-  if (p.Dk == 128) return gated ? launch_t<128, true, PRE>(p, w, st) : launch_t<128, false, PRE>(p, w, st);
-  return gated ? launch_t<64, true, PRE>(p, w, st) : launch_t<64, false, PRE>(p, w, st);
-}
-
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  return p.prestep ? launch_pre<true>(p, w, st) : launch_pre<false>(p, w, st);
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
+  return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
 }
 
 }  // namespace dn

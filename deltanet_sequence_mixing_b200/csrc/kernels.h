@@ -72,11 +72,14 @@ struct WyWorkspace {
   __nv_bfloat16* tbg;  // [B*H][chunks][C][C]  T diag(beta) diag(exp(g))   (gated)
   float* g;            // [B*H][chunks][C]     cumulative log decay        (gated)
   __nv_bfloat16* khat; // [B*H][T][Dk]          keys after the layer's pre-step (pre-step only)
+  __nv_bfloat16* qhat; // [B*H][T][Dk]          queries after the layer's pre-step (pre-step only)
 };
 size_t wy_workspace_bytes(int B, int H, int T, int C);
-// Bytes of the mapped keys the pre-step adds after the factors (256-byte aligned start).
+// Bytes of the mapped keys and queries the pre-step adds after the factors
+// (each region starts on a 256-byte boundary).
 size_t wy_khat_bytes(int B, int H, int T, int Dk);
-WyWorkspace wy_carve(void* base, int B, int H, int T, int C);
+// Dk: head size of q and k, for the pre-step regions (any value when unused)
+WyWorkspace wy_carve(void* base, int B, int H, int T, int C, int Dk);
 cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
 
 // tcgen05 chunked delta rule after the pre-pass (bf16, C = 64).

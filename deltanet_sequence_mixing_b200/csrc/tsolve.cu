@@ -74,12 +74,49 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
   for (int t = 0; t < f.num_elements; ++t) f.x[t] = __uint_as_float(__float_as_uint(f.x[t]) & 0xFFFFE000u);
 }
 
+// The layer's pre-step on one query row in global memory, two lanes per row
+// (lane parity `part` takes columns [part * DK/2, (part + 1) * DK/2)):
+// dst <- silu(src) / max(||silu(src)||_2, 1e-12).  All 32 lanes of the warp
+// call it (`live` false skips the memory accesses of rows past T).
+template <int DK>
+__device__ __forceinline__ void prestep_row_global(const __nv_bfloat16* src, __nv_bfloat16* dst, bool live,
+                                                   int part) {
+  constexpr int NCH = DK / 16;  // 16-byte chunks per lane
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + part * (DK / 2));
+  float ss = 0.f;
+  if (live) {
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      float x[8];
+      unpack_bf16x8(s4[j], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float y = silu_f(x[e]);
+        ss = fmaf(y, y, ss);
+      }
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, ss, 1);
+  const float inv = 1.f / fmaxf(sqrtf(part == 0 ? ss + other : other + ss), 1e-12f);
+  if (live) {
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      float x[8];
+      unpack_bf16x8(s4[j], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = silu_f(x[e]) * inv;
+      st_bf16x8(dst + part * (DK / 2) + j * 8, x);
+    }
+  }
+}
+
 template <int C, int DK, bool GATED, bool PRE>
 __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
                   const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
                   __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out,
-                  __nv_bfloat16* __restrict__ khat, int T, int nchunks, unsigned int* status) {
+                  __nv_bfloat16* __restrict__ khat, const __nv_bfloat16* __restrict__ qraw,
+                  __nv_bfloat16* __restrict__ qhat, int T, int nchunks, unsigned int* status) {
   using Sh = TsolveShape<C>;
   using SL = TsolveSmem<C, DK>;
   constexpr int kC = C, kApad = Sh::kApad;
@@ -154,6 +191,9 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     if (ok)
       prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, r, tid & 1,
                             r < n ? khat + ((size_t)bh * T + c0 + r) * DK : nullptr);
+    // and on the chunk's queries, global to global (the chunk kernel reads them there)
+    const size_t qrow = ((size_t)bh * T + c0 + min(r, n - 1)) * DK;
+    prestep_row_global<DK>(qraw + qrow, qhat + qrow, r < n, tid & 1);
     fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
   }
@@ -422,7 +462,8 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((size_t)nchunks * p.B * p.H));  // at most INT_MAX (checked by the caller)
-  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, w.khat, p.T,
+  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, w.khat,
+                                                      static_cast<const __nv_bfloat16*>(p.q), w.qhat, p.T,
                                                       nchunks, p.status);
   return cudaGetLastError();
 }
@@ -449,9 +490,12 @@ size_t wy_workspace_bytes(int B, int H, int T, int C) {
   return tiles * (2 * (size_t)C * C * 2 + (size_t)C * 4);  // Tb, Tbg (bf16) and g (f32)
 }
 
-size_t wy_khat_bytes(int B, int H, int T, int Dk) { return (size_t)B * H * T * Dk * 2; }
+size_t wy_khat_bytes(int B, int H, int T, int Dk) {
+  const size_t one = ((size_t)B * H * T * Dk * 2 + 255) / 256 * 256;
+  return 2 * one;  // k-hat, then q-hat
+}
 
-WyWorkspace wy_carve(void* base, int B, int H, int T, int C) {
+WyWorkspace wy_carve(void* base, int B, int H, int T, int C, int Dk) {
   const size_t nch = ((size_t)T + C - 1) / C;
   const size_t tiles = (size_t)B * H * nch;
   uint8_t* q = static_cast<uint8_t*>(base);
@@ -459,8 +503,9 @@ WyWorkspace wy_carve(void* base, int B, int H, int T, int C) {
   w.tb = reinterpret_cast<__nv_bfloat16*>(q);
   w.tbg = reinterpret_cast<__nv_bfloat16*>(q + tiles * C * C * 2);
   w.g = reinterpret_cast<float*>(q + 2 * tiles * C * C * 2);
-  // mapped keys (pre-step only): after the factors, on a 256-byte boundary
+  // mapped keys, then queries (pre-step only): after the factors, on 256-byte boundaries
   w.khat = reinterpret_cast<__nv_bfloat16*>(q + (wy_workspace_bytes(B, H, T, C) + 255) / 256 * 256);
+  w.qhat = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(w.khat) + wy_khat_bytes(B, H, T, Dk) / 2);
   return w;
 }
 

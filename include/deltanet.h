@@ -131,9 +131,10 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   scalar gating replaced by per-dimension gating).  alpha must not be NULL.
  *
  * Paths: the options are built for C = 64 (C = 128 gives DN_ERR_UNSUPPORTED).
- * DN_OPT_PRESTEP alone on bf16 inputs runs on the tcgen05 path (the maps are
- * applied to the q and k tiles in shared memory, K identically in the pre-pass
- * and the chunk kernel) with the workspace of deltanet_workspace_bytes; every
+ * DN_OPT_PRESTEP alone on bf16 inputs runs on the tcgen05 path: the pre-pass
+ * maps each chunk's q and k once and writes them to the workspace, where the
+ * chunk kernel reads them (the workspace of deltanet_workspace_bytes plus
+ * 2 * B*H*T*Dk bf16 values); every
  * other combination (per-dimension decay, float32 inputs) runs on the
  * CUDA-core kernel (float32 arithmetic) and needs only the 256-byte status
  * word.  deltanet_workspace_bytes_ex gives the size for each case.  The

@@ -241,10 +241,11 @@ def test_option_flags_are_validated_on_the_host(L):
     # the per-dimension alpha covers B*H*T*Dk floats: an alpha that ends inside o overlaps it
     assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 256 * MB - 2 * 2 * 100 * 64 * 4 + 64) == E.DN_ERR_INVALID_ARG
     # the pre-step alone on bf16 runs on the tcgen05 path: the pre-pass factors,
-    # then (from a 256-byte boundary) the mapped keys, B*H*T*Dk bf16
+    # then (each from a 256-byte boundary) the mapped keys and queries, B*H*T*Dk bf16 each
     base = L.deltanet_workspace_bytes(2, 2, 100, 64, 64, 64, 1)
+    r256 = lambda x: (x + 255) // 256 * 256
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 1) == \
-        256 + (base - 256 + 255) // 256 * 256 + 2 * 2 * 100 * 64 * 2
+        256 + r256(base - 256) + 2 * r256(2 * 2 * 100 * 64 * 2)
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 0, 1) == 256
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 2) == 256
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 3) == 256
