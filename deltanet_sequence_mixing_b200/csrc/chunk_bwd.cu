@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
   };
 
   // T = (I + A)^-1 with A = strict_lower(diag(beta) (K K^T * Gamma)): A into
-  // M1, then forward substitution, one column per thread of warp 0.
+  // M1, then forward substitution, one column per lane of warp 0.
   auto solve_T = [&]() {
     for (int idx = tid; idx < C * C; idx += kThreads) {
       const int r = idx / C, s = idx % C;
@@ -149,20 +149,18 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
       M1[r * CP + s] = acc;
     }
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0) {  // right-looking: each finished element feeds every later row at once
       const int j = lane;
-      for (int i = 0; i < C; ++i) {
-        float t;
-        if (i < j) {
-          t = 0.f;
-        } else if (i == j) {
-          t = 1.f;
-        } else {
-          float acc = 0.f;
-          for (int m = j; m < i; ++m) acc += M1[i * CP + m] * Ts[m * CP + j];
-          t = -acc;
-        }
-        Ts[i * CP + j] = t;
+      float acc[C];
+#pragma unroll
+      for (int i = 0; i < C; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int m = 0; m < C; ++m) {
+        const float cm = m == j ? 1.f : (m > j ? -acc[m] : 0.f);
+        Ts[m * CP + j] = cm;
+#pragma unroll
+        for (int i = 0; i < C; ++i)
+          if (i > m) acc[i] = fmaf(M1[i * CP + m], cm, acc[i]);
       }
     }
     __syncthreads();

@@ -50,6 +50,26 @@ __device__ __forceinline__ float elu_plus_one(float x) { return x > 0.f ? x + 1.
 
 __device__ __forceinline__ float silu(float x) { return x / (1.f + __expf(-x)); }
 
+// Column j of T = (I + A)^-1 for a strictly lower-triangular A (row stride CP),
+// into T.  Right-looking: once element m of the column is final it is pushed
+// into the partial sums of every later row, so the C^2 / 2 multiply-adds are
+// independent of one another except through the one element per step, and
+// the column's partial sums stay in registers (the loops are unrolled).
+template <int C, int CP>
+__device__ __forceinline__ void solve_unit_lower_column(const float* A, float* T, int j) {
+  float acc[C];
+#pragma unroll
+  for (int i = 0; i < C; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int m = 0; m < C; ++m) {
+    const float cm = m == j ? 1.f : (m > j ? -acc[m] : 0.f);
+    T[m * CP + j] = cm;
+#pragma unroll
+    for (int i = 0; i < C; ++i)
+      if (i > m) acc[i] = fmaf(A[i * CP + m], cm, acc[i]);
+  }
+}
+
 // GATE: 0 none, 1 one decay per token (Gamma table), 2 one decay per token and
 // key dimension (a table of the cumulative log decay G, C x DK).
 template <int DK, int DVS, int C, int GATE>
@@ -230,21 +250,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
     }
     __syncthreads();
     // ---- T = (I + A)^-1 by forward substitution, one column per thread ----
-    for (int j = tid; j < C; j += kThreads) {
-      for (int i = 0; i < C; ++i) {
-        float t;
-        if (i < j) {
-          t = 0.f;
-        } else if (i == j) {
-          t = 1.f;
-        } else {
-          float acc = 0.f;
-          for (int m = j; m < i; ++m) acc += Ps[i * CP + m] * Ts[m * CP + j];
-          t = -acc;
-        }
-        Ts[i * CP + j] = t;
-      }
-    }
+    if (tid < C) solve_unit_lower_column<C, CP>(Ps, Ts, tid);
     if constexpr (GATE == 2) {
       // Per-dimension decay (G[r][i] = cumulative log decay of key dimension i
       // within the chunk, non-increasing in r).  Every exponential below has a
