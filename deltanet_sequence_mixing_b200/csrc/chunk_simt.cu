@@ -70,6 +70,36 @@ __device__ __forceinline__ void solve_unit_lower_column(const float* A, float* T
   }
 }
 
+// Register-tiled product for a CTA of 256 threads as a 16 x 16 grid: thread
+// (r0, c0) = (tid / 16, tid % 16) accumulates the 4 x 4 outputs (r0 + 16a,
+// c0 + 16b) of sum_k A(r, k) B(k, c), with A(r, k) = A[r * ars + k * acs] and
+// B(k, c) = B[k * brs + c * bcs].  Four loads of A and four of B feed sixteen
+// multiply-adds (a warp reads two rows of A, broadcast, and sixteen columns of
+// B, on distinct banks for unit or odd strides).
+template <int NK>
+__device__ __forceinline__ void mm44(const float* A, int ars, int acs, const float* B, int brs, int bcs,
+                                     float (&acc)[4][4]) {
+  const int r0 = threadIdx.x >> 4, c0 = threadIdx.x & 15;
+#pragma unroll 4
+  for (int k = 0; k < NK; ++k) {
+    float a[4], b[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) a[x] = A[(r0 + 16 * x) * ars + k * acs];
+#pragma unroll
+    for (int y = 0; y < 4; ++y) b[y] = B[k * brs + (c0 + 16 * y) * bcs];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
+  }
+}
+__device__ __forceinline__ void zero44(float (&acc)[4][4]) {
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+}
+
 // GATE: 0 none, 1 one decay per token (Gamma table), 2 one decay per token and
 // key dimension (a table of the cumulative log decay G, C x DK).
 template <int DK, int DVS, int C, int GATE>
@@ -107,6 +137,163 @@ __device__ void stage_keys(float* X, const TI* src, size_t base, int c0, int n, 
       const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
       for (int i = 0; i < DK; ++i) X[r * KP + i] *= inv;
     }
+  }
+}
+
+// One chunk of the delta rule with a per-dimension decay (G[r][i]: the
+// cumulative log decay of key dimension i within the chunk, non-increasing in
+// r; rows past n have zero inputs and a flat G), entered with the state slice
+// S (DK x DVS) and leaving it updated:
+//   A[r][s] = beta_r sum_i K[r][i] K[s][i] e^(G[r][i] - G[s][i])   (s < r),  T = (I + A)^-1
+//   P[r][s] = sum_i Q[r][i] K[s][i] e^(G[r][i] - G[s][i])          (s <= r)
+//   X = V - (K * e^G) S,   U = T diag(beta) X,   O = (Q * e^G) S + P U
+//   S <- diag(e^G[n-1]) S + (K * e^(G[n-1] - G))^T U
+// While each dimension's decay range within the chunk stays below 160 (in log
+// space), e^(G_r - G_s) = e^(G_r - m) e^(m - G_s) about the dimension's midpoint
+// m splits into row and column factors that stay within e^(+-80), and A and P
+// become plain products of scaled tiles; past that, one exponential per term.
+// Every other exponential has a non-positive argument.  The smem tables Q, K
+// are reloaded from global memory (L2) where a product needs another scaling.
+template <typename TI, bool PRE, int DK, int DVS, int C>
+__device__ void kda_chunk(float* Qs, float* Ks, float* Vs, float* Us, float* Ss, float* Ts, float* Ps,
+                          const float* Gd, const float* bs, float* ms, const TI* q, const TI* k, TI* o,
+                          size_t qk_base, size_t v_base, int c0, int n, int Dv, int j0) {
+  static_assert(C == 64 && DVS == 64, "the 16 x 16 thread grid covers 64 x 64 tiles");
+  constexpr int KP = DK + 1, VP = DVS + 1, CP = C + 1;
+  const int tid = threadIdx.x, r0 = tid >> 4, cc0 = tid & 15;
+  float acc[4][4];
+  // per-dimension midpoints; the factored form needs every range <= 160
+  bool fact = true;
+  for (int i = tid; i < DK; i += kThreads) {
+    ms[i] = 0.5f * (Gd[i] + Gd[(C - 1) * KP + i]);
+    fact = fact && (Gd[i] - Gd[(C - 1) * KP + i] <= 160.f);
+  }
+  fact = __syncthreads_and(fact);
+  // ---- A ----
+  if (fact) {  // Qs <- K e^(G - m), Ks <- K e^(m - G)
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      const float kv = Ks[r * KP + i], e = Gd[r * KP + i] - ms[i];
+      Qs[r * KP + i] = kv * __expf(e);
+      Ks[r * KP + i] = kv * __expf(-e);
+    }
+    __syncthreads();
+    zero44(acc);
+    mm44<DK>(Qs, KP, 1, Ks, 1, KP, acc);
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int r = r0 + 16 * x, s2 = cc0 + 16 * y;
+        Ps[r * CP + s2] = s2 < r ? bs[r] * acc[x][y] : 0.f;
+      }
+  } else {
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s2 = idx % C;
+      float a = 0.f;
+      if (s2 < r)
+        for (int i = 0; i < DK; ++i)
+          a += Ks[r * KP + i] * Ks[s2 * KP + i] * __expf(Gd[r * KP + i] - Gd[s2 * KP + i]);
+      Ps[r * CP + s2] = bs[r] * a;
+    }
+  }
+  __syncthreads();
+  if (tid < C) solve_unit_lower_column<C, CP>(Ps, Ts, tid);
+  __syncthreads();
+  // ---- P (over A, which the solve has consumed) ----
+  if (fact) {  // Qs <- Q e^(G - m); Ks still holds K e^(m - G)
+    stage_keys<TI, PRE, DK, KP, C>(Qs, q, qk_base, c0, n, false);
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      Qs[r * KP + i] *= __expf(Gd[r * KP + i] - ms[i]);
+    }
+    __syncthreads();
+    zero44(acc);
+    mm44<DK>(Qs, KP, 1, Ks, 1, KP, acc);
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int r = r0 + 16 * x, s2 = cc0 + 16 * y;
+        Ps[r * CP + s2] = s2 <= r ? acc[x][y] : 0.f;
+      }
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += kThreads) {  // Q e^G = (Q e^(G - m)) e^m, m <= 0
+      const int r = idx / DK, i = idx % DK;
+      Qs[r * KP + i] *= __expf(ms[i]);
+    }
+  } else {  // Qs still holds Q
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+      const int r = idx / C, s2 = idx % C;
+      float a = 0.f;
+      if (s2 <= r)
+        for (int i = 0; i < DK; ++i)
+          a += Qs[r * KP + i] * Ks[s2 * KP + i] * __expf(Gd[r * KP + i] - Gd[s2 * KP + i]);
+      Ps[r * CP + s2] = a;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int r = idx / DK, i = idx % DK;
+      Qs[r * KP + i] *= __expf(Gd[r * KP + i]);
+    }
+  }
+  // ---- K e^G, then X = diag(beta) (V - (K e^G) S) in place of V ----
+  stage_keys<TI, PRE, DK, KP, C>(Ks, k, qk_base, c0, n, false);
+  __syncthreads();
+  for (int idx = tid; idx < C * DK; idx += kThreads) {
+    const int r = idx / DK, i = idx % DK;
+    Ks[r * KP + i] *= __expf(Gd[r * KP + i]);
+  }
+  __syncthreads();
+  zero44(acc);
+  mm44<DK>(Ks, KP, 1, Ss, VP, 1, acc);
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int r = r0 + 16 * x, j = cc0 + 16 * y;
+      Vs[r * VP + j] = bs[r] * (Vs[r * VP + j] - acc[x][y]);
+    }
+  __syncthreads();
+  // ---- U = T X ----
+  zero44(acc);
+  mm44<C>(Ts, CP, 1, Vs, VP, 1, acc);
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) Us[(r0 + 16 * x) * VP + cc0 + 16 * y] = acc[x][y];
+  __syncthreads();
+  // ---- O = (Q e^G) S + P U ----
+  zero44(acc);
+  mm44<DK>(Qs, KP, 1, Ss, VP, 1, acc);
+  mm44<C>(Ps, CP, 1, Us, VP, 1, acc);
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int r = r0 + 16 * x;
+      if (r < n) store_out(o, v_base + (size_t)(c0 + r) * Dv + j0 + cc0 + 16 * y, acc[x][y]);
+    }
+  // ---- K e^(G[n-1] - G), then S <- diag(e^G[n-1]) S + (K e^(G[n-1] - G))^T U ----
+  stage_keys<TI, PRE, DK, KP, C>(Ks, k, qk_base, c0, n, false);
+  __syncthreads();
+  for (int idx = tid; idx < C * DK; idx += kThreads) {
+    const int r = idx / DK, i = idx % DK;
+    Ks[r * KP + i] *= __expf(Gd[(n - 1) * KP + i] - Gd[r * KP + i]);
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int h = 0; h < DK / 64; ++h) {  // rows i of S in blocks of 64
+    zero44(acc);
+    mm44<C>(Ks + 64 * h, 1, KP, Us, VP, 1, acc);
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int i = 64 * h + r0 + 16 * x, j = cc0 + 16 * y;
+        Ss[i * VP + j] = __expf(Gd[(n - 1) * KP + i]) * Ss[i * VP + j] + acc[x][y];
+      }
   }
 }
 
@@ -232,17 +419,17 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
       }
       __syncthreads();
     }
+    if constexpr (GATE == 2) {
+      kda_chunk<TI, PRE, DK, DVS, C>(Qs, Ks, Vs, Us, Ss, Ts, Ps, Gd, bs, zs, q, k, o, qk_base, v_base, c0, n,
+                                     Dv, j0);
+      continue;
+    }
     // ---- A = strict_lower(diag(beta) (K K^T * Gamma)) ----
     for (int idx = tid; idx < C * C; idx += kThreads) {
       const int r = idx / C, s = idx % C;
       float acc = 0.f;
       if (s < r) {
-        if (GATE == 2) {
-          for (int i = 0; i < DK; ++i)
-            acc += Ks[r * KP + i] * Ks[s * KP + i] * __expf(Gd[r * KP + i] - Gd[s * KP + i]);
-        } else {
-          for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
-        }
+        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
         acc *= bs[r];
         if (GATED) acc *= Gm[r * CP + s];
       }
@@ -251,69 +438,6 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(const ChunkProblem
     __syncthreads();
     // ---- T = (I + A)^-1 by forward substitution, one column per thread ----
     if (tid < C) solve_unit_lower_column<C, CP>(Ps, Ts, tid);
-    if constexpr (GATE == 2) {
-      // Per-dimension decay (G[r][i] = cumulative log decay of key dimension i
-      // within the chunk, non-increasing in r).  Every exponential below has a
-      // non-positive argument, so nothing overflows:
-      //   P[r][s] = sum_i Q[r][i] K[s][i] e^(G[r][i] - G[s][i])      (s <= r)
-      //   X = V - (K * e^G) S,   U = T diag(beta) X
-      //   O = (Q * e^G) S + P U
-      //   S = diag(e^G[n-1]) S + (K * e^(G[n-1] - G))^T U
-      __syncthreads();  // T is complete; A in Ps may be overwritten
-      for (int idx = tid; idx < C * C; idx += kThreads) {
-        const int r = idx / C, s2 = idx % C;
-        float acc = 0.f;
-        if (s2 <= r)
-          for (int i = 0; i < DK; ++i)
-            acc += Qs[r * KP + i] * Ks[s2 * KP + i] * __expf(Gd[r * KP + i] - Gd[s2 * KP + i]);
-        Ps[r * CP + s2] = acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < C * DK; idx += kThreads) {  // Q, K -> Q e^G, K e^G
-        const int r = idx / DK, i = idx % DK;
-        const float e = __expf(Gd[r * KP + i]);
-        Qs[r * KP + i] *= e;
-        Ks[r * KP + i] *= e;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < C * DVS; idx += kThreads) {
-        const int r = idx / DVS, j = idx % DVS;
-        float acc = 0.f;
-        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ss[i * VP + j];
-        Vs[r * VP + j] -= acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < C * DVS; idx += kThreads) {
-        const int r = idx / DVS, j = idx % DVS;
-        float acc = 0.f;
-        for (int s2 = 0; s2 <= r; ++s2) acc += Ts[r * CP + s2] * bs[s2] * Vs[s2 * VP + j];
-        Us[r * VP + j] = acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < C * DVS; idx += kThreads) {
-        const int r = idx / DVS, j = idx % DVS;
-        if (r >= n) continue;
-        float acc = 0.f;
-        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ss[i * VP + j];
-        for (int s2 = 0; s2 <= r; ++s2) acc += Ps[r * CP + s2] * Us[s2 * VP + j];
-        store_out(o, v_base + (size_t)(c0 + r) * Dv + j0 + j, acc);
-      }
-      // K again, weighted for the state update: K[s][i] e^(G[n-1][i] - G[s][i])
-      stage_keys<TI, PRE, DK, KP, C>(Ks, k, qk_base, c0, n, false);
-      __syncthreads();
-      for (int idx = tid; idx < C * DK; idx += kThreads) {
-        const int r = idx / DK, i = idx % DK;
-        Ks[r * KP + i] *= __expf(Gd[(n - 1) * KP + i] - Gd[r * KP + i]);
-      }
-      __syncthreads();
-      for (int idx = tid; idx < DK * DVS; idx += kThreads) {
-        const int i = idx / DVS, j = idx % DVS;
-        float acc = 0.f;
-        for (int s2 = 0; s2 < n; ++s2) acc += Ks[s2 * KP + i] * Us[s2 * VP + j];
-        Ss[i * VP + j] = __expf(Gd[(n - 1) * KP + i]) * Ss[i * VP + j] + acc;
-      }
-      continue;
-    }
     // ---- X = V - diag(gamma) K S (in place in Vs) ----
     for (int idx = tid; idx < C * DVS; idx += kThreads) {
       const int r = idx / DVS, j = idx % DVS;
