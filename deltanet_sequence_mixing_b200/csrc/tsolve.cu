@@ -49,7 +49,7 @@ struct TsolveShape {
 // Gram operand's rows 64-127 read whatever follows a block (those TMEM rows are
 // not used).  That keeps the CTA at 26 KB, eight per SM; at C = 128, K and A
 // side by side take 103 KB, two per SM.
-template <int C, int DK>
+template <int C, int DK, bool PRE = false>
 struct TsolveSmem {
   static constexpr uint32_t kKBytes = (DK / 64) * C * 128;
   static constexpr uint32_t kTBytes = C * TsolveShape<C>::kApad * 4;
@@ -57,7 +57,9 @@ struct TsolveSmem {
   static constexpr uint32_t AM_OFF = C == 64 ? 0 : round1k(kKBytes);
   static constexpr uint32_t kRegion =
       C == 64 ? round1k(kTBytes > kKBytes + 8192 ? kTBytes : kKBytes + 8192) : AM_OFF + kTBytes;
-  static constexpr uint32_t VEC_OFF = kRegion;  // beta, g, e^g, e^(m-g) (C each), 8 warp totals
+  // the pre-step maps the chunk's q tile here (TMA, 128-byte swizzle), after the region
+  static constexpr uint32_t QT_OFF = round1k(kRegion);
+  static constexpr uint32_t VEC_OFF = PRE ? QT_OFF + kKBytes : kRegion;  // beta, g, e^g, e^(m-g), 8 warp totals
   static constexpr uint32_t BAR_OFF = (VEC_OFF + (4 * C + 8) * 4 + 7) / 8 * 8;  // FULL, MMA, TMEM slot
   static constexpr uint32_t BYTES = BAR_OFF + 32;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // 1024-byte alignment of the K tile
@@ -74,51 +76,16 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
   for (int t = 0; t < f.num_elements; ++t) f.x[t] = __uint_as_float(__float_as_uint(f.x[t]) & 0xFFFFE000u);
 }
 
-// The layer's pre-step on one query row in global memory, two lanes per row
-// (lane parity `part` takes columns [part * DK/2, (part + 1) * DK/2)):
-// dst <- silu(src) / max(||silu(src)||_2, 1e-12).  All 32 lanes of the warp
-// call it (`live` false skips the memory accesses of rows past T).
-template <int DK>
-__device__ __forceinline__ void prestep_row_global(const __nv_bfloat16* src, __nv_bfloat16* dst, bool live,
-                                                   int part) {
-  constexpr int NCH = DK / 16;  // 16-byte chunks per lane
-  const uint4* s4 = reinterpret_cast<const uint4*>(src + part * (DK / 2));
-  float ss = 0.f;
-  if (live) {
-#pragma unroll
-    for (int j = 0; j < NCH; ++j) {
-      float x[8];
-      unpack_bf16x8(s4[j], x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float y = silu_f(x[e]);
-        ss = fmaf(y, y, ss);
-      }
-    }
-  }
-  const float other = __shfl_xor_sync(0xffffffffu, ss, 1);
-  const float inv = 1.f / fmaxf(sqrtf(part == 0 ? ss + other : other + ss), 1e-12f);
-  if (live) {
-#pragma unroll
-    for (int j = 0; j < NCH; ++j) {
-      float x[8];
-      unpack_bf16x8(s4[j], x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = silu_f(x[e]) * inv;
-      st_bf16x8(dst + part * (DK / 2) + j * 8, x);
-    }
-  }
-}
-
 template <int C, int DK, bool GATED, bool PRE>
 __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     tsolve_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ beta,
-                  const float* __restrict__ alpha, __nv_bfloat16* __restrict__ tb_out,
+                  const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ alpha,
+                  __nv_bfloat16* __restrict__ tb_out,
                   __nv_bfloat16* __restrict__ tbg_out, float* __restrict__ g_out,
-                  __nv_bfloat16* __restrict__ khat, const __nv_bfloat16* __restrict__ qraw,
-                  __nv_bfloat16* __restrict__ qhat, int T, int nchunks, unsigned int* status) {
+                  __nv_bfloat16* __restrict__ khat, __nv_bfloat16* __restrict__ qhat, int T, int nchunks,
+                  unsigned int* status) {
   using Sh = TsolveShape<C>;
-  using SL = TsolveSmem<C, DK>;
+  using SL = TsolveSmem<C, DK, PRE>;
   constexpr int kC = C, kApad = Sh::kApad;
   extern __shared__ uint8_t tsolve_smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsolve_smem_raw) + 1023) &
@@ -159,12 +126,14 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
   const uint32_t tmem = warp_uniform(*tmem_slot);
   const WaitCtl wc{abort_flag, status, kWaitLimitNs};
   if (tid == 0) {
-    mbar_expect_tx(bar_full, (uint32_t)SL::kKBytes);
+    mbar_expect_tx(bar_full, (uint32_t)SL::kKBytes * (PRE ? 2 : 1));
 #pragma unroll
     for (int kb = 0; kb < DK / 64; ++kb)
 #pragma unroll
-      for (int rb = 0; rb < kC / 64; ++rb)
+      for (int rb = 0; rb < kC / 64; ++rb) {
         tma_load_3d(sb + kb * (kC * 128) + rb * 8192, &tmK, bar_full, kb * 64, c0 + rb * 64, bh);
+        if (PRE) tma_load_3d(sb + SL::QT_OFF + kb * (kC * 128) + rb * 8192, &tmQ, bar_full, kb * 64, c0 + rb * 64, bh);
+      }
   }
   float glog = 0.f;
   if (tid < kC) {
@@ -188,12 +157,12 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     // mapped rows also go to the workspace, where the chunk kernel reads them.
     ok = __all_sync(0xffffffffu, mbar_wait(bar_full, 0, wc));  // warp-uniform for the shuffles
     const int r = tid >> 1;
-    if (ok)
-      prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, r, tid & 1,
-                            r < n ? khat + ((size_t)bh * T + c0 + r) * DK : nullptr);
-    // and on the chunk's queries, global to global (the chunk kernel reads them there)
-    const size_t qrow = ((size_t)bh * T + c0 + min(r, n - 1)) * DK;
-    prestep_row_global<DK>(qraw + qrow, qhat + qrow, r < n, tid & 1);
+    if (ok) {
+      const size_t row = ((size_t)bh * T + c0 + r) * DK;
+      prestep_row_sw128<DK>(sm, (uint32_t)kC * 128, r, tid & 1, r < n ? khat + row : nullptr);
+      // and on the chunk's queries (the chunk kernel reads both from the workspace)
+      prestep_row_sw128<DK>(sm + SL::QT_OFF, (uint32_t)kC * 128, r, tid & 1, r < n ? qhat + row : nullptr);
+    }
     fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
   }
@@ -455,16 +424,16 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
 template <int C, int DK, bool GATED>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   const int nchunks = (p.T + C - 1) / C;
-  constexpr size_t smem = TsolveSmem<C, DK>::ALLOC;
-  CUtensorMap mk;
-  if (!make_tmap_3d_bf16(&mk, p.k, DK, p.T, p.B * p.H)) return cudaErrorInvalidValue;
+  const size_t smem = p.prestep ? TsolveSmem<C, DK, true>::ALLOC : TsolveSmem<C, DK, false>::ALLOC;
+  CUtensorMap mk, mq;
+  if (!make_tmap_3d_bf16(&mk, p.k, DK, p.T, p.B * p.H) || !make_tmap_3d_bf16(&mq, p.q, DK, p.T, p.B * p.H))
+    return cudaErrorInvalidValue;
   auto kern = p.prestep ? tsolve_kernel<C, DK, GATED, true> : tsolve_kernel<C, DK, GATED, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((size_t)nchunks * p.B * p.H));  // at most INT_MAX (checked by the caller)
-  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, p.alpha, w.tb, w.tbg, w.g, w.khat,
-                                                      static_cast<const __nv_bfloat16*>(p.q), w.qhat, p.T,
-                                                      nchunks, p.status);
+  kern<<<grid, TsolveShape<C>::kThreads, smem, st>>>(mk, p.beta, mq, p.alpha, w.tb, w.tbg, w.g, w.khat, w.qhat,
+                                                      p.T, nchunks, p.status);
   return cudaGetLastError();
 }
 
