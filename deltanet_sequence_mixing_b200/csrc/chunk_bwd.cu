@@ -51,12 +51,41 @@ __device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16* p, size_
   return __bfloat162float(p[i]);
 }
 
+// Register-tiled product for the CTA's 256 threads as a 16 x 16 grid: thread
+// (r0, c0) = (tid / 16, tid % 16) accumulates the RX x RY outputs
+// (r0 + 16x, c0 + 16y) of sum_{k < nk} A(r, k) B(k, c), A(r, k) = A[r * ars + k * acs],
+// B(k, c) = B[k * brs + c * bcs].  RX + RY loads feed RX * RY multiply-adds.
+template <int RX, int RY>
+__device__ __forceinline__ void mmt(int nk, const float* A, int ars, int acs, const float* B, int brs, int bcs,
+                                    float (&acc)[RX][RY]) {
+  const int r0 = threadIdx.x >> 4, c0 = threadIdx.x & 15;
+#pragma unroll 2
+  for (int k = 0; k < nk; ++k) {
+    float a[RX], b[RY];
+#pragma unroll
+    for (int x = 0; x < RX; ++x) a[x] = A[(r0 + 16 * x) * ars + k * acs];
+#pragma unroll
+    for (int y = 0; y < RY; ++y) b[y] = B[k * brs + (c0 + 16 * y) * bcs];
+#pragma unroll
+    for (int x = 0; x < RX; ++x)
+#pragma unroll
+      for (int y = 0; y < RY; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
+  }
+}
+template <int RX, int RY>
+__device__ __forceinline__ void zero_acc(float (&acc)[RX][RY]) {
+#pragma unroll
+  for (int x = 0; x < RX; ++x)
+#pragma unroll
+    for (int y = 0; y < RY; ++y) acc[x][y] = 0.f;
+}
+
 template <int DK>
 struct BwdSmem {
   static constexpr int KP = DK + 1;
   static constexpr int kFloats = 2 * C * KP      // Q, K
                                  + 2 * DK * VP   // S, dS
-                                 + 7 * C * VP    // V, dO, KS, X, U, dU, dBV
+                                 + 9 * C * VP    // V, dO, KS, X, U, dU, dBV, QS, KD
                                  + 3 * C * CP    // T, M1, M2
                                  + 8 * C;        // beta, g, gamma, e_out, dg, dbeta, red, spare
   static constexpr size_t kBytes = sizeof(float) * kFloats;
@@ -78,7 +107,9 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
   float* Us = Xs + C * VP;
   float* dUs = Us + C * VP;
   float* dBVs = dUs + C * VP;
-  float* Ts = dBVs + C * VP;
+  float* QSs = dBVs + C * VP;  // Q S (reverse sweep), e_out U (forward sweep)
+  float* KDs = QSs + C * VP;   // K dS+
+  float* Ts = KDs + C * VP;
   float* M1 = Ts + C * CP;
   float* M2 = M1 + C * CP;
   float* bs = M2 + C * CP;
@@ -90,6 +121,7 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
   float* red = db + C;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tr = tid >> 4, tc = tid & 15;  // this thread's place in the 16 x 16 grid of mmt
   const int bh = blockIdx.x, slice = blockIdx.y, j0 = slice * DVS;
   const int T = p.T, Dv = p.Dv, nch = (T + C - 1) / C;
   const TI* q = static_cast<const TI*>(p.q);
@@ -139,14 +171,17 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
   // T = (I + A)^-1 with A = strict_lower(diag(beta) (K K^T * Gamma)): A into
   // M1, then forward substitution, one column per lane of warp 0.
   auto solve_T = [&]() {
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      float acc = 0.f;
-      if (s < r) {
-        for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ks[s * KP + i];
-        acc *= bs[r] * gamma_rs(r, s);
-      }
-      M1[r * CP + s] = acc;
+    {
+      float acc[2][2];
+      zero_acc(acc);
+      mmt<2, 2>(DK, Ks, KP, 1, Ks, 1, KP, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int r = tr + 16 * x, s2 = tc + 16 * y;
+          M1[r * CP + s2] = s2 < r ? acc[x][y] * bs[r] * gamma_rs(r, s2) : 0.f;
+        }
     }
     __syncthreads();
     if (warp == 0) {  // right-looking: each finished element feeds every later row at once
@@ -168,19 +203,28 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
 
   // KS = K S, X = diag(beta) (V - diag(gamma) K S), U = T X
   auto forward_u = [&]() {
-    for (int idx = tid; idx < C * DVS; idx += kThreads) {
-      const int r = idx / DVS, j = idx % DVS;
-      float acc = 0.f;
-      for (int i = 0; i < DK; ++i) acc += Ks[r * KP + i] * Ss[i * VP + j];
-      KSs[r * VP + j] = acc;
-      Xs[r * VP + j] = bs[r] * (Vs[r * VP + j] - gam[r] * acc);
+    {
+      float acc[2][4];
+      zero_acc(acc);
+      mmt<2, 4>(DK, Ks, KP, 1, Ss, VP, 1, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int r = tr + 16 * x, j = tc + 16 * y;
+          KSs[r * VP + j] = acc[x][y];
+          Xs[r * VP + j] = bs[r] * (Vs[r * VP + j] - gam[r] * acc[x][y]);
+        }
     }
     __syncthreads();
-    for (int idx = tid; idx < C * DVS; idx += kThreads) {
-      const int r = idx / DVS, j = idx % DVS;
-      float acc = 0.f;
-      for (int s = 0; s <= r; ++s) acc += Ts[r * CP + s] * Xs[s * VP + j];
-      Us[r * VP + j] = acc;
+    {  // T is lower triangular with explicit zeros above the diagonal
+      float acc[2][4];
+      zero_acc(acc);
+      mmt<2, 4>(C, Ts, CP, 1, Xs, VP, 1, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) Us[(tr + 16 * x) * VP + tc + 16 * y] = acc[x][y];
     }
     __syncthreads();
   };
@@ -198,11 +242,22 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
     __syncthreads();
     solve_T();
     forward_u();
-    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
-      const int i = idx / DVS, j = idx % DVS;
-      float acc = 0.f;
-      for (int s = 0; s < C; ++s) acc += eo[s] * Ks[s * KP + i] * Us[s * VP + j];
-      Ss[i * VP + j] = gam[C - 1] * Ss[i * VP + j] + acc;
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {  // e_out U
+      const int r = idx / DVS, j = idx % DVS;
+      QSs[r * VP + j] = eo[r] * Us[r * VP + j];
+    }
+    __syncthreads();
+    {
+      float acc[DK / 16][4];
+      zero_acc(acc);
+      mmt<DK / 16, 4>(C, Ks, 1, KP, QSs, VP, 1, acc);
+#pragma unroll
+      for (int x = 0; x < DK / 16; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int i = tr + 16 * x, j = tc + 16 * y;
+          Ss[i * VP + j] = gam[C - 1] * Ss[i * VP + j] + acc[x][y];
+        }
     }
   }
 
@@ -222,39 +277,60 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
     solve_T();
     forward_u();
     // P = tril(Q K^T) * Gamma into M1
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      float acc = 0.f;
-      if (s <= r) {
-        for (int i = 0; i < DK; ++i) acc += Qs[r * KP + i] * Ks[s * KP + i];
-        acc *= gamma_rs(r, s);
-      }
-      M1[r * CP + s] = acc;
+    {
+      float acc[2][2];
+      zero_acc(acc);
+      mmt<2, 2>(DK, Qs, KP, 1, Ks, 1, KP, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int r = tr + 16 * x, s2 = tc + 16 * y;
+          M1[r * CP + s2] = s2 <= r ? acc[x][y] * gamma_rs(r, s2) : 0.f;
+        }
     }
     __syncthreads();
-    // dU = P^T dO + diag(e_out) K dS+
-    for (int idx = tid; idx < C * DVS; idx += kThreads) {
-      const int r = idx / DVS, j = idx % DVS;
-      float acc = 0.f;
-      for (int t = r; t < C; ++t) acc += M1[t * CP + r] * dOs[t * VP + j];
-      float ks = 0.f;
-      for (int i = 0; i < DK; ++i) ks += Ks[r * KP + i] * dSs[i * VP + j];
-      dUs[r * VP + j] = acc + eo[r] * ks;
+    // KD = K dS+, QS = Q S, then dU = P^T dO + diag(e_out) KD
+    {
+      float kd[2][4], qs[2][4], pt[2][4];
+      zero_acc(kd);
+      zero_acc(qs);
+      zero_acc(pt);
+      mmt<2, 4>(DK, Ks, KP, 1, dSs, VP, 1, kd);
+      mmt<2, 4>(DK, Qs, KP, 1, Ss, VP, 1, qs);
+      mmt<2, 4>(C, M1, 1, CP, dOs, VP, 1, pt);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int r = tr + 16 * x, j = tc + 16 * y;
+          KDs[r * VP + j] = kd[x][y];
+          QSs[r * VP + j] = qs[x][y];
+          dUs[r * VP + j] = pt[x][y] + eo[r] * kd[x][y];
+        }
     }
     __syncthreads();
     // dP = tril(dO U^T) into M2;  dBV = T^T dU
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      float acc = 0.f;
-      if (s <= r)
-        for (int j = 0; j < DVS; ++j) acc += dOs[r * VP + j] * Us[s * VP + j];
-      M2[r * CP + s] = acc;
+    {
+      float acc[2][2];
+      zero_acc(acc);
+      mmt<2, 2>(DVS, dOs, VP, 1, Us, 1, VP, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int r = tr + 16 * x, s2 = tc + 16 * y;
+          M2[r * CP + s2] = s2 <= r ? acc[x][y] : 0.f;
+        }
     }
-    for (int idx = tid; idx < C * DVS; idx += kThreads) {
-      const int r = idx / DVS, j = idx % DVS;
-      float acc = 0.f;
-      for (int a = r; a < C; ++a) acc += Ts[a * CP + r] * dUs[a * VP + j];
-      dBVs[r * VP + j] = acc;
+    {
+      float acc[2][4];
+      zero_acc(acc);
+      mmt<2, 4>(C, Ts, 1, CP, dUs, VP, 1, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) dBVs[(tr + 16 * x) * VP + tc + 16 * y] = acc[x][y];
     }
     __syncthreads();
     // Per-row sums, one warp per row (lanes over the slice's columns):
@@ -264,15 +340,10 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
     for (int r = warp; r < C; r += kWarps) {
       float t_qs = 0.f, t_bk = 0.f, t_bv = 0.f, t_co = 0.f;
       for (int j = lane; j < DVS; j += 32) {
-        float qs = 0.f, kd = 0.f;
-        for (int i = 0; i < DK; ++i) {
-          qs += Qs[r * KP + i] * Ss[i * VP + j];
-          kd += Ks[r * KP + i] * dSs[i * VP + j];
-        }
-        t_qs += dOs[r * VP + j] * qs;
+        t_qs += dOs[r * VP + j] * QSs[r * VP + j];
         t_bk += dBVs[r * VP + j] * KSs[r * VP + j];
         t_bv += dBVs[r * VP + j] * Vs[r * VP + j];
-        t_co += Us[r * VP + j] * kd;
+        t_co += Us[r * VP + j] * KDs[r * VP + j];
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -314,23 +385,42 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
       for (int s = 0; s < C; ++s) acc += M2[r * CP + s] * M1[r * CP + s] - M2[s * CP + r] * M1[s * CP + r];
       dg[r] += acc;
     }
+    __syncthreads();
+    if (GATED)  // dP * Gamma in place (dq and dk use only that)
+      for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, s2 = idx % C;
+        if (s2 <= r) M2[r * CP + s2] *= gamma_rs(r, s2);
+      }
+    __syncthreads();
     // dq = diag(gamma) dO S^T + (dP * Gamma) K
-    for (int idx = tid; idx < C * DK; idx += kThreads) {
-      const int r = idx / DK, i = idx % DK;
-      if (r >= n) continue;
-      float a = 0.f, b = 0.f;
-      for (int j = 0; j < DVS; ++j) a += dOs[r * VP + j] * Ss[i * VP + j];
-      for (int s = 0; s <= r; ++s) b += M2[r * CP + s] * gamma_rs(r, s) * Ks[s * KP + i];
-      atomicAdd(p.dq + qk_base + (size_t)(c0 + r) * DK + i, gam[r] * a + b);
+#pragma unroll 1
+    for (int h = 0; h < DK / 64; ++h) {  // columns i of dq in blocks of 64
+      float a[2][4], b[2][4];
+      zero_acc(a);
+      zero_acc(b);
+      mmt<2, 4>(DVS, dOs, VP, 1, Ss + 64 * h * VP, 1, VP, a);
+      mmt<2, 4>(C, M2, CP, 1, Ks + 64 * h, KP, 1, b);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int r = tr + 16 * x, i = 64 * h + tc + 16 * y;
+          if (r < n) atomicAdd(p.dq + qk_base + (size_t)(c0 + r) * DK + i, gam[r] * a[x][y] + b[x][y]);
+        }
     }
     __syncthreads();
     // dT = dU X^T (strictly lower part: only it reaches dA), into M1
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      float acc = 0.f;
-      if (s < r)
-        for (int j = 0; j < DVS; ++j) acc += dUs[r * VP + j] * Xs[s * VP + j];
-      M1[r * CP + s] = acc;
+    {
+      float acc[2][2];
+      zero_acc(acc);
+      mmt<2, 2>(DVS, dUs, VP, 1, Xs, 1, VP, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int r = tr + 16 * x, s2 = tc + 16 * y;
+          M1[r * CP + s2] = s2 < r ? acc[x][y] : 0.f;
+        }
     }
     __syncthreads();
     // Y = dT T^T, row by row in place (row a of Y needs only row a of dT)
@@ -353,15 +443,17 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
     }
     __syncthreads();
     // E = dA * MA into Ts (T is no longer needed), MA = K K^T * Gamma
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      float e = 0.f;
-      if (s < r) {
-        float kk = 0.f;
-        for (int i = 0; i < DK; ++i) kk += Ks[r * KP + i] * Ks[s * KP + i];
-        e = M1[r * CP + s] * kk * gamma_rs(r, s);
-      }
-      Ts[r * CP + s] = e;
+    {
+      float acc[2][2];
+      zero_acc(acc);
+      mmt<2, 2>(DK, Ks, KP, 1, Ks, 1, KP, acc);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int r = tr + 16 * x, s2 = tc + 16 * y;
+          Ts[r * CP + s2] = s2 < r ? M1[r * CP + s2] * acc[x][y] * gamma_rs(r, s2) : 0.f;
+        }
     }
     __syncthreads();
     // dbeta += rowsum(dA * MA);  dg += beta_r rowsum(E) - sum_t beta_t E[t][r];
@@ -377,26 +469,36 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
       if (GATED) dg[r] += bs[r] * rs - cs;
     }
     __syncthreads();
+    // (dMA * Gamma) + its transpose into Ts (E is no longer needed), dMA = diag(beta) dA
     for (int idx = tid; idx < C * C; idx += kThreads) {
-      const int r = idx / C, s = idx % C;
-      M1[r * CP + s] *= bs[r];
+      const int r = idx / C, s2 = idx % C;
+      float m = 0.f;
+      if (s2 < r) m = bs[r] * M1[r * CP + s2] * gamma_rs(r, s2);
+      if (r < s2) m = bs[s2] * M1[s2 * CP + r] * gamma_rs(s2, r);
+      Ts[r * CP + s2] = m;
     }
     __syncthreads();
     // dk = (dP * Gamma)^T Q + diag(e_out) U dS+^T - diag(beta gamma) dBV S^T
-    //      + (dMA * Gamma) K + (dMA * Gamma)^T K
-    for (int idx = tid; idx < C * DK; idx += kThreads) {
-      const int s = idx / DK, i = idx % DK;
-      if (s >= n) continue;
-      float a = 0.f, u = 0.f, bv = 0.f, m = 0.f;
-      for (int r = s; r < C; ++r) a += M2[r * CP + s] * gamma_rs(r, s) * Qs[r * KP + i];
-      for (int j = 0; j < DVS; ++j) {
-        u += Us[s * VP + j] * dSs[i * VP + j];
-        bv += dBVs[s * VP + j] * Ss[i * VP + j];
-      }
-      for (int t = 0; t < s; ++t) m += M1[s * CP + t] * gamma_rs(s, t) * Ks[t * KP + i];
-      for (int r = s + 1; r < C; ++r) m += M1[r * CP + s] * gamma_rs(r, s) * Ks[r * KP + i];
-      atomicAdd(p.dk + qk_base + (size_t)(c0 + s) * DK + i,
-                a + eo[s] * u - bs[s] * gam[s] * bv + m);
+    //      + ((dMA * Gamma) + (dMA * Gamma)^T) K
+#pragma unroll 1
+    for (int h = 0; h < DK / 64; ++h) {  // columns i of dk in blocks of 64
+      float pl[2][4], ue[2][4], bg[2][4];
+      zero_acc(pl);
+      zero_acc(ue);
+      zero_acc(bg);
+      mmt<2, 4>(C, M2, 1, CP, Qs + 64 * h, KP, 1, pl);
+      mmt<2, 4>(C, Ts, CP, 1, Ks + 64 * h, KP, 1, pl);
+      mmt<2, 4>(DVS, Us, VP, 1, dSs + 64 * h * VP, 1, VP, ue);
+      mmt<2, 4>(DVS, dBVs, VP, 1, Ss + 64 * h * VP, 1, VP, bg);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int s2 = tr + 16 * x, i = 64 * h + tc + 16 * y;
+          if (s2 < n)
+            atomicAdd(p.dk + qk_base + (size_t)(c0 + s2) * DK + i,
+                      pl[x][y] + eo[s2] * ue[x][y] - bs[s2] * gam[s2] * bg[x][y]);
+        }
     }
     // dv = diag(beta) dBV (this slice's columns: a plain store)
     for (int idx = tid; idx < C * DVS; idx += kThreads) {
@@ -419,13 +521,26 @@ __global__ void __launch_bounds__(kThreads) chunk_bwd_kernel(const BwdProblem p)
       }
     }
     __syncthreads();
-    // dS = (diag(gamma) Q)^T dO + gamma_n dS+ - K^T diag(beta gamma) dBV, in place
-    for (int idx = tid; idx < DK * DVS; idx += kThreads) {
-      const int i = idx / DVS, j = idx % DVS;
-      float acc = gam[C - 1] * dSs[i * VP + j];
-      for (int r = 0; r < C; ++r)
-        acc += gam[r] * (Qs[r * KP + i] * dOs[r * VP + j] - bs[r] * Ks[r * KP + i] * dBVs[r * VP + j]);
-      dSs[i * VP + j] = acc;
+    // dS = Q^T diag(gamma) dO + gamma_n dS+ - K^T diag(beta gamma) dBV, in place;
+    // the row scales go onto dO and dBV first (neither is read again this chunk)
+    for (int idx = tid; idx < C * DVS; idx += kThreads) {
+      const int r = idx / DVS, j = idx % DVS;
+      dOs[r * VP + j] *= gam[r];
+      dBVs[r * VP + j] *= -bs[r] * gam[r];
+    }
+    __syncthreads();
+    {
+      float acc[DK / 16][4];
+      zero_acc(acc);
+      mmt<DK / 16, 4>(C, Qs, 1, KP, dOs, VP, 1, acc);
+      mmt<DK / 16, 4>(C, Ks, 1, KP, dBVs, VP, 1, acc);
+#pragma unroll
+      for (int x = 0; x < DK / 16; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int i = tr + 16 * x, j = tc + 16 * y;
+          dSs[i * VP + j] = gam[C - 1] * dSs[i * VP + j] + acc[x][y];
+        }
     }
   }
   __syncthreads();
