@@ -7,7 +7,7 @@
 // snippet of "How a Baseten Engineer Traced 7 Years of Attention Mechanism
 // Evolution"), with the normaliser z carried like S.  Per chunk c of 64 rows
 // (Q' = ELU(Q) + 1, K' = ELU(K) + 1, rows past T zero), entered with S, z:
-//   P = tril(Q' K'^T)                                (M = 128 MMA [K'; Q'] K'^T)
+//   P = tril(Q' K'^T)
 //   O = (Q' S + P V) / (Q' z + P 1)                  (Q'S + PV in one TMEM tile)
 //   S <- S + K'^T V,  z <- z + K'^T 1
 // The normaliser rides along in the products: V is augmented with a column of
@@ -16,17 +16,23 @@
 // denominator.  Only S and z carry from chunk to chunk, and their increment
 // does not depend on them, so everything but the accumulate is pipelined ahead.
 //
-// One CTA per (b, h, 64-column slice of Dv), 14 warps:
-//   warp 12    producer: TMA of K, Q, V into a three-stage ring
-//   warp 13    MMA issuer (warp-uniform, one elected lane): Gram (c+1) and
-//              K'^T [V|1] (c+1) while chunk c waits for its state tile, then
-//              O (c) = Q'[S|z] + P[V|1]
-//   warps 4-11 prep: feature maps in place (rows past T zeroed)
-//   warps 0-3  state: [S|z] += K'^T [V|1] in float32 registers, the bf16
-//              state tile for the next chunk (double-buffered); warps 2-3 turn
-//              the Gram rows (TMEM lanes 64-127) into P; warps 0-1 drain
-//              O / (Q'z + P 1) to global memory
-// Accumulators live in TMEM (G[2], dS[2], O[2]: 448 of 512 columns).  Every
+// One CTA per (b, h, 64-column slice of Dv), 18 warps, each role on warps of
+// its own so that the per-chunk steps of different roles overlap:
+//   warp 16     producer: TMA of K, Q, V into a three-stage ring
+//   warp 17     MMA issuer (warp-uniform, one elected lane), per chunk c:
+//               Gram (c+1), O (c) = Q'[S|z] + P[V|1] once chunk c's state and
+//               P tiles are ready, then dS (c+1) = K'^T [V|1] (c+1)
+//   warps 4-11  prep: feature maps in place (rows past T zeroed)
+//   warps 0-3   state: [S|z] += K'^T [V|1] in float32 registers, then the
+//               bf16 state tile for the next chunk (double-buffered)
+//   warps 12-15 P and O: per chunk c, the Gram rows to the bf16 P tile (c),
+//               then O (c-1) / (Q'z + P 1) to a bf16 staging tile, stored to
+//               global memory by TMA (double-buffered)
+// The 64-row products (Q'K'^T, Q'[S|z] + P[V|1]) are M = 64 MMAs: their left
+// operands are the 64-row Q' and P tiles alone, and their accumulators hold
+// row r on TMEM lane 32 (r / 16) + r % 16, so each of warps 12-15 owns 16
+// rows.  Accumulators live in TMEM (G[2], dS[2], O[2]: 448 of 512 columns).
+// Every
 // mbarrier completes once per chunk or per use of a parity, so parity waits
 // are unambiguous.  All waits are bounded; a wait that runs out sets the
 // status word and the CTA winds down (copies drained, MMAs retired, TMEM
@@ -46,11 +52,12 @@ constexpr int NST = 3;
 constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
 constexpr int kWG = 128;
 constexpr int kPrep = 256;                  // prep threads (warps 4-11)
-constexpr int kThreads = kWG + kPrep + 64;  // state 0-3, prep 4-11, producer 12, issuer 13
-constexpr int kBarState = 1, kBarLo = 2, kBarHi = 3, kBarPrep = 4;
+constexpr int kThreads = kWG + kPrep + 192;  // state 0-3, prep 4-11, P and O 12-15, producer 16, issuer 17
+constexpr int kWarpProducer = 16, kWarpIssuer = 17;
+constexpr int kBarState = 1, kBarPO = 2, kBarPrep = 4;
 constexpr int kNA = 80;  // augmented width: 64 columns of V (or S) + the ones (or z) column, padded to 16
 
-// TMEM columns: Gram[2] (lanes 64-127: Q'K'^T), dS[2] (K'^T [V|1]), O[2] (lanes 0-63)
+// TMEM columns: Gram[2] (Q'K'^T), dS[2] (K'^T [V|1]), O[2]
 constexpr uint32_t TM_G = 0, TM_DS = 128, TM_O = 320, kAugStride = 96;
 
 template <int DK>
@@ -65,7 +72,8 @@ struct LinLayout {
   // bf16 [S | z] tiles [2]: block 0 = S (DK rows x 128 B), block 1 = z in column 0
   static constexpr uint32_t SBLK = DK * 128;
   static constexpr uint32_t S_OFF = P_OFF + 2 * kTile;
-  static constexpr uint32_t BAR_OFF = S_OFF + 4 * SBLK;
+  static constexpr uint32_t OST_OFF = S_OFF + 4 * SBLK;  // O staging tiles [2] for the TMA store
+  static constexpr uint32_t BAR_OFF = OST_OFF + 2 * kTile;
   static constexpr uint32_t BYTES = BAR_OFF + 256;
   static constexpr uint32_t ALLOC = BYTES + 1024;
   static_assert(STAGE % 1024 == 0 && P_OFF % 1024 == 0, "128-byte swizzle atoms stay aligned");
@@ -79,6 +87,26 @@ __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
   return r;
 }
 
+// ELU(x) + 1 = max(x, 0) + 2^(min(x, 0) log2(e)) on a pair of bf16 values, in
+// bf16 arithmetic: the result is a bf16 MMA operand, and a pair costs six
+// instructions (one of them the exponential for both halves) instead of a
+// float32 round trip per element.  log2(e) is split into two bf16 constants
+// (1.4453125 - 0.00262451171875, within 5e-6 of it) so the exponent argument
+// is the exactly rounded product; the argument's own bf16 rounding leaves the
+// mapped values within 1.4 % (relative, largest for the most negative inputs)
+// of the exact map, against 0.4 % for rounding the exact map to bf16.
+__device__ __forceinline__ uint32_t elu1_bf16x2(uint32_t x) {
+  constexpr uint32_t kZero = 0u, kOne = 0x3F803F80u, kL1 = 0x3FB93FB9u, kL2 = 0xBB2CBB2Cu;
+  uint32_t m, u, t, e, pos, r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(x), "r"(kZero));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(u) : "r"(m), "r"(kL2), "r"(kZero));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(t) : "r"(m), "r"(kL1), "r"(u));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(t));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(pos) : "r"(x), "r"(kZero));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(pos), "r"(kOne), "r"(e));
+  return r;
+}
+
 // mbarrier slots (8 bytes each).  FULL, EMPTY and FMAP per stage; the rest per
 // chunk parity.
 constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_FMAP = 48, B_GDONE = 72, B_DSDONE = 88, B_PREADY = 104,
@@ -88,7 +116,8 @@ constexpr uint32_t B_FULL = 0, B_EMPTY = 24, B_FMAP = 48, B_GDONE = 72, B_DSDONE
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const ChunkProblem p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const ChunkProblem p) {
   using L = LinLayout<DK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -146,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   auto stage = [&](int c) { return sb + (c % NST) * L::STAGE; };
 
-  if (warp == 12) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -180,61 +209,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = issued > NST ? issued - NST : 0; c < issued; ++c)
         (void)mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, drain);
     }
-  } else if (warp == 13) {
+  } else if (warp == kWarpIssuer) {
     // -------------------------------------------------------------- issuer --
-    // Gram (c) = [K'; Q'] K'^T into G[c & 1] and dS (c) = K'^T V into dS[c & 1]
-    auto issue_gram_ds = [&](int c) {
+    // Descriptors are formed once per product and stepped by adding the byte
+    // offset / 16 to the start-address field (no carry: shared memory ends
+    // below 2^18 bytes), which keeps the single issuing warp's instruction
+    // count per MMA low while it shares its scheduler with busy warps.
+    // Gram (c) = Q' K'^T into G[c & 1] (M = 64)
+    auto issue_gram = [&](int c) {
       const uint32_t st = stage(c);
       const int b = c & 1;
-      constexpr uint32_t idg = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idg = idesc_bf16(64, 64, false, false);
+      const uint64_t dq = desc_k(st + L::Q_OFF), dk = desc_k(st + L::K_OFF);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::K_OFF + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem + TM_G + 64 * b, desc_k(a), desc_k(a), idg, ks > 0);
+        constexpr uint32_t kOff[4] = {0, 2, 4, 6};
+        const uint64_t off = (uint64_t)((ks >> 2) * (L::KB_STRIDE >> 4) + kOff[ks & 3]);
+        mma_bf16_ss_elect(tmem + TM_G + 64 * b, dq + off, dk + off, idg, ks > 0);
       }
       mma_commit_elect(bar + B_GDONE + 8 * b);
+    };
+    // dS (c) = K'^T [V|1] into dS[c & 1]
+    auto issue_ds = [&](int c) {
+      const uint32_t st = stage(c);
+      const int b = c & 1;
       constexpr uint32_t idd = idesc_bf16(128, kNA, true, true);
       const uint32_t ones_lbo = sb + L::ONES_OFF - (st + L::V_OFF);  // [V | 1]: the ones block follows V
+      const uint64_t da = desc_mn(st + L::K_OFF, L::KB_STRIDE), dv = desc_mn(st + L::V_OFF, ones_lbo);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_DS + kAugStride * b, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                          desc_mn(st + L::V_OFF + ks * 2048, ones_lbo), idd, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_DS + kAugStride * b, da + (uint64_t)(ks * 128), dv + (uint64_t)(ks * 128), idd,
+                          ks > 0);
       mma_commit_elect(bar + B_DSDONE + 8 * b);
     };
-    // O (c) = Q' [S|z] + P [V|1] into O[c & 1] (lanes 0-63)
+    // O (c) = Q' [S|z] + P [V|1] into O[c & 1] (M = 64)
     auto issue_o = [&](int c) {
       const uint32_t st = stage(c);
       const int b = c & 1;
-      constexpr uint32_t ido = idesc_bf16(128, kNA, false, true);
+      constexpr uint32_t ido = idesc_bf16(64, kNA, false, true);
       const uint32_t ones_lbo = sb + L::ONES_OFF - (st + L::V_OFF);
+      const uint64_t dq = desc_k(st + L::Q_OFF), ds = desc_mn(sb + L::S_OFF + b * 2 * L::SBLK, L::SBLK);
+      const uint64_t dp = desc_k(sb + L::P_OFF + b * kTile), dv = desc_mn(st + L::V_OFF, ones_lbo);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_k(a),
-                          desc_mn(sb + L::S_OFF + b * 2 * L::SBLK + ks * 2048, L::SBLK), ido, ks > 0);
+        constexpr uint32_t kOff[4] = {0, 2, 4, 6};
+        const uint64_t off = (uint64_t)((ks >> 2) * (L::KB_STRIDE >> 4) + kOff[ks & 3]);
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, dq + off, ds + (uint64_t)(ks * 128), ido, ks > 0);
       }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_k(sb + L::P_OFF + b * kTile + ks * 32),
-                          desc_mn(st + L::V_OFF + ks * 2048, ones_lbo), ido, 1);
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, dp + (uint64_t)(2 * ks), dv + (uint64_t)(ks * 128), ido, 1);
       mma_commit_elect(bar + B_ODONE + 8 * b);
       mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));  // stage c: Gram, dS and O have read it
     };
+    // Per iteration c: Gram (c+1), then O (c) once chunk c's state and P tiles
+    // are ready, then dS (c+1).  The tensor pipe runs MMAs in issue order, so
+    // Gram (c+1) (all that P (c+1) needs) runs before O (c) and P (c+1)
+    // overlaps O (c); O (c), the last reader of stage c, runs before dS (c+1),
+    // so the ring turns over as soon as the state allows.
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP, 0, wc));  // stage 0, first use
     if (ok) {
       tc_fence_after();
-      issue_gram_ds(0);
+      issue_gram(0);
+      issue_ds(0);
     }
     for (int c = 0; c < nchunks && ok; ++c) {
       const int b = c & 1;
-      if (c + 1 < nchunks) {  // the next chunk's Gram and K'^T V run while chunk c waits for its state
-        // G[(c+1) & 1] was read by the P rows of chunk c-1 (PREADY waited below in
-        // iteration c-1); dS[(c+1) & 1] must have been added to S (DSFREE of chunk c-1)
-        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc) &&
-                                         (c < 1 || mbar_wait(bar + B_DSFREE + 8 * (b ^ 1), ((c - 1) >> 1) & 1, wc)));
+      const bool next = c + 1 < nchunks;
+      // G[(c+1) & 1] was read by the P rows of chunk c-1 (PREADY waited in iteration c-1)
+      if (next) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FMAP + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        issue_gram_ds(c + 1);
+        issue_gram(c + 1);
       }
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar + B_PREADY + 8 * b, (c >> 1) & 1, wc) &&
@@ -243,13 +290,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       issue_o(c);
+      if (next) {  // dS[(c+1) & 1] must have been added to S (DSFREE of chunk c-1)
+        ok = __all_sync(0xffffffffu, c < 1 || mbar_wait(bar + B_DSFREE + 8 * (b ^ 1), ((c - 1) >> 1) & 1, wc));
+        if (!ok) break;
+        tc_fence_after();
+        issue_ds(c + 1);
+      }
     }
     tc_fence_after();  // no MMA may outlive TMEM
     mma_commit_elect(bar + B_FIN);
     int zero = 0;
     const WaitCtl fin{&zero, p.status, kWaitLimitNs};
     (void)mbar_wait(bar + B_FIN, 0, fin);
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------------- prep --
     const int pt = tid - kWG;
     bool ok = true;
@@ -259,9 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = named_bar_and(kBarPrep, kPrep, mbar_wait(bar + B_FULL + 8 * (c % NST), (c / NST) & 1, wc));
       if (!ok) break;
       // ---- feature maps in place: K, Q -> ELU + 1 (rows >= n -> 0) ----
-      // Four 16-byte pieces per thread per round, in stages (all loads, all
-      // exponentials, then the packs and stores) so the exponentials of 32
-      // elements are in flight together.
+      // Four 16-byte pieces per thread per round, loaded together so that
+      // their exponentials are in flight together.
       constexpr int kPieces = L::KB * 2 * (int)(kTile / 16);  // 16-byte pieces of the K and Q tiles
       constexpr int kNpf = 4;
       static_assert(kPieces % (kNpf * kPrep) == 0, "whole rounds of pieces per thread");
@@ -275,28 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t16 = i / (int)(kTile / 16), off = (i % (int)(kTile / 16)) * 16;
           ptr[j] = stp + (t16 >> 1) * L::KB_STRIDE + (t16 & 1) * kTile + off;
           live[j] = (off >> 7) < n;
-          u[j] = live[j] ? *reinterpret_cast<const uint4*>(ptr[j]) : make_uint4(0, 0, 0, 0);
-        }
-        float f[kNpf * 8], ex[kNpf * 8];
-#pragma unroll
-        for (int j = 0; j < kNpf; ++j) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(&u[j]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {  // bf16 pair -> two floats (low element first)
-            f[j * 8 + 2 * e] = __uint_as_float(w[e] << 16);
-            f[j * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-          }
+          u[j] = *reinterpret_cast<const uint4*>(ptr[j]);
         }
 #pragma unroll
-        for (int k = 0; k < kNpf * 8; ++k) ex[k] = __expf(fminf(f[k], 0.f));
-#pragma unroll
         for (int j = 0; j < kNpf; ++j) {
-          uint4 r;
-          uint32_t* w = reinterpret_cast<uint32_t*>(&r);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)  // ELU(x) + 1 = max(x, 0) + e^min(x, 0)
-            w[e] = pack2_bf16(fmaxf(f[j * 8 + 2 * e], 0.f) + ex[j * 8 + 2 * e],
-                              fmaxf(f[j * 8 + 2 * e + 1], 0.f) + ex[j * 8 + 2 * e + 1]);
+          uint4 r = make_uint4(elu1_bf16x2(u[j].x), elu1_bf16x2(u[j].y), elu1_bf16x2(u[j].z),
+                               elu1_bf16x2(u[j].w));
           if (!live[j]) r = make_uint4(0, 0, 0, 0);
           *reinterpret_cast<uint4*>(ptr[j]) = r;
         }
@@ -305,10 +341,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(kBarPrep, kPrep);
       if (pt == 0) mbar_arrive(bar + B_FMAP + 8 * (c % NST));
     }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------- P and O --
+    // Row r of the M = 64 accumulators is lane r % 16 of warp 12 + r / 16.
+    // Per chunk c: P (c) = tril(Q'K'^T) into the bf16 tile P[c & 1] (the O
+    // product that read it two chunks ago was drained by these warps in the
+    // previous iteration), then O (c-1) / (Q'z + P 1) into the staging tile
+    // [(c-1) & 1] and one TMA store of the 64 x 64 tile (rows past T clipped).
+    const int row = 16 * (warp & 3) + lane;
+    const bool live = lane < 16;
+    const bool leader = warp == 12 && lane == 0;
+    auto make_p = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!named_bar_and(kBarPO, 128, mbar_wait(bar + B_GDONE + 8 * b, (c >> 1) & 1, wc))) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // 32 columns at a time
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_base + TM_G + 64 * b + 32 * h, g);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int sc = 32 * h + c16 * 8 + e;
+              x[e] = sc <= row ? __uint_as_float(g[c16 * 8 + e]) : 0.f;
+            }
+            st_bf16x8(sm + L::P_OFF + b * kTile + sw128_off(row, 4 * h + c16), x);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarPO, 128);
+      if (leader) mbar_arrive(bar + B_PREADY + 8 * b);
+      return true;
+    };
+    auto drain_o = [&](int c) -> bool {
+      const int b = c & 1;
+      if (leader) bulk_wait_group_read<1>();  // the store of chunk c-2 has read staging tile b
+      if (!named_bar_and(kBarPO, 128, mbar_wait(bar + B_ODONE + 8 * b, (c >> 1) & 1, wc))) return false;
+      tc_fence_after();
+      const uint32_t o0 = tmem + lane_base + TM_O + kAugStride * b;
+      const float inv = 1.f / __uint_as_float(tmem_ld1(o0 + 64));
+      uint8_t* stg = sm + L::OST_OFF + b * kTile;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t ov[32];
+        tmem_ld32(o0 + 32 * h, ov);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[c16 * 8 + e]) * inv;
+            st_bf16x8(stg + sw128_off(row, 4 * h + c16), x);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarPO, 128);
+      if (leader) {
+        mbar_arrive(bar + B_OFREE + 8 * b);
+        tma_store_3d(&tmO, smem_u32(stg), j0, c * kC, bh);
+        bulk_commit_group();
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int c = 0; c <= nchunks && ok; ++c) {
+      if (c < nchunks) ok = make_p(c);
+      if (ok && c >= 1) ok = drain_o(c - 1);
+    }
+    if (leader) bulk_wait_group_all();
   } else {
     // --------------------------------------------------------------- state --
     const int ct = tid;
-    const int row = ct & 63;
     const size_t s_base = (size_t)bh * DK * Dv;
     float sreg[kDVS], zreg = 0.f;
     // one row of [S | z] as bf16 into tile t (z in column 0 of the second block)
@@ -333,50 +445,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(kBarState, kWG);
     if (ct == 0) mbar_arrive(bar + B_SREADY);  // the state entering chunk 0, in tile 0
 
-    bool ok = true, ok_lo = true, ok_hi = true;
+    bool ok = true;
     for (int c = 0; c < nchunks && ok; ++c) {
       const int b = c & 1;
-      const int n = min(kC, T - c * kC);
-      // ---- P = tril(Q'K'^T) rows (TMEM lanes 64-127) to bf16 (warps 2-3) ----
-      if (ct >= 64) {
-        ok_hi = named_bar_and(kBarHi, 64, mbar_wait(bar + B_GDONE + 8 * b, (c >> 1) & 1, wc));
-        if (ok_hi) {
-          tc_fence_after();
-          uint32_t g[64];
-          tmem_ld32(tmem + lane_base + TM_G + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(g));
-          tmem_ld32(tmem + lane_base + TM_G + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(g + 32));
-          tmem_wait_ld();
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int sc = c16 * 8 + e;
-              x[e] = sc <= row ? __uint_as_float(g[sc]) : 0.f;
-            }
-            st_bf16x8(sm + L::P_OFF + b * kTile + sw128_off(row, c16), x);
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          named_bar_sync(kBarHi, 64);
-          if (ct == 64) mbar_arrive(bar + B_PREADY + 8 * b);
-        }
-      }
       // ---- [S | z] += K'^T [V | 1] (c) ----
-      ok = named_bar_and(kBarState, kWG,
-                         ok_hi && ok_lo && mbar_wait(bar + B_DSDONE + 8 * b, (c >> 1) & 1, wc));
+      ok = named_bar_and(kBarState, kWG, mbar_wait(bar + B_DSDONE + 8 * b, (c >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
       if (ct < DK) {
         const uint32_t d0 = tmem + lane_base + TM_DS + kAugStride * b;
-        uint32_t ds[64];
-        tmem_ld32(d0, *reinterpret_cast<uint32_t(*)[32]>(ds));
-        tmem_ld32(d0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
-        const uint32_t dz = tmem_ld1(d0 + 64);
-        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; ++e) sreg[e] += __uint_as_float(ds[e]);
-        zreg += __uint_as_float(dz);
+        for (int h = 0; h < 4; ++h) {  // 16 columns at a time (the state already holds 64 registers)
+          uint32_t ds[16];
+          tmem_ld16(d0 + 16 * h, ds);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) sreg[16 * h + e] += __uint_as_float(ds[e]);
+        }
+        zreg += __uint_as_float(tmem_ld1(d0 + 64));
       }
       tc_fence_before();
       named_bar_sync(kBarState, kWG);
@@ -390,34 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(kBarState, kWG);
         if (ct == 0) mbar_arrive(bar + B_SREADY + 8 * (b ^ 1));
-      }
-      // ---- O (c) / (Q'z + P 1) -> global (warps 0-1, TMEM lanes 0-63) ----
-      if (ct < 64) {
-        ok_lo = named_bar_and(kBarLo, 64, mbar_wait(bar + B_ODONE + 8 * b, (c >> 1) & 1, wc));
-        if (ok_lo) {
-          tc_fence_after();
-          const uint32_t o0 = tmem + lane_base + TM_O + kAugStride * b;
-          uint32_t ov[64];
-          tmem_ld32(o0, *reinterpret_cast<uint32_t(*)[32]>(ov));
-          tmem_ld32(o0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
-          const uint32_t od = tmem_ld1(o0 + 64);
-          tmem_wait_ld();
-          if (row < n) {
-            const float inv = 1.f / __uint_as_float(od);
-            __nv_bfloat16* orow =
-                static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c * kC + row) * Dv + j0;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              float x[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(ov[cc * 8 + e]) * inv;
-              st_bf16x8(orow + cc * 8, x);
-            }
-          }
-          tc_fence_before();
-          named_bar_sync(kBarLo, 64);
-          if (ct == 0) mbar_arrive(bar + B_OFREE + 8 * b);
-        }
       }
     }
     if (ct < DK) {
@@ -440,16 +498,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int DK>
 cudaError_t launch_t(const ChunkProblem& p, cudaStream_t st) {
   using L = LinLayout<DK>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const int BH = p.B * p.H;
   if (!make_tmap_3d_bf16(&mq, p.q, DK, p.T, BH) || !make_tmap_3d_bf16(&mk, p.k, DK, p.T, BH) ||
-      !make_tmap_3d_bf16(&mv, p.v, p.Dv, p.T, BH))
+      !make_tmap_3d_bf16(&mv, p.v, p.Dv, p.T, BH) || !make_tmap_3d_bf16(&mo, p.o, p.Dv, p.T, BH))
     return cudaErrorInvalidValue;
   auto kern = linear_tc_kernel<DK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
-  kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, p);
+  kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
 
