@@ -250,10 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_qkt = [&](int c) {
       const uint32_t st = stage(c);
       constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+      const uint64_t dq = desc_k(st + L::Q_OFF), dk = desc_k(st + L::K_OFF);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
         const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem + TM_G, desc_k(st + L::Q_OFF + off), desc_k(st + L::K_OFF + off), id, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_G, desc_step(dq, off), desc_step(dk, off), id, ks > 0);
       }
     };
     // W = Tbg K (lanes 64-127 of TM_W), Uh = Tb V (lanes 64-127 of Uh[c & 1]).
@@ -264,22 +265,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t st = stage(c);
       if (!GATED && (c & 1) == 0) {
         constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
+        const uint64_t da = desc_k(st + L::V_OFF), db = desc_mn(st + L::K_OFF, L::KB_STRIDE);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss_elect(tmem + TM_W, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
-                            desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE), id, ks > 0);
+          mma_bf16_ss_elect(tmem + TM_W, desc_step(da, ks * 32),  // rows 64-127: Tb
+                            desc_step(db, ks * 2048), id, ks > 0);
       } else {
         constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
         constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
         // rows 64-127 of the A operand: Tbg (gated) or Tb
         const uint32_t wa = st + (GATED ? L::TB_OFF : L::V_OFF);
         const uint32_t uh = (c & 1) ? TM_UH1 : TM_UH0;
+        const uint64_t dw = desc_k(wa), dk = desc_mn(st + L::K_OFF, L::KB_STRIDE);
+        const uint64_t dt = desc_k(st + L::V_OFF), dv = desc_mn(st + L::V_OFF, kTile);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ss_elect(tmem + TM_W, desc_k(wa + ks * 32), desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                            idw, ks > 0);
-          mma_bf16_ss_elect(tmem + uh, desc_k(st + L::V_OFF + ks * 32),  // rows 64-127: Tb
-                            desc_mn(st + L::V_OFF + ks * 2048, kTile), idu, ks > 0);
+          mma_bf16_ss_elect(tmem + TM_W, desc_step(dw, ks * 32), desc_step(dk, ks * 2048), idw, ks > 0);
+          mma_bf16_ss_elect(tmem + uh, desc_step(dt, ks * 32),  // rows 64-127: Tb
+                            desc_step(dv, ks * 2048), idu, ks > 0);
         }
       }
     };
@@ -287,31 +290,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_qw = [&](int c) {
       const uint32_t st = stage(c);
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+      const uint64_t dq = desc_k(st + L::Q_OFF), ds = desc_mn(sb + L::S_OFF, kTile);
 #pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = st + (ks >> 2) * L::KB_STRIDE + L::Q_OFF + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(a), desc_mn(sb + L::S_OFF + ks * 2048, kTile),
-                          id, ks > 0);
-      }
+      for (int ks = 0; ks < DK / 16; ++ks)
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_step(dq, (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32),
+                          desc_step(ds, ks * 2048), id, ks > 0);
     };
     // dS = K^T U~
     auto issue_ds = [&](int c) {
       const uint32_t st = stage(c);
       const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
       constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+      const uint64_t dk = desc_mn(st + L::K_OFF, L::KB_STRIDE), du = desc_mn(ut, kTile);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_DS, desc_mn(st + L::K_OFF + ks * 2048, L::KB_STRIDE),
-                          desc_mn(ut + ks * 2048, kTile), id, ks > 0);
+        mma_bf16_ss_elect(tmem + TM_DS, desc_step(dk, ks * 2048), desc_step(du, ks * 2048), id, ks > 0);
     };
     // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
     auto issue_pu = [&](int c) {
-      const uint32_t pa = sb + L::P_OFF;
       constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+      const uint64_t dp = desc_k(sb + L::P_OFF), du = desc_mn(sb + L::U_OFF, kTile);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_k(pa + ks * 32),
-                          desc_mn(sb + L::U_OFF + ks * 2048, kTile), id, 1);
+        mma_bf16_ss_elect(tmem + TM_QW + 64 * (c & 1), desc_step(dp, ks * 32), desc_step(du, ks * 2048), id, 1);
     };
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL, 0, wc));
     if (ok) {

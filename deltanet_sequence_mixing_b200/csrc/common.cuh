@@ -308,6 +308,13 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t addr, uint32_t lbo) {
   return sw128_desc(addr, lbo, 1024);
 }
 
+// The descriptor of the same layout `bytes` further on: the start address is
+// the low 14-bit field (address / 16), and shared memory ends below 2^18 bytes,
+// so the sum never carries into the next field.  Forming a product's
+// descriptors once and stepping them keeps the issuing warp's instruction
+// count per MMA low.
+__device__ __forceinline__ uint64_t desc_step(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 // Named barrier over `count` threads; the AND form returns true only if every
 // participating thread passed true (a uniform decision for the whole group).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {

@@ -211,10 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpIssuer) {
     // -------------------------------------------------------------- issuer --
-    // Descriptors are formed once per product and stepped by adding the byte
-    // offset / 16 to the start-address field (no carry: shared memory ends
-    // below 2^18 bytes), which keeps the single issuing warp's instruction
-    // count per MMA low while it shares its scheduler with busy warps.
+    // Descriptors are formed once per product and stepped (desc_step): the
+    // single issuing warp shares its scheduler with busy warps.
     // Gram (c) = Q' K'^T into G[c & 1] (M = 64)
     auto issue_gram = [&](int c) {
       const uint32_t st = stage(c);
@@ -223,9 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = desc_k(st + L::Q_OFF), dk = desc_k(st + L::K_OFF);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        constexpr uint32_t kOff[4] = {0, 2, 4, 6};
-        const uint64_t off = (uint64_t)((ks >> 2) * (L::KB_STRIDE >> 4) + kOff[ks & 3]);
-        mma_bf16_ss_elect(tmem + TM_G + 64 * b, dq + off, dk + off, idg, ks > 0);
+        const uint32_t off = (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32;
+        mma_bf16_ss_elect(tmem + TM_G + 64 * b, desc_step(dq, off), desc_step(dk, off), idg, ks > 0);
       }
       mma_commit_elect(bar + B_GDONE + 8 * b);
     };
@@ -238,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t da = desc_mn(st + L::K_OFF, L::KB_STRIDE), dv = desc_mn(st + L::V_OFF, ones_lbo);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_DS + kAugStride * b, da + (uint64_t)(ks * 128), dv + (uint64_t)(ks * 128), idd,
+        mma_bf16_ss_elect(tmem + TM_DS + kAugStride * b, desc_step(da, ks * 2048), desc_step(dv, ks * 2048), idd,
                           ks > 0);
       mma_commit_elect(bar + B_DSDONE + 8 * b);
     };
@@ -251,14 +248,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = desc_k(st + L::Q_OFF), ds = desc_mn(sb + L::S_OFF + b * 2 * L::SBLK, L::SBLK);
       const uint64_t dp = desc_k(sb + L::P_OFF + b * kTile), dv = desc_mn(st + L::V_OFF, ones_lbo);
 #pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks) {
-        constexpr uint32_t kOff[4] = {0, 2, 4, 6};
-        const uint64_t off = (uint64_t)((ks >> 2) * (L::KB_STRIDE >> 4) + kOff[ks & 3]);
-        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, dq + off, ds + (uint64_t)(ks * 128), ido, ks > 0);
-      }
+      for (int ks = 0; ks < DK / 16; ++ks)
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_step(dq, (ks >> 2) * L::KB_STRIDE + (ks & 3) * 32),
+                          desc_step(ds, ks * 2048), ido, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, dp + (uint64_t)(2 * ks), dv + (uint64_t)(ks * 128), ido, 1);
+        mma_bf16_ss_elect(tmem + TM_O + kAugStride * b, desc_step(dp, ks * 32), desc_step(dv, ks * 2048), ido, 1);
       mma_commit_elect(bar + B_ODONE + 8 * b);
       mma_commit_elect(bar + B_EMPTY + 8 * (c % NST));  // stage c: Gram, dS and O have read it
     };
