@@ -188,20 +188,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- phase A: P = Q K^T, W = Tb(g) K, Uh = Tb V ----
       {
         constexpr uint32_t idp = idesc_bf16(128, 128, false, false);
+        const uint64_t dq = desc_k(sb + L::Q_OFF), dk = desc_k(sb + L::K_OFF);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
-          mma_bf16_ss_elect(tmem + TM::P, desc_k(sb + L::Q_OFF + off), desc_k(sb + L::K_OFF + off), idp, ks > 0);
+          mma_bf16_ss_elect(tmem + TM::P, desc_step(dq, off), desc_step(dk, off), idp, ks > 0);
         }
         constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
         constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
-        const uint32_t wa = sb + (GATED ? L::TBG_OFF : L::TB_OFF);
+        const uint64_t dw = desc_k(sb + (GATED ? L::TBG_OFF : L::TB_OFF)), dt = desc_k(sb + L::TB_OFF);
+        const uint64_t dkm = desc_mn(sb + L::K_OFF, kBlk), dv = desc_mn(sb + L::V_OFF, kBlk);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
-          mma_bf16_ss_elect(tmem + TM::W, desc_k(wa + off), desc_mn(sb + L::K_OFF + ks * 2048, kBlk), idw, ks > 0);
-          mma_bf16_ss_elect(tmem + TM::UH, desc_k(sb + L::TB_OFF + off), desc_mn(sb + L::V_OFF + ks * 2048, kBlk),
-                            idu, ks > 0);
+          mma_bf16_ss_elect(tmem + TM::W, desc_step(dw, off), desc_step(dkm, ks * 2048), idw, ks > 0);
+          mma_bf16_ss_elect(tmem + TM::UH, desc_step(dt, off), desc_step(dv, ks * 2048), idu, ks > 0);
         }
         mma_commit_elect(bar + B_MMAA);
       }
@@ -211,12 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- phase B: QS = Q S, WS = W S ----
       {
         constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+        const uint64_t ds = desc_mn(sb + L::S_OFF, kBlk), dq = desc_k(sb + L::Q_OFF), dw = desc_k(sb + L::W_OFF);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
-          const uint64_t bs = desc_mn(sb + L::S_OFF + ks * 2048, kBlk);
-          mma_bf16_ss_elect(tmem + TM::QS, desc_k(sb + L::Q_OFF + off), bs, id, ks > 0);
-          mma_bf16_ss_elect(tmem + TM::WS, desc_k(sb + L::W_OFF + off), bs, id, ks > 0);
+          const uint64_t bs = desc_step(ds, ks * 2048);
+          mma_bf16_ss_elect(tmem + TM::QS, desc_step(dq, off), bs, id, ks > 0);
+          mma_bf16_ss_elect(tmem + TM::WS, desc_step(dw, off), bs, id, ks > 0);
         }
         mma_commit_elect(bar + B_MMAB);
       }
@@ -227,14 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         constexpr uint32_t ido = idesc_bf16(128, 64, false, true);
         constexpr uint32_t idd = idesc_bf16(128, 64, true, true);
-        const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
+        const uint64_t dp = desc_k(sb + L::P_OFF), du = desc_mn(sb + L::U_OFF, kBlk);
+        const uint64_t dkm = desc_mn(sb + L::K_OFF, kBlk), dut = desc_mn(sb + (GATED ? L::UT_OFF : L::U_OFF), kBlk);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kBlk + (ks & 3) * 32;
-          mma_bf16_ss_elect(tmem + TM::QS, desc_k(sb + L::P_OFF + off), desc_mn(sb + L::U_OFF + ks * 2048, kBlk),
-                            ido, 1);
-          mma_bf16_ss_elect(tmem + TM::DS, desc_mn(sb + L::K_OFF + ks * 2048, kBlk), desc_mn(ut + ks * 2048, kBlk),
-                            idd, ks > 0);
+          mma_bf16_ss_elect(tmem + TM::QS, desc_step(dp, off), desc_step(du, ks * 2048), ido, 1);
+          mma_bf16_ss_elect(tmem + TM::DS, desc_step(dkm, ks * 2048), desc_step(dut, ks * 2048), idd, ks > 0);
         }
         mma_commit_elect(bar + B_MMAC);
       }

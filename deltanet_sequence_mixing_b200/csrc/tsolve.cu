@@ -178,10 +178,11 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     if (ok) {
       tc_fence_after();
       constexpr uint32_t id = idesc_bf16(128, kC, false, false);
+      const uint64_t d0 = desc_k(sb);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t a = sb + (ks >> 2) * (kC * 128) + (ks & 3) * 32;
-        mma_bf16_ss_elect(tmem, desc_k(a), desc_k(a), id, ks > 0);
+        const uint64_t d = desc_step(d0, (ks >> 2) * (kC * 128) + (ks & 3) * 32);
+        mma_bf16_ss_elect(tmem, d, d, id, ks > 0);
       }
     }
     mma_commit_elect(bar_mma);  // arrives even with no MMA in flight
