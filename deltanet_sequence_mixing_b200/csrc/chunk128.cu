@@ -317,18 +317,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                       reinterpret_cast<const float*>(v) + cc * 8);
         }
         if (GATED) {
+          // (each 64-column block loaded whole before its stores, which the
+          // compiler cannot tell apart from the loads)
           const float gam = __expf(gr);
 #pragma unroll
-          for (int c16 = 0; c16 < DK / 8; ++c16) {
-            uint8_t* ptr = sm + L::Q_OFF + (c16 >> 3) * kBlk + sw128_off(r, c16 & 7);
-            uint4 u = *reinterpret_cast<uint4*>(ptr);
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+          for (int kb = 0; kb < DK / 64; ++kb) {
+            uint4 u[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wv[e]));
-              wv[e] = pack2_bf16(f.x * gam, f.y * gam);
+            for (int c16 = 0; c16 < 8; ++c16)
+              u[c16] = *reinterpret_cast<const uint4*>(sm + L::Q_OFF + kb * kBlk + sw128_off(r, c16));
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) {
+              float x[8];
+              unpack_bf16x8(u[c16], x);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) x[e] *= gam;
+              st_bf16x8(sm + L::Q_OFF + kb * kBlk + sw128_off(r, c16), x);
             }
-            *reinterpret_cast<uint4*>(ptr) = u;
           }
         }
       }

@@ -393,16 +393,32 @@ __device__ __forceinline__ void prestep_row_sw128(uint8_t* tile, uint32_t blk_st
   const float other = __shfl_xor_sync(0xffffffffu, ss, 1);
   const float tot = part == 0 ? ss + other : other + ss;
   const float inv = 1.f / fmaxf(sqrtf(tot), 1e-12f);
+  // Rewrite in groups of four chunks, each group loaded whole before its
+  // stores (a store may alias a later load as far as the compiler knows, so a
+  // load issued after it waits for it).
 #pragma unroll
-  for (int j = 0; j < NCH; ++j) {
-    const int cg = part * NCH + j, blk = cg >> 3, c16 = cg & 7;
-    uint4* at = reinterpret_cast<uint4*>(tile + blk * blk_stride + sw128_off(row, c16));
-    float x[8];
-    unpack_bf16x8(*at, x);
+  for (int j0 = 0; j0 < NCH; j0 += 4) {
+    uint4 raw[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = silu_f(x[e]) * inv;
-    st_bf16x8(at, x);
-    if (dst) *reinterpret_cast<uint4*>(dst + cg * 8) = *at;
+    for (int j = 0; j < 4; ++j) {
+      const int cg = part * NCH + j0 + j;
+      raw[j] = *reinterpret_cast<const uint4*>(tile + (cg >> 3) * blk_stride + sw128_off(row, cg & 7));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cg = part * NCH + j0 + j;
+      float x[8];
+      unpack_bf16x8(raw[j], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = silu_f(x[e]) * inv;
+      uint4 m;
+      m.x = pack2_bf16(x[0], x[1]);
+      m.y = pack2_bf16(x[2], x[3]);
+      m.z = pack2_bf16(x[4], x[5]);
+      m.w = pack2_bf16(x[6], x[7]);
+      *reinterpret_cast<uint4*>(tile + (cg >> 3) * blk_stride + sw128_off(row, cg & 7)) = m;
+      if (dst) *reinterpret_cast<uint4*>(dst + cg * 8) = m;
+    }
   }
 }
 
