@@ -48,7 +48,9 @@ int validate_problem(const dn::ChunkProblem& p) {
     return DN_ERR_UNSUPPORTED;
   if (p.alpha_per_dim && !p.alpha && p.T > 0) return DN_ERR_INVALID_ARG;
   if ((long long)p.B * p.H > INT_MAX) return DN_ERR_UNSUPPORTED;
-  // the pre-pass runs one CTA per (b, h, chunk), on a one-dimensional grid
+  // the chunk kernels run one CTA per (b, h, 64-column slice of Dv) on a
+  // one-dimensional grid, the pre-pass one CTA per (b, h, chunk)
+  if ((long long)p.B * p.H * ((p.Dv + 63) / 64) > INT_MAX) return DN_ERR_UNSUPPORTED;
   if ((long long)p.B * p.H * ((p.T + (long long)p.C - 1) / p.C) > INT_MAX) return DN_ERR_UNSUPPORTED;
   // With T == 0 no token buffer is ever dereferenced (empty tensors may carry a
   // null data pointer); otherwise every token buffer is required.

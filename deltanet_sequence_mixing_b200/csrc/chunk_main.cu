@@ -132,8 +132,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = warp_uniform(smem_u32(sm));
   const int tid = threadIdx.x, lane = tid & 31;
   const int warp = (int)warp_uniform((uint32_t)tid >> 5);  // role branches stay warp-uniform
-  const int bh = blockIdx.x;
-  const int j0 = blockIdx.y * kDVS;
+  // 1-D grid with the D_v slices of a head adjacent: they are scheduled
+  // together, so the second slice's K, Q (and pre-pass) tiles come from L2
+  // even when the grid takes more than one wave.
+  const int nsl = p.Dv / kDVS;
+  const int bh = blockIdx.x / nsl, slice = blockIdx.x % nsl;
+  const int j0 = slice * kDVS;
   const int T = p.T, Dv = p.Dv;
   const int nchunks = (T + kC - 1) / kC;
   const uint32_t bar = sb + L::BAR_OFF;
@@ -616,7 +620,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   auto kern = chunk_main_kernel<DK, GATED>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
+  dim3 grid((unsigned)(BH * (p.Dv / kDVS)));
   // Programmatic dependent launch: CTAs may start (TMEM, barriers, state
   // load) while the pre-pass drains; the producer waits for its results.
   cudaLaunchConfig_t cfg = {};

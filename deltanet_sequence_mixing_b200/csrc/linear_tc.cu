@@ -125,8 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = warp_uniform(smem_u32(sm));
   const int tid = threadIdx.x, lane = tid & 31;
   const int warp = (int)warp_uniform((uint32_t)tid >> 5);
-  const int bh = blockIdx.x;
-  const int j0 = blockIdx.y * kDVS;
+  // 1-D grid with the D_v slices of a head adjacent: they are scheduled
+  // together, so the second slice's K, Q (and pre-pass) tiles come from L2
+  // even when the grid takes more than one wave.
+  const int nsl = p.Dv / kDVS;
+  const int bh = blockIdx.x / nsl, slice = blockIdx.x % nsl;
+  const int j0 = slice * kDVS;
   const int T = p.T, Dv = p.Dv;
   const int nchunks = (T + kC - 1) / kC;
   const uint32_t bar = sb + L::BAR_OFF;
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < kDVS; j += 4)
           *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
       }
-      if (p.z_out && blockIdx.y == 0) p.z_out[(size_t)bh * DK + ct] = zreg;
+      if (p.z_out && slice == 0) p.z_out[(size_t)bh * DK + ct] = zreg;
     }
   }
 
@@ -501,7 +505,7 @@ cudaError_t launch_t(const ChunkProblem& p, cudaStream_t st) {
   auto kern = linear_tc_kernel<DK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)BH, (unsigned)(p.Dv / kDVS));
+  dim3 grid((unsigned)(BH * (p.Dv / kDVS)));
   kern<<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
