@@ -14,7 +14,9 @@
 //                                accumulated onto the same tile)
 //   S <- gamma_last S + K^T (diag(Gamma_last,.) U)             (float32 registers)
 //
-// One CTA per (b, h, 64-column slice of Dv), 10 warps:
+// One CTA per (b, h, slice of DVS = 64 columns of Dv; 32 when 64-column
+// slices would leave most SMs idle and 32-column ones still fit one wave),
+// 10 warps:
 //   warp 9     MMA issuer (warp-uniform, one elected lane issues): every
 //              tcgen05.mma of the CTA, in a fixed order that keeps the state
 //              chain fed:
@@ -48,7 +50,6 @@ namespace dn {
 namespace {
 
 constexpr int kC = 64;
-constexpr int kDVS = 64;
 constexpr uint32_t kTile = 8192;  // 64 rows x 128 bytes
 constexpr int kWG = 128;
 constexpr int kThreads = 2 * kWG + 64;  // chain 0-3, prep 4-7, producer 8, issuer 9
@@ -117,7 +118,7 @@ __device__ __forceinline__ void u_epilogue_half(uint32_t ws_addr, uint32_t uh_ad
   }
 }
 
-template <int DK, bool GATED>
+template <int DK, bool GATED, int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
@@ -135,9 +136,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 1-D grid with the D_v slices of a head adjacent: they are scheduled
   // together, so the second slice's K, Q (and pre-pass) tiles come from L2
   // even when the grid takes more than one wave.
-  const int nsl = p.Dv / kDVS;
+  const int nsl = p.Dv / DVS;
   const int bh = blockIdx.x / nsl, slice = blockIdx.x % nsl;
-  const int j0 = slice * kDVS;
+  const int j0 = slice * DVS;
+  // V comes as the 64-column box holding the slice; a 32-column slice starts
+  // 64 bytes into the box's 128-byte rows when it is the box's second half
+  const int jv = j0 & ~63;
+  const uint32_t vcol = (uint32_t)(j0 & 63) * 2;
   const int T = p.T, Dv = p.Dv;
   const int nchunks = (T + kC - 1) / kC;
   const uint32_t bar = sb + L::BAR_OFF;
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + B_CMMA4, 1);
     mbar_init(bar + B_PMMA1, 1);
     mbar_init(bar + B_PMMA2, 1);
-    mbar_init(bar + B_UREADY, 2);  // both column halves of the U epilogue
+    mbar_init(bar + B_UREADY, DVS / 32);  // the column halves of the U epilogue
     mbar_init(bar + B_SREADY, 1);
     mbar_init(bar + B_WREADY, 1);
     mbar_init(bar + B_QSCALED, 1);  // gated: the QS rows of TM_QW scaled by gamma
@@ -206,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(st + kb * L::KB_STRIDE + L::K_OFF, &tmK, full, kb * 64, c0, bh);
           tma_load_3d(st + kb * L::KB_STRIDE + L::Q_OFF, &tmQ, full, kb * 64, c0, bh);
         }
-        tma_load_3d(st + L::V_OFF, &tmV, full, j0, c0, bh);
+        tma_load_3d(st + L::V_OFF, &tmV, full, jv, c0, bh);
         tma_load_3d(st + L::TB_OFF, &tmTb, full, 0, c0, bh);
         if (GATED) tma_load_3d(st + L::TBG_OFF, &tmTbg, full, 0, c0, bh);
       }
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_l2_3d(&tmK, kb * 64, cn, bh);
             prefetch_l2_3d(&tmQ, kb * 64, cn, bh);
           }
-          prefetch_l2_3d(&tmV, j0, cn, bh);
+          prefetch_l2_3d(&tmV, jv, cn, bh);
           prefetch_l2_3d(&tmTb, 0, cn, bh);
           if (GATED) {
             prefetch_l2_3d(&tmTbg, 0, cn, bh);
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // N = Dk + 64 product.
     auto issue_wu = [&](int c) {
       const uint32_t st = stage(c);
-      if (!GATED && (c & 1) == 0) {
+      if (!GATED && DVS == 64 && (c & 1) == 0) {
         constexpr uint32_t id = idesc_bf16(128, DK + 64, false, true);
         const uint64_t da = desc_k(st + L::V_OFF), db = desc_mn(st + L::K_OFF, L::KB_STRIDE);
 #pragma unroll
@@ -276,12 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             desc_step(db, ks * 2048), id, ks > 0);
       } else {
         constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
-        constexpr uint32_t idu = idesc_bf16(128, 64, false, true);
+        constexpr uint32_t idu = idesc_bf16(128, DVS, false, true);
         // rows 64-127 of the A operand: Tbg (gated) or Tb
         const uint32_t wa = st + (GATED ? L::TB_OFF : L::V_OFF);
         const uint32_t uh = (c & 1) ? TM_UH1 : TM_UH0;
         const uint64_t dw = desc_k(wa), dk = desc_mn(st + L::K_OFF, L::KB_STRIDE);
-        const uint64_t dt = desc_k(st + L::V_OFF), dv = desc_mn(st + L::V_OFF, kTile);
+        const uint64_t dt = desc_k(st + L::V_OFF), dv = desc_mn(st + L::V_OFF + vcol, kTile);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           mma_bf16_ss_elect(tmem + TM_W, desc_step(dw, ks * 32), desc_step(dk, ks * 2048), idw, ks > 0);
@@ -293,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // [Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
     auto issue_qw = [&](int c) {
       const uint32_t st = stage(c);
-      constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+      constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
       const uint64_t dq = desc_k(st + L::Q_OFF), ds = desc_mn(sb + L::S_OFF, kTile);
 #pragma unroll
       for (int ks = 0; ks < DK / 16; ++ks)
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_ds = [&](int c) {
       const uint32_t st = stage(c);
       const uint32_t ut = sb + (GATED ? L::UT_OFF : L::U_OFF);
-      constexpr uint32_t id = idesc_bf16(128, 64, true, true);
+      constexpr uint32_t id = idesc_bf16(128, DVS, true, true);
       const uint64_t dk = desc_mn(st + L::K_OFF, L::KB_STRIDE), du = desc_mn(ut, kTile);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // O = diag(gamma) QS + P U (accumulated onto lanes 0-63 of TM_QW[c & 1])
     auto issue_pu = [&](int c) {
-      constexpr uint32_t id = idesc_bf16(128, 64, false, true);
+      constexpr uint32_t id = idesc_bf16(128, DVS, false, true);
       const uint64_t dp = desc_k(sb + L::P_OFF), du = desc_mn(sb + L::U_OFF, kTile);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
@@ -401,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 192) mbar_arrive(bar + B_WREADY);
 
       // ---- columns 32-63 of the U epilogue of chunk c (rows on lanes 64-127) ----
+      if (DVS == 32) continue;  // a 32-column slice: the chain warps take all of it
       ok = named_bar_and(kBarPrepW, 64, mbar_wait(bar + B_CMMA3, c & 1, wc));
       if (!ok) break;
       tc_fence_after();
@@ -486,16 +492,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ct = tid;
     const int row = ct & 63;
     const size_t s_base = (size_t)bh * DK * Dv;
-    float sreg[kDVS];
+    float sreg[DVS];
     if (ct < DK) {
       const float* src = p.S0 ? p.S0 + s_base + (size_t)ct * Dv + j0 : nullptr;
 #pragma unroll
-      for (int j = 0; j < kDVS; j += 4) {
+      for (int j = 0; j < DVS; j += 4) {
         const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
       }
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
+      for (int c16 = 0; c16 < DVS / 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
     }
     fence_proxy_async_smem();
     named_bar_sync(kBarChain, kWG);
@@ -529,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float gam = __expf(vb[row]);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < DVS / 32; ++q) {
             uint32_t v[32];
             tmem_ld32(qw + lane_base + q * 32, v);
             tmem_wait_ld();
@@ -550,14 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- state update (lanes 0..DK-1) ----
       if (ct < DK) {
         const float carry = GATED ? __expf(vb[n - 1]) : 1.f;
-        uint32_t ds[64];
-        tmem_ld32(tmem + lane_base + TM_DS, *reinterpret_cast<uint32_t(*)[32]>(ds));
-        tmem_ld32(tmem + lane_base + TM_DS + 32, *reinterpret_cast<uint32_t(*)[32]>(ds + 32));
+        uint32_t ds[DVS];
+#pragma unroll
+        for (int q = 0; q < DVS / 32; ++q)
+          tmem_ld32(tmem + lane_base + TM_DS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(ds + 32 * q));
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 64; ++e) sreg[e] = fmaf(carry, sreg[e], __uint_as_float(ds[e]));
+        for (int e = 0; e < DVS; ++e) sreg[e] = fmaf(carry, sreg[e], __uint_as_float(ds[e]));
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
+        for (int c16 = 0; c16 < DVS / 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + row) * Dv + j0;
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < DVS / 32; ++q) {
             uint32_t ov[32];
             tmem_ld32(qw + lane_base + q * 32, ov);
             tmem_wait_ld();
@@ -590,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.S_out && ct < DK) {
       float* dst = p.S_out + s_base + (size_t)ct * Dv + j0;
 #pragma unroll
-      for (int j = 0; j < kDVS; j += 4)
+      for (int j = 0; j < DVS; j += 4)
         *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
     }
   }
@@ -601,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, bool GATED>
+template <int DK, bool GATED, int DVS>
 cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   using L = MainLayout<DK, GATED>;
   const int BH = p.B * p.H;
@@ -617,10 +624,10 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
       !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
       !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))
     return cudaErrorInvalidValue;
-  auto kern = chunk_main_kernel<DK, GATED>;
+  auto kern = chunk_main_kernel<DK, GATED, DVS>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(BH * (p.Dv / kDVS)));
+  dim3 grid((unsigned)(BH * (p.Dv / DVS)));
   // Programmatic dependent launch: CTAs may start (TMEM, barriers, state
   // load) while the pre-pass drains; the producer waits for its results.
   cudaLaunchConfig_t cfg = {};
@@ -643,10 +650,32 @@ bool chunk_main_supported(const ChunkProblem& p) {
          (p.Dv == 64 || p.Dv == 128);
 }
 
+// The SM count of the current device (queried once per device).
+static int sm_count() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    counts[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+  }
+  return counts[dev];
+}
+
+template <int DK, bool GATED>
+cudaError_t launch_dvs(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+  // Each CTA runs the whole chunk chain of its (b, h, slice); the chain's
+  // length per chunk hardly depends on the slice width.  When 64-column
+  // slices leave most SMs idle (long sequences over few heads), 32-column
+  // slices give twice the CTAs, as long as they still fit one wave.
+  if ((long long)p.B * p.H * (p.Dv / 32) <= sm_count()) return launch_t<DK, GATED, 32>(p, w, st);
+  return launch_t<DK, GATED, 64>(p, w, st);
+}
+
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
   const bool gated = p.alpha != nullptr;
-  if (p.Dk == 128) return gated ? launch_t<128, true>(p, w, st) : launch_t<128, false>(p, w, st);
-  return gated ? launch_t<64, true>(p, w, st) : launch_t<64, false>(p, w, st);
+  if (p.Dk == 128) return gated ? launch_dvs<128, true>(p, w, st) : launch_dvs<128, false>(p, w, st);
+  return gated ? launch_dvs<64, true>(p, w, st) : launch_dvs<64, false>(p, w, st);
 }
 
 }  // namespace dn

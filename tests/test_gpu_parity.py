@@ -76,6 +76,25 @@ def test_delta_shapes_ragged(dn, oracle_mod, dtype, Dk, Dv, T):
     _check_delta(dn, oracle_mod, x)
 
 
+@pytest.mark.parametrize("gated", [False, True])
+def test_slice_width_wide_and_narrow_grids(dn, oracle_mod, gated):
+    """The bf16 C = 64 kernel splits Dv into 64-column slices, or into 32-column
+    ones when the problem has so few heads that twice the CTAs still fit one wave
+    on the B200's 148 SMs.  80 heads (320 32-column slices) take the 64-column
+    grid and one of its heads alone the 32-column grid: both match the oracle
+    (ragged T, initial state, decay) and give the same bits for the same head."""
+    B, H, T = 10, 8, 200
+    x = gen.make_inputs(B, H, T, 128, 128, torch.bfloat16, gated=gated, seed=91 + gated)
+    S0 = torch.randn(B, H, 128, 128, generator=torch.Generator().manual_seed(5)) * 0.05
+    o, S = _run_delta(dn, x, 64, S0)
+    o_ref, S_ref = oracle_mod.deltanet(x["q"], x["k"], x["v"], x["beta"], x["alpha"], S0.double())
+    tol = TOL[torch.bfloat16]
+    assert rel_l2(o, o_ref) <= tol and rel_l2(S, S_ref) <= tol
+    one = {k: (None if v is None else v[2:3, 5:6].contiguous()) for k, v in x.items()}
+    o1, S1 = _run_delta(dn, one, 64, S0[2:3, 5:6].contiguous())
+    assert np.array_equal(o1, o[2:3, 5:6]) and np.array_equal(S1, S[2:3, 5:6])
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("T", [64, 257])
 def test_gated(dn, oracle_mod, dtype, T):
