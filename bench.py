@@ -22,6 +22,7 @@ batched decode) under "extras".
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -493,9 +494,13 @@ def profile_run(args):
 
     dev = torch.device("cuda", 0)
     n = args.warmup + 1
-    if args.profile in ("chunk", "gated", "linear", "long64", "long128"):
+    if args.profile in ("chunk", "gated", "linear", "long64", "long128", "long64q", "long128q"):
+        # long64q / long128q: the long workloads on a quarter of the sequence
+        # (T = 16384, still far larger than L2), small enough for a full ncu capture
+        quarter = lambda w: dataclasses.replace(w, T=w.T // 4, name=w.name.replace("T65536", "T16384"))
         w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR,
-             "long64": gen.LONG64, "long128": gen.LONG128}[args.profile]
+             "long64": gen.LONG64, "long128": gen.LONG128,
+             "long64q": quarter(gen.LONG64), "long128q": quarter(gen.LONG128)}[args.profile]
         x = gen.make_workload(w, seed=0, device=dev)
         for _ in range(n):
             if args.profile == "linear":
@@ -523,7 +528,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--profile", choices=["chunk", "linear", "gated", "long64", "long128", "decode"],
+    ap.add_argument("--profile", choices=["chunk", "linear", "gated", "long64", "long128", "long64q", "long128q",
+                                          "decode"],
                     default=None,
                     help="untimed run for a profiler: --warmup launches of one kernel on its "
                          "workload, then one more (the one to capture)")
