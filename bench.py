@@ -410,6 +410,22 @@ def extras_measure(dn, gen, dev, stream, peaks):
                                "tc_frac": fl / (ms * 1e-3) / 1e12 / tc}
         del x, o, S
 
+    # long context over few heads (B1 H8 T65536 D128 bf16 C64): unsplit, and with
+    # the sequence split (segments side by side, joined afterwards)
+    w = dataclasses.replace(gen.LONG64, H=8, name=gen.LONG64.name.replace("H32", "H8"))
+    x = gen.make_workload(w, seed=4, device=dev)
+    o = torch.empty_like(x["v"])
+    S = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev)
+    fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
+    for split in (False, True):
+        ms = timed(lambda: dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], C=w.C, o=o, S_out=S,
+                                                 seq_split=split), 5, 2)
+        key = "long_8heads_split" if split else "long_8heads"
+        out[key] = {"segments": dn.seq_segments(w.B, w.H, w.T, w.Dk, w.Dv) if split else 1,
+                    "tokens_per_s": w.B * w.T / (ms * 1e-3), "ms": ms, "GBps": by / (ms * 1e-3) / 1e9,
+                    "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm}
+    del x, o, S
+
     # the options and the backward on the prefill shape (B4 H16 T4096 D128 bf16)
     w = gen.PREFILL
     fl, by = algo_counts(w.B, w.H, w.T, w.Dk, w.Dv, w.C)
@@ -494,19 +510,23 @@ def profile_run(args):
 
     dev = torch.device("cuda", 0)
     n = args.warmup + 1
-    if args.profile in ("chunk", "gated", "linear", "long64", "long128", "long64q", "long128q"):
+    if args.profile in ("chunk", "gated", "linear", "long64", "long128", "long64q", "long128q", "split8"):
         # long64q / long128q: the long workloads on a quarter of the sequence
-        # (T = 16384, still far larger than L2), small enough for a full ncu capture
+        # (T = 16384, still far larger than L2), small enough for a full ncu capture;
+        # split8: the long workload over 8 heads (B1 H8 T65536) with the sequence split
         quarter = lambda w: dataclasses.replace(w, T=w.T // 4, name=w.name.replace("T65536", "T16384"))
         w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR,
              "long64": gen.LONG64, "long128": gen.LONG128,
-             "long64q": quarter(gen.LONG64), "long128q": quarter(gen.LONG128)}[args.profile]
+             "long64q": quarter(gen.LONG64), "long128q": quarter(gen.LONG128),
+             "split8": dataclasses.replace(gen.LONG64, H=8, name=gen.LONG64.name.replace("H32", "H8"))
+             }[args.profile]
         x = gen.make_workload(w, seed=0, device=dev)
         for _ in range(n):
             if args.profile == "linear":
                 dn.linear_attn_fwd(x["q"], x["k"], x["v"], C=w.C)
             else:
-                dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C)
+                dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C,
+                                      seq_split=args.profile == "split8")
     else:
         B, H, D = gen.DECODE_SEQS, gen.DECODE_HEADS, 128
         S = torch.randn(B, H, D, D, device=dev) * 0.01
@@ -529,7 +549,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--profile", choices=["chunk", "linear", "gated", "long64", "long128", "long64q", "long128q",
-                                          "decode"],
+                                          "split8", "decode"],
                     default=None,
                     help="untimed run for a profiler: --warmup launches of one kernel on its "
                          "workload, then one more (the one to capture)")

@@ -20,7 +20,7 @@ from ._lib import DeltaNetError, check, lib, status_string  # noqa: F401
 
 __all__ = [
     "deltanet_chunk_fwd", "deltanet_chunk_fwd_host", "deltanet_decode_step", "linear_attn_fwd",
-    "deltanet_chunk_bwd",
+    "deltanet_chunk_bwd", "seq_segments",
     "workspace_for", "host_workspace_for",
     "deltanet_get_device_status", "deltanet_selftest_wait_timeout", "DeltaNetError",
 ]
@@ -78,12 +78,13 @@ def _options(prestep, alpha, per_dim_rank):
 
 
 def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, S_out=None,
-                       workspace=None, prestep: bool = False):
+                       workspace=None, prestep: bool = False, seq_split: bool = False):
     """Chunkwise DeltaNet forward.  q, k: (B,H,T,Dk); v: (B,H,T,Dv) (bf16 or f32);
     beta: (B,H,T) f32; alpha: (B,H,T) f32 (one decay per token) or (B,H,T,Dk)
     (one per key dimension); S0: (B,H,Dk,Dv) f32.  ``prestep``: q, k are raw
     projections and beta logits (silu + L2 normalise and sigmoid run inside).
-    Returns (o, S_out)."""
+    ``seq_split``: permission to run each sequence as segments side by side
+    (DN_OPT_SEQ_SPLIT; see seq_segments).  Returns (o, S_out)."""
     _need(q, "q")
     dev, dtype = q.device, q.dtype
     if dtype not in _DT:
@@ -104,7 +105,7 @@ def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, 
     _need(o, "o", dtype, dev)
     _need(S_out, "S_out", torch.float32, dev)
     dt = _DT[dtype]
-    opts = _options(prestep, alpha, 4)
+    opts = _options(prestep, alpha, 4) | (_lib.DN_OPT_SEQ_SPLIT if seq_split else 0)
     nb = lib().deltanet_workspace_bytes_ex(B, H, T, Dk, Dv, C, dt, opts)
     if nb == 0:
         raise DeltaNetError("deltanet_workspace_bytes_ex", _lib.DN_ERR_UNSUPPORTED)
@@ -118,6 +119,15 @@ def deltanet_chunk_fwd(q, k, v, beta, alpha=None, S0=None, C: int = 64, o=None, 
             _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S_out),
             B, H, T, Dk, Dv, C, dt, opts, _ptr(ws), ws.numel(), _stream(dev)))
     return o, S_out
+
+
+def seq_segments(B, H, T, Dk, Dv, C=64, dtype=torch.bfloat16, prestep=False, per_dim=False,
+                 seq_split=True) -> int:
+    """Segments a deltanet_chunk_fwd call with these arguments runs on the
+    current device (1: the sequence is not split)."""
+    opts = (_lib.DN_OPT_PRESTEP if prestep else 0) | (_lib.DN_OPT_GATE_PER_DIM if per_dim else 0) | (
+        _lib.DN_OPT_SEQ_SPLIT if seq_split else 0)
+    return int(lib().deltanet_seq_segments(B, H, T, Dk, Dv, C, _DT[dtype], opts))
 
 
 def deltanet_chunk_bwd(q, k, v, beta, dO, alpha=None, S0=None, dS_T=None, workspace=None):

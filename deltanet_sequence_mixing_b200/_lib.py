@@ -20,7 +20,7 @@ DN_ERR_CUDA = -4
 DN_ERR_DEVICE_TIMEOUT = -5
 DN_ERR_WORKSPACE = -6
 DN_F32, DN_BF16 = 0, 1
-DN_OPT_PRESTEP, DN_OPT_GATE_PER_DIM = 1, 2
+DN_OPT_PRESTEP, DN_OPT_GATE_PER_DIM, DN_OPT_SEQ_SPLIT = 1, 2, 4
 
 # Every symbol include/deltanet.h declares, with (restype, argtypes).
 _vp, _sz, _i, _ll, _u = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong,
@@ -34,6 +34,7 @@ SIGNATURES = {
     "deltanet_decode_step_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _u,
                                      _vp]),
     "deltanet_workspace_bytes_ex": (_sz, [_i, _i, _i, _i, _i, _i, _i, _u]),
+    "deltanet_seq_segments": (_i, [_i, _i, _i, _i, _i, _i, _i, _u]),
     "deltanet_chunk_fwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _i, _i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp]),
     "linear_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

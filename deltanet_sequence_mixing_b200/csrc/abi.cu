@@ -13,7 +13,7 @@
 namespace {
 
 constexpr size_t kStatusBytes = 256;  // status word + padding (keeps 256-byte alignment)
-constexpr unsigned int kKnownOptions = DN_OPT_PRESTEP | DN_OPT_GATE_PER_DIM;
+constexpr unsigned int kKnownOptions = DN_OPT_PRESTEP | DN_OPT_GATE_PER_DIM | DN_OPT_SEQ_SPLIT;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -209,13 +209,156 @@ cudaError_t host_queues(int dev, HostQueues** out) {
   return cudaSuccess;
 }
 
+// ----------------------------------------------------------- sequence split --
+// DN_OPT_SEQ_SPLIT: the sequence reshaped to (B*H*G, T/G) runs through the
+// pre-pass once; the forward from the segments' entry states (S0 for segment
+// 0, zero for the rest) and the homogeneous chain of every segment then run
+// side by side on two streams, and two small kernels join the segments.
+constexpr int kMinSegChunks = 8;       // 64-token chunks per segment, at least
+constexpr int kMaxSegments = 16;
+// The segment count minimises an estimate of the critical path in units of one
+// chunk of the chain (about 1.35 us on the B200): the chunks of one segment,
+// plus the sequential join (one step per segment boundary, about three chunks
+// each), plus the fixed cost of the split (the homogeneous chain's start, the
+// join's launches and the output correction, about eight chunks).
+constexpr int kJoinStepChunks = 3;
+constexpr int kSplitFixedChunks = 8;
+
+int sm_count_now() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
+  if (options != DN_OPT_SEQ_SPLIT || dt != DN_BF16 || C != 64 || T <= 0) return 1;
+  if (!valid_dim(Dk) || !valid_dim(Dv) || B < 1 || H < 1) return 1;
+  const int sms = sm_count_now();
+  int best = 1;
+  long long best_cost = (T + 63) / 64;  // the plain call
+  for (int G = 2; G <= kMaxSegments; ++G) {
+    const int chunks = (T / G + 63) / 64;
+    if (T % G != 0 || chunks < kMinSegChunks) continue;
+    // both chunk kernels of pass 1 at once, one wave: 64-column slices of Dv and of Dk
+    if ((long long)B * H * G * (Dv / 64 + Dk / 64) > sms) continue;
+    const long long cost = chunks + (long long)kJoinStepChunks * (G - 1) + kSplitFixedChunks;
+    if (cost < best_cost) {
+      best = G;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+struct SplitLayout {  // byte offsets inside the workspace
+  size_t wy, R, S0seg, Send, A, Sin, bytes;
+};
+
+SplitLayout split_layout(int B, int H, int T, int Dk, int Dv, int G) {
+  const size_t BH = (size_t)B * H, BHG = BH * G;
+  SplitLayout L{};
+  size_t off = kStatusBytes;
+  auto take = [&](size_t n) {
+    const size_t at = off;
+    off += (n + 255) / 256 * 256;
+    return at;
+  };
+  L.wy = take(dn::wy_workspace_bytes(1, (int)BHG, T / G, 64));
+  L.R = take(BH * T * Dk * 2);
+  L.S0seg = take(BHG * Dk * Dv * 4);
+  L.Send = take(BHG * Dk * Dv * 4);
+  L.A = take(BHG * Dk * Dk * 4);
+  L.Sin = take(BHG * Dk * Dv * 4);
+  L.bytes = off;
+  return L;
+}
+
+// The second stream and its events, created once per device.
+struct SplitQueues {
+  bool ready = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t prepass = nullptr, hom = nullptr;
+};
+SplitQueues g_split_queues[64];
+std::mutex g_split_mutex;  // held while a call creates or enqueues on them
+
+int run_split(dn::ChunkProblem& p, int G, void* ws, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_split_mutex);
+  SplitQueues& q = g_split_queues[dev];
+  cudaError_t e = cudaSuccess;
+  if (!q.ready) {
+    e = cudaStreamCreateWithFlags(&q.side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&q.prepass, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&q.hom, cudaEventDisableTiming);
+    if (e != cudaSuccess) return map_cuda(e);
+    q.ready = true;
+  }
+  const SplitLayout L = split_layout(p.B, p.H, p.T, p.Dk, p.Dv, G);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int BH = p.B * p.H, Tg = p.T / G;
+  const size_t blk = (size_t)p.Dk * p.Dv * sizeof(float);
+  float* S0seg = reinterpret_cast<float*>(base + L.S0seg);
+  float* Send = reinterpret_cast<float*>(base + L.Send);
+  float* A = reinterpret_cast<float*>(base + L.A);
+  float* Sin = reinterpret_cast<float*>(base + L.Sin);
+  void* R = base + L.R;
+  // entry states of pass 1: S0 for segment 0 of every head, zero for the others
+  e = cudaMemsetAsync(S0seg, 0, (size_t)BH * G * blk, st);
+  if (e == cudaSuccess && p.S0)
+    e = cudaMemcpy2DAsync(S0seg, G * blk, p.S0, blk, blk, BH, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return map_cuda(e);
+  // the sequence as (B*H*G, T/G): a view of the same contiguous tensors
+  dn::ChunkProblem p1 = p;
+  p1.B = BH * G;
+  p1.H = 1;
+  p1.T = Tg;
+  p1.S0 = S0seg;
+  p1.S_out = Send;
+  p1.status = static_cast<unsigned int*>(ws);
+  const dn::WyWorkspace w = dn::wy_carve(base + L.wy, p1.B, 1, Tg, 64, p.Dk);
+  e = dn::launch_tsolve(p1, w, st);
+  if (e == cudaSuccess) e = cudaEventRecord(q.prepass, st);
+  // the homogeneous chains on the side stream, once the factors are in place
+  dn::ChunkProblem p2 = p1;
+  p2.hom = 1;
+  p2.v = p1.k;  // mapped, never read
+  p2.Dv = p.Dk;
+  p2.o = R;
+  p2.S0 = nullptr;
+  p2.S_out = A;
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(q.side, q.prepass, 0);
+  if (e == cudaSuccess) e = dn::launch_chunk_main_only(p2, w, q.side, 64, false);
+  if (e == cudaSuccess) e = cudaEventRecord(q.hom, q.side);
+  // the forward beside it
+  if (e == cudaSuccess) e = dn::launch_chunk_main_only(p1, w, st, 64, false);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, q.hom, 0);
+  // join: the entry state of every segment and S_out, then the outputs
+  if (e == cudaSuccess) e = dn::launch_seg_combine(Send, A, Sin, p.S_out, BH, G, p.Dk, p.Dv, st);
+  if (e == cudaSuccess) e = dn::launch_seg_correct(p.o, R, Sin, BH, G, Tg, p.Dk, p.Dv, st);
+  return map_cuda(e);
+}
+
 }  // namespace
 
 extern "C" {
 
+int deltanet_seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
+  return seq_segments(B, H, T, Dk, Dv, C, dt, options);
+}
+
 size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
                                    unsigned int options) {
   if (options & ~kKnownOptions) return 0;
+  if (options & DN_OPT_SEQ_SPLIT) {
+    const size_t plain = deltanet_workspace_bytes_ex(B, H, T, Dk, Dv, C, dt, options & ~DN_OPT_SEQ_SPLIT);
+    const int G = seq_segments(B, H, T, Dk, Dv, C, dt, options);
+    if (plain == 0 || G == 1) return plain;
+    const size_t split = split_layout(B, H, T, Dk, Dv, G).bytes;
+    return split > plain ? split : plain;
+  }
   if (options == 0) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);
   if (C != 64 || deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt) == 0) return 0;
   // the pre-step alone runs on the tcgen05 path for bf16 (the per-chunk factors
@@ -261,6 +404,8 @@ int deltanet_chunk_fwd_ex(const void* q, const void* k, const void* v, const flo
   p.alpha_per_dim = (options & DN_OPT_GATE_PER_DIM) != 0;
   const int rc = validate_chunked(p, ws_bytes, workspace, options);
   if (rc != DN_OK) return rc;
+  const int G = seq_segments(B, H, T, Dk, Dv, C, dt, options);
+  if (G > 1) return run_split(p, G, workspace, static_cast<cudaStream_t>(cuda_stream));
   return run_chunked(p, workspace, cuda_stream);
 }
 

@@ -118,7 +118,9 @@ __device__ __forceinline__ void u_epilogue_half(uint32_t ws_addr, uint32_t uh_ad
   }
 }
 
-template <int DK, bool GATED, int DVS>
+// HOM: the homogeneous chain of the sequence split (v = 0, S0 = I); a
+// template switch, so that the plain kernels carry none of its code.
+template <int DK, bool GATED, int DVS, bool HOM>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmTb,
@@ -172,6 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (HOM) {  // the homogeneous chain: V is zero (no copy ever lands on these tiles)
+    for (int s = 0; s < NST; ++s)
+      for (int i = tid; i < (int)(kTile / 16); i += kThreads)
+        *reinterpret_cast<uint4*>(sm + s * L::STAGE + L::V_OFF + i * 16) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -182,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = warp_uniform(*tmem_slot);
   const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t tile_bytes = (2 * L::KB + (GATED ? 3 : 2)) * kTile;
+  const uint32_t tile_bytes = (2 * L::KB + (GATED ? 3 : 2) - (HOM ? 1 : 0)) * kTile;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(st + kb * L::KB_STRIDE + L::K_OFF, &tmK, full, kb * 64, c0, bh);
           tma_load_3d(st + kb * L::KB_STRIDE + L::Q_OFF, &tmQ, full, kb * 64, c0, bh);
         }
-        tma_load_3d(st + L::V_OFF, &tmV, full, jv, c0, bh);
+        if (!HOM) tma_load_3d(st + L::V_OFF, &tmV, full, jv, c0, bh);
         tma_load_3d(st + L::TB_OFF, &tmTb, full, 0, c0, bh);
         if (GATED) tma_load_3d(st + L::TBG_OFF, &tmTbg, full, 0, c0, bh);
       }
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_l2_3d(&tmK, kb * 64, cn, bh);
             prefetch_l2_3d(&tmQ, kb * 64, cn, bh);
           }
-          prefetch_l2_3d(&tmV, jv, cn, bh);
+          if (!HOM) prefetch_l2_3d(&tmV, jv, cn, bh);
           prefetch_l2_3d(&tmTb, 0, cn, bh);
           if (GATED) {
             prefetch_l2_3d(&tmTbg, 0, cn, bh);
@@ -500,6 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
       }
+      if (HOM) {  // the identity (Dv == Dk): row ct has its 1 in column ct
+#pragma unroll
+        for (int j = 0; j < DVS; ++j) sreg[j] = (ct == j0 + j) ? 1.f : 0.f;
+      }
 #pragma unroll
       for (int c16 = 0; c16 < DVS / 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(ct, c16), sreg + 8 * c16);
     }
@@ -608,13 +620,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-template <int DK, bool GATED, int DVS>
-cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+template <int DK, bool GATED, int DVS, bool HOM>
+cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st, bool after_prepass) {
   using L = MainLayout<DK, GATED>;
   const int BH = p.B * p.H;
   const int nchunks = (p.T + kC - 1) / kC;
-  cudaError_t e = launch_tsolve(p, w, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   CUtensorMap mq, mk, mv, mtb, mtbg;
   // with the layer's pre-step, q and k come mapped from the pre-pass (workspace)
   const void* qsrc = p.prestep ? static_cast<const void*>(w.qhat) : p.q;
@@ -624,7 +635,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
       !make_tmap_3d_bf16(&mtb, w.tb, kC, nchunks * kC, BH) ||
       !make_tmap_3d_bf16(&mtbg, GATED ? w.tbg : w.tb, kC, nchunks * kC, BH))
     return cudaErrorInvalidValue;
-  auto kern = chunk_main_kernel<DK, GATED, DVS>;
+  auto kern = chunk_main_kernel<DK, GATED, DVS, HOM>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(BH * (p.Dv / DVS)));
@@ -639,7 +650,7 @@ cudaError_t launch_t(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = after_prepass ? 1 : 0;  // otherwise griddepcontrol.wait returns at once
   return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mtb, mtbg, p, w.g);
 }
 
@@ -663,19 +674,31 @@ static int sm_count() {
 }
 
 template <int DK, bool GATED>
-cudaError_t launch_dvs(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
+cudaError_t launch_dvs(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st, int dvs, bool after) {
   // Each CTA runs the whole chunk chain of its (b, h, slice); the chain's
   // length per chunk hardly depends on the slice width.  When 64-column
   // slices leave most SMs idle (long sequences over few heads), 32-column
   // slices give twice the CTAs, as long as they still fit one wave.
-  if ((long long)p.B * p.H * (p.Dv / 32) <= sm_count()) return launch_t<DK, GATED, 32>(p, w, st);
-  return launch_t<DK, GATED, 64>(p, w, st);
+  if (p.hom) return dvs == 64 ? launch_t<DK, GATED, 64, true>(p, w, st, after) : cudaErrorInvalidValue;
+  if (dvs == 0) dvs = (long long)p.B * p.H * (p.Dv / 32) <= sm_count() ? 32 : 64;
+  if (dvs == 32) return launch_t<DK, GATED, 32, false>(p, w, st, after);
+  return launch_t<DK, GATED, 64, false>(p, w, st, after);
+}
+
+cudaError_t launch_chunk_main_only(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st, int dvs,
+                                   bool after_prepass) {
+  const bool gated = p.alpha != nullptr;
+  if (p.Dk == 128)
+    return gated ? launch_dvs<128, true>(p, w, st, dvs, after_prepass)
+                 : launch_dvs<128, false>(p, w, st, dvs, after_prepass);
+  return gated ? launch_dvs<64, true>(p, w, st, dvs, after_prepass)
+               : launch_dvs<64, false>(p, w, st, dvs, after_prepass);
 }
 
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st) {
-  const bool gated = p.alpha != nullptr;
-  if (p.Dk == 128) return gated ? launch_dvs<128, true>(p, w, st) : launch_dvs<128, false>(p, w, st);
-  return gated ? launch_dvs<64, true>(p, w, st) : launch_dvs<64, false>(p, w, st);
+  cudaError_t e = launch_tsolve(p, w, st);
+  if (e != cudaSuccess) return e;
+  return launch_chunk_main_only(p, w, st, 0, true);
 }
 
 }  // namespace dn

@@ -34,6 +34,11 @@ struct ChunkProblem {
   int prestep;         // Delta only: q, k raw and beta logits (silu + L2 normalise, sigmoid inside)
   int alpha_per_dim;   // Delta only: alpha is (B,H,T,Dk), one decay per key dimension
   unsigned int* status;  // device status word (workspace)
+  // Delta, tcgen05 C = 64 only: the homogeneous chain (v taken as zero, S0 as the
+  // identity, Dv == Dk): o receives the rows of R = (diag(gamma) Q - P W) S and
+  // S_out the product of the chunk transitions.  v must still point at a
+  // (B,H,T,Dv) bf16 tensor (it is mapped, never read).
+  int hom;
 };
 
 // CUDA-core (float32 arithmetic) chunked kernel: both modes, both input types.
@@ -85,6 +90,20 @@ cudaError_t launch_tsolve(const ChunkProblem& p, const WyWorkspace& w, cudaStrea
 // tcgen05 chunked delta rule after the pre-pass (bf16, C = 64).
 bool chunk_main_supported(const ChunkProblem& p);
 cudaError_t launch_chunk_main(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st);
+// The chunk kernel alone, its factors already in `w`: `dvs` = 64 or 32 (the Dv
+// slice width; 0 picks as launch_chunk_main does), `after_prepass` = launched
+// as a programmatic dependent of a pre-pass just enqueued on `st`.
+cudaError_t launch_chunk_main_only(const ChunkProblem& p, const WyWorkspace& w, cudaStream_t st, int dvs,
+                                   bool after_prepass);
+
+// The sequence split (segments run side by side, then combined; abi.cu):
+//   combine: per (b, h), Sin[1] = Send[0], Sin[g+1] = A[g] Sin[g] + Send[g],
+//            S_out = A[G-1] Sin[G-1] + Send[G-1]  (float32; G >= 2)
+//   correct: o rows of segment g >= 1 += R rows of segment g  Sin[g]  (bf16 o, R)
+cudaError_t launch_seg_combine(const float* Send, const float* A, float* Sin, float* S_out, int BH, int G,
+                               int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_seg_correct(void* o, const void* R, const float* Sin, int BH, int G, int Tg, int Dk,
+                               int Dv, cudaStream_t st);
 
 // tcgen05 chunked delta rule after the pre-pass (bf16, C = 128).
 bool chunk128_supported(const ChunkProblem& p);

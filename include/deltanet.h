@@ -129,8 +129,29 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   for the chunked call and (B,H,Dk) for the decode step: row i of the state
  *   decays by alpha_t[i] before the delta write ([P1], the KDA paragraph:
  *   scalar gating replaced by per-dimension gating).  alpha must not be NULL.
+ * DN_OPT_SEQ_SPLIT (chunked call; ignored by the decode step): permission to
+ *   cut each sequence into G segments that run side by side.  The chunk
+ *   transition is affine in the state ([P3] "DeltaNet (Parallelizing linear
+ *   transformers with delta rule)": a product of generalised Householder
+ *   factors plus a write), so segment g >= 1 runs from a zero state next to
+ *   its homogeneous chain (v = 0, S0 = I), and the segments are joined after:
+ *   entry states Sin[g+1] = A_g Sin[g] + Send_g, outputs O_g += R_g Sin[g].
+ *   The result equals the unsplit call up to rounding (R and the entry states
+ *   enter one product in bf16).  The library takes G > 1 only for bf16
+ *   inputs, C = 64, no other option, G <= 16 dividing T, at least 8 chunks
+ *   per segment, and few enough heads that both chains of every segment fit
+ *   the GPU's SMs at once (B*H*G*(Dk + Dv)/64 <= SM count); among those it
+ *   picks the G with the shortest estimated critical path (chunks per
+ *   segment, plus about three chunks per segment boundary for the join, plus
+ *   a fixed eight), and G = 1 when no split beats the plain call's T/64
+ *   chunks.  deltanet_seq_segments gives G.  With G > 1 the workspace
+ *   (deltanet_workspace_bytes_ex) adds
+ *   B*H*T*Dk bf16 values and four (B*H*G, Dk, Dv | Dk) float32 state arrays,
+ *   and the call uses a second stream of the library's own, joined to
+ *   cuda_stream by events.
  *
- * Paths: the options are built for C = 64 (C = 128 gives DN_ERR_UNSUPPORTED).
+ * Paths: DN_OPT_PRESTEP and DN_OPT_GATE_PER_DIM are built for C = 64 (C = 128
+ * gives DN_ERR_UNSUPPORTED; DN_OPT_SEQ_SPLIT alone runs unsplit there).
  * DN_OPT_PRESTEP alone on bf16 inputs runs on the tcgen05 path: the pre-pass
  * maps each chunk's q and k once and writes them to the workspace, where the
  * chunk kernel reads them (the workspace of deltanet_workspace_bytes plus
@@ -143,8 +164,14 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  */
 enum {
     DN_OPT_PRESTEP = 1,
-    DN_OPT_GATE_PER_DIM = 2
+    DN_OPT_GATE_PER_DIM = 2,
+    DN_OPT_SEQ_SPLIT = 4
 };
+
+/* The number of segments G a deltanet_chunk_fwd_ex call with these arguments
+ * runs (1: no split), for the current device.  Host only. */
+int deltanet_seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                          unsigned int options);
 
 /* deltanet_workspace_bytes for a deltanet_chunk_fwd_ex call with `options`. */
 size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,

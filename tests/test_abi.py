@@ -234,7 +234,7 @@ def test_option_flags_are_validated_on_the_host(L):
                                        vp(alpha), None, vp(A + 256 * MB), vp(A + 320 * MB),
                                        2, 2, T, 64, 64, C, 1, opts, vp(A + 400 * MB), 1 << 20, None)
 
-    assert ex(4) == E.DN_ERR_INVALID_ARG
+    assert ex(8) == E.DN_ERR_INVALID_ARG
     assert ex(E.DN_OPT_GATE_PER_DIM) == E.DN_ERR_INVALID_ARG  # per-dimension gate needs alpha
     assert ex(E.DN_OPT_PRESTEP, C=128) == E.DN_ERR_UNSUPPORTED
     assert ex(E.DN_OPT_GATE_PER_DIM, alpha=A + 500 * MB, C=128) == E.DN_ERR_UNSUPPORTED
@@ -251,6 +251,17 @@ def test_option_flags_are_validated_on_the_host(L):
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 3) == 256
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 128, 1, 1) == 0
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 8) == 0
+    # the sequence split is a permission: where it does not apply (here: no GPU to
+    # size it against, float32, C = 128, other options) the call runs unsplit
+    plain = L.deltanet_workspace_bytes(2, 2, 4096, 64, 64, 64, 1)
+    assert L.deltanet_workspace_bytes_ex(2, 2, 4096, 64, 64, 64, 1, 4) == plain
+    assert L.deltanet_workspace_bytes_ex(2, 2, 4096, 64, 64, 128, 1, 4) == \
+        L.deltanet_workspace_bytes(2, 2, 4096, 64, 64, 128, 1)
+    assert L.deltanet_workspace_bytes_ex(2, 2, 4096, 64, 64, 64, 0, 4) == 256
+    assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 5) == \
+        L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 1)
+    for opts in (4, 5, 6):
+        assert L.deltanet_seq_segments(2, 2, 4096, 64, 64, 64, 1, opts) == 1
     assert L.deltanet_workspace_bytes_ex(2, 2, 100, 64, 64, 64, 1, 0) == \
         L.deltanet_workspace_bytes(2, 2, 100, 64, 64, 64, 1)
 
@@ -258,7 +269,7 @@ def test_option_flags_are_validated_on_the_host(L):
         return L.deltanet_decode_step_ex(vp(A), vp(A + MB), vp(A + 2 * MB), vp(A + 3 * MB), vp(alpha),
                                          vp(A + 8 * MB), vp(A + 4 * MB), 4, 2, 128, 128, 1, opts, None)
 
-    assert dec(4) == E.DN_ERR_INVALID_ARG
+    assert dec(8) == E.DN_ERR_INVALID_ARG
     assert dec(E.DN_OPT_GATE_PER_DIM) == E.DN_ERR_INVALID_ARG
     # a (B,H,Dk) alpha of 4*2*128 floats starting 1 KB before S overlaps S
     assert dec(E.DN_OPT_GATE_PER_DIM, alpha=A + 8 * MB - 1024) == E.DN_ERR_INVALID_ARG
