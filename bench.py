@@ -510,15 +510,17 @@ def profile_run(args):
 
     dev = torch.device("cuda", 0)
     n = args.warmup + 1
-    if args.profile in ("chunk", "gated", "linear", "long64", "long128", "long64q", "long128q", "split8"):
+    if args.profile in ("chunk", "gated", "linear", "long64", "long128", "long64q", "long128q", "split8",
+                        "split2"):
         # long64q / long128q: the long workloads on a quarter of the sequence
         # (T = 16384, still far larger than L2), small enough for a full ncu capture;
-        # split8: the long workload over 8 heads (B1 H8 T65536) with the sequence split
+        # split8 / split2: the long workload over 8 / 2 heads (B1 T65536) with the sequence split
         quarter = lambda w: dataclasses.replace(w, T=w.T // 4, name=w.name.replace("T65536", "T16384"))
         w = {"chunk": gen.PREFILL, "gated": gen.FORGET, "linear": gen.PREFILL_LINEAR,
              "long64": gen.LONG64, "long128": gen.LONG128,
              "long64q": quarter(gen.LONG64), "long128q": quarter(gen.LONG128),
-             "split8": dataclasses.replace(gen.LONG64, H=8, name=gen.LONG64.name.replace("H32", "H8"))
+             "split8": dataclasses.replace(gen.LONG64, H=8, name=gen.LONG64.name.replace("H32", "H8")),
+             "split2": dataclasses.replace(gen.LONG64, H=2, name=gen.LONG64.name.replace("H32", "H2")),
              }[args.profile]
         x = gen.make_workload(w, seed=0, device=dev)
         for _ in range(n):
@@ -526,7 +528,7 @@ def profile_run(args):
                 dn.linear_attn_fwd(x["q"], x["k"], x["v"], C=w.C)
             else:
                 dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C,
-                                      seq_split=args.profile == "split8")
+                                      seq_split=args.profile.startswith("split"))
     else:
         B, H, D = gen.DECODE_SEQS, gen.DECODE_HEADS, 128
         S = torch.randn(B, H, D, D, device=dev) * 0.01
@@ -549,7 +551,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--profile", choices=["chunk", "linear", "gated", "long64", "long128", "long64q", "long128q",
-                                          "split8", "decode"],
+                                          "split8", "split2", "decode"],
                     default=None,
                     help="untimed run for a profiler: --warmup launches of one kernel on its "
                          "workload, then one more (the one to capture)")

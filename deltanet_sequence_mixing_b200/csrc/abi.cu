@@ -218,10 +218,10 @@ constexpr int kMinSegChunks = 8;       // 64-token chunks per segment, at least
 constexpr int kMaxSegments = 16;
 // The segment count minimises an estimate of the critical path in units of one
 // chunk of the chain (about 1.35 us on the B200): the chunks of one segment,
-// plus the sequential join (one step per segment boundary, about three chunks
-// each), plus the fixed cost of the split (the homogeneous chain's start, the
-// join's launches and the output correction, about eight chunks).
-constexpr int kJoinStepChunks = 3;
+// plus the sequential join (one step per segment boundary, about 2.7 us, two
+// chunks), plus the fixed cost of the split (the homogeneous chain's start,
+// the join's launches and the output correction, about eight chunks).
+constexpr int kJoinStepChunks = 2;
 constexpr int kSplitFixedChunks = 8;
 
 int sm_count_now() {

@@ -142,7 +142,7 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   per segment, and few enough heads that both chains of every segment fit
  *   the GPU's SMs at once (B*H*G*(Dk + Dv)/64 <= SM count); among those it
  *   picks the G with the shortest estimated critical path (chunks per
- *   segment, plus about three chunks per segment boundary for the join, plus
+ *   segment, plus about two chunks per segment boundary for the join, plus
  *   a fixed eight), and G = 1 when no split beats the plain call's T/64
  *   chunks.  deltanet_seq_segments gives G.  With G > 1 the workspace
  *   (deltanet_workspace_bytes_ex) adds
