@@ -11,6 +11,7 @@ per-head rel-L2 of each workload is printed as a diagnostic.  Sizes:
   prefill-linear  the same shape, ELU+1 linear attention
   long            B1 H32 T65536 D128 bf16, C64 and C128
   forget          B8 H16 T8192 D128 bf16 gated C64
+  long, 8 heads   B1 H8 T65536 D128 bf16 C64 with the sequence split
   decode          256 sequences x 32 heads, D128, fp32 states from a 512-token
                   prefill, then 1024 single-token steps with fresh inputs:
                   every state's final S and every step's output
@@ -145,3 +146,33 @@ def test_full_size_decode_all_states(dn, oracle_mod, capsys):
         eo[sl] = _per_head(o_dec[sl].float().numpy(), o_ref[0, :, n_pre:])
         es[sl] = _per_head(S_c[sl].numpy(), S_ref[0])
     _report(capsys, "decode 256x32 D128, 1024 steps", {"o": eo, "S": es})
+
+
+def test_full_size_sequence_split_all_heads(dn, oracle_mod, capsys):
+    """The long workload over 8 heads (B1 H8 T65536 D128 bf16 C64) with the
+    sequence split, as the benchmark times it (4 segments on the B200): every
+    head against the float64 oracle of the unsplit recurrence."""
+    import dataclasses
+
+    w = dataclasses.replace(gen.LONG64, H=8, name=gen.LONG64.name.replace("H32", "H8"))
+    G = dn.seq_segments(w.B, w.H, w.T, w.Dk, w.Dv)
+    assert G > 1
+    dev = torch.device("cuda")
+    x = gen.make_workload(w, seed=12, device=dev)
+    o = torch.empty_like(x["v"])
+    S = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev)
+    dn.deltanet_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["alpha"], C=w.C, o=o, S_out=S, seq_split=True)
+    torch.cuda.synchronize()
+    assert dn.deltanet_get_device_status() == 0
+    fx = {k: _flat(v) for k, v in x.items()}
+    o_c, S_c = _flat(o).float(), _flat(S)
+    del x, o, S
+    n = w.B * w.H
+    eo, es = np.zeros(n), np.zeros(n)
+    per = max(1, (1 << 28) // (w.T * w.Dv * 8))
+    for sl in _batches(n, per):
+        sub = {k: (None if v is None else v[sl].unsqueeze(0)) for k, v in fx.items()}
+        o_ref, S_ref = oracle_mod.deltanet(sub["q"], sub["k"], sub["v"], sub["beta"], sub["alpha"])
+        eo[sl] = _per_head(o_c[sl].numpy(), o_ref[0])
+        es[sl] = _per_head(S_c[sl].numpy(), S_ref[0])
+    _report(capsys, f"{w.name}, sequence split into {G} segments", {"o": eo, "S": es})
