@@ -232,7 +232,8 @@ int sm_count_now() {
 }
 
 int seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
-  if (options != DN_OPT_SEQ_SPLIT || dt != DN_BF16 || C != 64 || T <= 0) return 1;
+  // the split runs the tcgen05 path: bf16, C = 64, optionally with the layer's pre-step
+  if ((options & ~DN_OPT_PRESTEP) != DN_OPT_SEQ_SPLIT || dt != DN_BF16 || C != 64 || T <= 0) return 1;
   if (!valid_dim(Dk) || !valid_dim(Dv) || B < 1 || H < 1) return 1;
   const int sms = sm_count_now();
   int best = 1;
@@ -255,7 +256,7 @@ struct SplitLayout {  // byte offsets inside the workspace
   size_t wy, R, S0seg, Send, A, Sin, bytes;
 };
 
-SplitLayout split_layout(int B, int H, int T, int Dk, int Dv, int G) {
+SplitLayout split_layout(int B, int H, int T, int Dk, int Dv, int G, bool prestep) {
   const size_t BH = (size_t)B * H, BHG = BH * G;
   SplitLayout L{};
   size_t off = kStatusBytes;
@@ -264,7 +265,9 @@ SplitLayout split_layout(int B, int H, int T, int Dk, int Dv, int G) {
     off += (n + 255) / 256 * 256;
     return at;
   };
-  L.wy = take(dn::wy_workspace_bytes(1, (int)BHG, T / G, 64));
+  // the pre-pass factors (and, with the pre-step, the mapped k and q after them)
+  const size_t wy = dn::wy_workspace_bytes(1, (int)BHG, T / G, 64);
+  L.wy = take(prestep ? (wy + 255) / 256 * 256 + dn::wy_khat_bytes(1, (int)BHG, T / G, Dk) : wy);
   L.R = take(BH * T * Dk * 2);
   L.S0seg = take(BHG * Dk * Dv * 4);
   L.Send = take(BHG * Dk * Dv * 4);
@@ -296,7 +299,7 @@ int run_split(dn::ChunkProblem& p, int G, void* ws, cudaStream_t st) {
     if (e != cudaSuccess) return map_cuda(e);
     q.ready = true;
   }
-  const SplitLayout L = split_layout(p.B, p.H, p.T, p.Dk, p.Dv, G);
+  const SplitLayout L = split_layout(p.B, p.H, p.T, p.Dk, p.Dv, G, p.prestep);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int BH = p.B * p.H, Tg = p.T / G;
   const size_t blk = (size_t)p.Dk * p.Dv * sizeof(float);
@@ -356,7 +359,7 @@ size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, d
     const size_t plain = deltanet_workspace_bytes_ex(B, H, T, Dk, Dv, C, dt, options & ~DN_OPT_SEQ_SPLIT);
     const int G = seq_segments(B, H, T, Dk, Dv, C, dt, options);
     if (plain == 0 || G == 1) return plain;
-    const size_t split = split_layout(B, H, T, Dk, Dv, G).bytes;
+    const size_t split = split_layout(B, H, T, Dk, Dv, G, (options & DN_OPT_PRESTEP) != 0).bytes;
     return split > plain ? split : plain;
   }
   if (options == 0) return deltanet_workspace_bytes(B, H, T, Dk, Dv, C, dt);

@@ -138,7 +138,9 @@ int deltanet_chunk_fwd(const void *q, const void *k, const void *v,
  *   entry states Sin[g+1] = A_g Sin[g] + Send_g, outputs O_g += R_g Sin[g].
  *   The result equals the unsplit call up to rounding (R and the entry states
  *   enter one product in bf16).  The library takes G > 1 only for bf16
- *   inputs, C = 64, no other option, G <= 16 dividing T, at least 8 chunks
+ *   inputs, C = 64, no other option but DN_OPT_PRESTEP (the pre-pass then
+ *   maps q and k once, and both chains read the mapped copies), G <= 16
+ *   dividing T, at least 8 chunks
  *   per segment, and few enough heads that both chains of every segment fit
  *   the GPU's SMs at once (B*H*G*(Dk + Dv)/64 <= SM count); among those it
  *   picks the G with the shortest estimated critical path (chunks per

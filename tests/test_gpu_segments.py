@@ -67,6 +67,41 @@ def test_split_matches_oracle(dn, oracle_mod, B, H, T, Dk, Dv, gated, with_s0, G
     assert rel_l2(o, o1) <= 1e-2 and rel_l2(S, S1) <= 1e-2
 
 
+def test_split_with_the_layer_prestep(dn, oracle_mod):
+    """The split with the layer's pre-step inside (raw q, k projections and
+    beta logits; the pre-pass maps them once for both chains)."""
+    B, H, T = 1, 2, 4096
+    assert dn.seq_segments(B, H, T, 128, 128, prestep=True) == 4
+    x = gen.make_inputs(B, H, T, 128, 128, torch.bfloat16, gated=True, seed=31, raw=True)
+    S0 = torch.randn(B, H, 128, 128, generator=torch.Generator().manual_seed(31)) * 0.1
+    g = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    o, S = dn.deltanet_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["alpha"], S0.cuda(), C=64, prestep=True,
+                                 seq_split=True)
+    torch.cuda.synchronize()
+    assert dn.deltanet_get_device_status() == 0
+    o_ref, S_ref = oracle_mod.deltanet(x["q"], x["k"], x["v"], x["beta"], x["alpha"], S0.double(), prestep=True)
+    eo, es = rel_l2(o.float().cpu().numpy(), o_ref), rel_l2(S.cpu().numpy(), S_ref)
+    assert eo <= TOL and es <= TOL, f"rel-L2 o={eo:.3e} S={es:.3e}"
+    o1, S1 = dn.deltanet_chunk_fwd(g["q"], g["k"], g["v"], g["beta"], g["alpha"], S0.cuda(), C=64, prestep=True)
+    torch.cuda.synchronize()
+    assert rel_l2(o.float().cpu().numpy(), o1.float().cpu().numpy()) <= 1e-2
+    assert rel_l2(S.cpu().numpy(), S1.cpu().numpy()) <= 1e-2
+
+
+def test_split_workspace_sizes(dn):
+    """With G > 1 the workspace grows by the split's arrays; the pre-step adds
+    the mapped k and q (B*H*T*Dk bf16 each, from 256-byte boundaries)."""
+    L = dn.lib()
+    B, H, T, D = 1, 2, 4096, 128
+    r256 = lambda x: (x + 255) // 256 * 256
+    plain = L.deltanet_workspace_bytes_ex(B, H, T, D, D, 64, 1, 0)
+    split = L.deltanet_workspace_bytes_ex(B, H, T, D, D, 64, 1, 4)
+    split_pre = L.deltanet_workspace_bytes_ex(B, H, T, D, D, 64, 1, 5)
+    # R (B*H*T*Dk bf16) and four (B*H*G, Dk, Dv) float32 states at least
+    assert split >= plain + B * H * T * D * 2 + 4 * B * H * 4 * D * D * 4
+    assert split_pre - split == 2 * r256(B * H * T * D * 2)
+
+
 def test_split_in_place_state(dn, oracle_mod):
     """S_out may be S0 itself: the split reads S0 before it writes S_out."""
     B, H, T = 1, 2, 4096
