@@ -22,9 +22,11 @@
 // ahead) as soon as the last MMA of a chunk has read them, overlapping the
 // output / state epilogue.
 //
-// One CTA per (b, h, 64-column slice of Dv), 5 warps: warps 0-3 own TMEM lanes
-// 0-127 (one chunk row each) and run the epilogues; warp 4 loads (one lane)
-// and issues the MMAs (warp-uniform, one elected lane).  Waits are bounded; a
+// One CTA per (b, h, 64-column slice of Dv), 9 warps: warps 0-7 run the
+// epilogues, warps w and w + 4 on the same TMEM lanes 32 (w % 4) .. + 31 (one
+// chunk row per lane), each taking one half of every epilogue's columns (and
+// of the state's); warp 8 loads (one lane) and issues the MMAs (warp-uniform,
+// one elected lane).  Waits are bounded; a
 // wait that runs out sets the status word and the CTA winds down without
 // trapping.
 #include <cuda.h>
@@ -39,7 +41,8 @@ namespace {
 constexpr int kC = 128;
 constexpr int kDVS = 64;
 constexpr uint32_t kBlk = 16384;  // 128 rows x 128 bytes: one 64-column block of a 128-row tile
-constexpr int kThreads = 160;
+constexpr int kThreads = 288;  // epilogues 0-7, loads and MMA issue 8
+constexpr int kEpi = 256;
 constexpr int kBarEpi = 1;
 
 template <int DK, bool GATED>
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtl wc{abort_flag, p.status, kWaitLimitNs};
   const uint32_t tile_bytes = (2 * L::KB * 2 + 2 + 4 + (GATED ? 4 : 0)) * 8192u;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // --------------------------------------------------- loads and MMA issue --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -259,22 +262,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     (void)mbar_wait(bar + B_FIN, 0, fin);
   } else {
     // -------------------------------------------------------------- epilogues --
-    const int r = tid;  // chunk row = TMEM lane
+    const int r = tid & 127;  // chunk row = TMEM lane
+    const int hf = tid >> 7;  // which half of the columns this thread takes
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const size_t s_base = (size_t)bh * DK * Dv;
-    float sreg[kDVS];
+    float sreg[kDVS / 2];  // columns j0 + 32 hf .. + 31 of state row r
     if (r < DK) {
-      const float* src = p.S0 ? p.S0 + s_base + (size_t)r * Dv + j0 : nullptr;
+      const float* src = p.S0 ? p.S0 + s_base + (size_t)r * Dv + j0 + 32 * hf : nullptr;
 #pragma unroll
-      for (int j = 0; j < kDVS; j += 4) {
+      for (int j = 0; j < kDVS / 2; j += 4) {
         const float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         sreg[j] = v.x; sreg[j + 1] = v.y; sreg[j + 2] = v.z; sreg[j + 3] = v.w;
       }
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(r, c16), sreg + 8 * c16);
+      for (int c = 0; c < 4; ++c) st_bf16x8(sm + L::S_OFF + sw128_off(r, 4 * hf + c), sreg + 8 * c);
     }
     fence_proxy_async_smem();
-    named_bar_sync(kBarEpi, 128);
+    named_bar_sync(kBarEpi, kEpi);
     if (tid == 0) mbar_arrive(bar + B_SREADY);  // the initial state tile is in place
 
     bool ok = true;
@@ -283,13 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c0 = c * kC, n = min(kC, T - c0);
       const float* gv = gvec + par * kC;
       // ---- P rows (masked, decayed), W rows; gated: Q <- diag(gamma) Q ----
-      ok = named_bar_and(kBarEpi, 128, mbar_wait(bar + B_MMAA, par, wc));
+      ok = named_bar_and(kBarEpi, kEpi, mbar_wait(bar + B_MMAA, par, wc));
       if (!ok) break;
       tc_fence_after();
       {
         const float gr = GATED ? gv[r] : 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int qq = 0; qq < 2; ++qq) {  // P columns 64 hf .. + 63, 32 at a time
+          const int q = 2 * hf + qq;
           uint32_t v[32];
           tmem_ld32(tmem + lane_base + TM::P + q * 32, v);
           tmem_wait_ld();
@@ -306,8 +311,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_bf16x8(sm + L::P_OFF + (q >> 1) * kBlk + sw128_off(r, (q & 1) * 4 + cc), x);
           }
         }
+        constexpr int WQ = DK / 64;  // 32-column groups of W per half
 #pragma unroll
-        for (int q = 0; q < DK / 32; ++q) {
+        for (int qq = 0; qq < WQ; ++qq) {
+          const int q = hf * WQ + qq;
           uint32_t v[32];
           tmem_ld32(tmem + lane_base + TM::W + q * 32, v);
           tmem_wait_ld();
@@ -317,100 +324,94 @@ __global__ void __launch_bounds__(kThreads, 1)
                       reinterpret_cast<const float*>(v) + cc * 8);
         }
         if (GATED) {
-          // (each 64-column block loaded whole before its stores, which the
-          // compiler cannot tell apart from the loads)
+          // (this thread's half of each 64-column block loaded whole before its
+          // stores, which the compiler cannot tell apart from the loads)
           const float gam = __expf(gr);
 #pragma unroll
           for (int kb = 0; kb < DK / 64; ++kb) {
-            uint4 u[8];
+            uint4 u[4];
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16)
-              u[c16] = *reinterpret_cast<const uint4*>(sm + L::Q_OFF + kb * kBlk + sw128_off(r, c16));
+            for (int c4 = 0; c4 < 4; ++c4)
+              u[c4] = *reinterpret_cast<const uint4*>(sm + L::Q_OFF + kb * kBlk + sw128_off(r, 4 * hf + c4));
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
+            for (int c4 = 0; c4 < 4; ++c4) {
               float x[8];
-              unpack_bf16x8(u[c16], x);
+              unpack_bf16x8(u[c4], x);
 #pragma unroll
               for (int e = 0; e < 8; ++e) x[e] *= gam;
-              st_bf16x8(sm + L::Q_OFF + kb * kBlk + sw128_off(r, c16), x);
+              st_bf16x8(sm + L::Q_OFF + kb * kBlk + sw128_off(r, 4 * hf + c4), x);
             }
           }
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(kBarEpi, 128);
+      named_bar_sync(kBarEpi, kEpi);
       if (tid == 0) mbar_arrive(bar + B_EPIA);
 
-      // ---- U = Uh - WS (gated also U~ = U e^(g_last - g_r)) ----
-      ok = named_bar_and(kBarEpi, 128, mbar_wait(bar + B_MMAB, par, wc));
+      // ---- U = Uh - WS (gated also U~ = U e^(g_last - g_r)), columns 32 hf .. + 31 ----
+      ok = named_bar_and(kBarEpi, kEpi, mbar_wait(bar + B_MMAB, par, wc));
       if (!ok) break;
       tc_fence_after();
       {
         const float wl = GATED ? __expf(gv[n - 1] - gv[r]) : 1.f;
+        uint32_t ws[32], uh[32];
+        tmem_ld32(tmem + lane_base + TM::WS + hf * 32, ws);
+        tmem_ld32(tmem + lane_base + TM::UH + hf * 32, uh);
+        tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t ws[32], uh[32];
-          tmem_ld32(tmem + lane_base + TM::WS + h * 32, ws);
-          tmem_ld32(tmem + lane_base + TM::UH + h * 32, uh);
-          tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+          float x[8], y[8];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float x[8], y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              x[e] = __uint_as_float(uh[cc * 8 + e]) - __uint_as_float(ws[cc * 8 + e]);
-              y[e] = x[e] * wl;
-            }
-            st_bf16x8(sm + L::U_OFF + sw128_off(r, h * 4 + cc), x);
-            if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(r, h * 4 + cc), y);
+          for (int e = 0; e < 8; ++e) {
+            x[e] = __uint_as_float(uh[cc * 8 + e]) - __uint_as_float(ws[cc * 8 + e]);
+            y[e] = x[e] * wl;
           }
+          st_bf16x8(sm + L::U_OFF + sw128_off(r, hf * 4 + cc), x);
+          if (GATED) st_bf16x8(sm + L::UT_OFF + sw128_off(r, hf * 4 + cc), y);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(kBarEpi, 128);
+      named_bar_sync(kBarEpi, kEpi);
       if (tid == 0) mbar_arrive(bar + B_EPIB);
 
-      // ---- O rows -> global; S <- gamma_last S + dS ----
-      ok = named_bar_and(kBarEpi, 128, mbar_wait(bar + B_MMAC, par, wc));
+      // ---- O rows -> global; S <- gamma_last S + dS (columns 32 hf .. + 31) ----
+      ok = named_bar_and(kBarEpi, kEpi, mbar_wait(bar + B_MMAC, par, wc));
       if (!ok) break;
       tc_fence_after();
       {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + r) * Dv + j0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * T + c0 + r) * Dv + j0 + 32 * hf;
+        {
           uint32_t ov[32];
-          tmem_ld32(tmem + lane_base + TM::QS + h * 32, ov);
+          tmem_ld32(tmem + lane_base + TM::QS + hf * 32, ov);
           tmem_wait_ld();
           if (r < n) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) st_bf16x8(orow + h * 32 + cc * 8, reinterpret_cast<const float*>(ov) + cc * 8);
+            for (int cc = 0; cc < 4; ++cc) st_bf16x8(orow + cc * 8, reinterpret_cast<const float*>(ov) + cc * 8);
           }
         }
         if (r < DK) {
           const float carry = GATED ? __expf(gv[n - 1]) : 1.f;
+          uint32_t ds[32];
+          tmem_ld32(tmem + lane_base + TM::DS + hf * 32, ds);
+          tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t ds[32];
-            tmem_ld32(tmem + lane_base + TM::DS + h * 32, ds);
-            tmem_wait_ld();
+          for (int e = 0; e < 32; ++e) sreg[e] = fmaf(carry, sreg[e], __uint_as_float(ds[e]));
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sreg[h * 32 + e] = fmaf(carry, sreg[h * 32 + e], __uint_as_float(ds[e]));
-          }
-#pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) st_bf16x8(sm + L::S_OFF + sw128_off(r, c16), sreg + 8 * c16);
+          for (int c4 = 0; c4 < 4; ++c4) st_bf16x8(sm + L::S_OFF + sw128_off(r, 4 * hf + c4), sreg + 8 * c4);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(kBarEpi, 128);
+      named_bar_sync(kBarEpi, kEpi);
       if (tid == 0) mbar_arrive(bar + B_SREADY);
     }
     if (p.S_out && r < DK) {
-      float* dst = p.S_out + s_base + (size_t)r * Dv + j0;
+      float* dst = p.S_out + s_base + (size_t)r * Dv + j0 + 32 * hf;
 #pragma unroll
-      for (int j = 0; j < kDVS; j += 4)
+      for (int j = 0; j < kDVS / 2; j += 4)
         *reinterpret_cast<float4*>(dst + j) = make_float4(sreg[j], sreg[j + 1], sreg[j + 2], sreg[j + 3]);
     }
   }
