@@ -35,6 +35,7 @@ SIGNATURES = {
                                      _vp]),
     "deltanet_workspace_bytes_ex": (_sz, [_i, _i, _i, _i, _i, _i, _i, _u]),
     "deltanet_seq_segments": (_i, [_i, _i, _i, _i, _i, _i, _i, _u]),
+    "deltanet_seq_segments_sm": (_i, [_i, _i, _i, _i, _i, _i, _i, _u, _i]),
     "deltanet_chunk_fwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _i, _i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp]),
     "linear_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

@@ -231,11 +231,10 @@ int sm_count_now() {
   return n;
 }
 
-int seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
+int seq_segments_for(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options, int sms) {
   // the split runs the tcgen05 path: bf16, C = 64, optionally with the layer's pre-step
   if ((options & ~DN_OPT_PRESTEP) != DN_OPT_SEQ_SPLIT || dt != DN_BF16 || C != 64 || T <= 0) return 1;
-  if (!valid_dim(Dk) || !valid_dim(Dv) || B < 1 || H < 1) return 1;
-  const int sms = sm_count_now();
+  if (!valid_dim(Dk) || !valid_dim(Dv) || B < 1 || H < 1 || sms < 1) return 1;
   int best = 1;
   long long best_cost = (T + 63) / 64;  // the plain call
   for (int G = 2; G <= kMaxSegments; ++G) {
@@ -250,6 +249,10 @@ int seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsign
     }
   }
   return best;
+}
+
+int seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
+  return seq_segments_for(B, H, T, Dk, Dv, C, dt, options, sm_count_now());
 }
 
 struct SplitLayout {  // byte offsets inside the workspace
@@ -350,6 +353,11 @@ extern "C" {
 
 int deltanet_seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options) {
   return seq_segments(B, H, T, Dk, Dv, C, dt, options);
+}
+
+int deltanet_seq_segments_sm(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt, unsigned int options,
+                             int sm_count) {
+  return seq_segments_for(B, H, T, Dk, Dv, C, dt, options, sm_count);
 }
 
 size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,

@@ -175,6 +175,11 @@ enum {
 int deltanet_seq_segments(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
                           unsigned int options);
 
+/* The same rule for a GPU with sm_count SMs (1 when sm_count < 1): plans a
+ * split for another device, or checks the rule without one.  Host only. */
+int deltanet_seq_segments_sm(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
+                             unsigned int options, int sm_count);
+
 /* deltanet_workspace_bytes for a deltanet_chunk_fwd_ex call with `options`. */
 size_t deltanet_workspace_bytes_ex(int B, int H, int T, int Dk, int Dv, int C, dn_dtype dt,
                                    unsigned int options);

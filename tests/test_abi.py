@@ -273,3 +273,35 @@ def test_option_flags_are_validated_on_the_host(L):
     assert dec(E.DN_OPT_GATE_PER_DIM) == E.DN_ERR_INVALID_ARG
     # a (B,H,Dk) alpha of 4*2*128 floats starting 1 KB before S overlaps S
     assert dec(E.DN_OPT_GATE_PER_DIM, alpha=A + 8 * MB - 1024) == E.DN_ERR_INVALID_ARG
+
+
+def test_sequence_split_segment_rule(L):
+    """The segment count the split takes, for a 148-SM B200 and other SM
+    counts (host logic, no GPU): a divisor G <= 16 of T with at least 8 chunks
+    per segment and B*H*G*(Dk + Dv)/64 <= SMs, minimising T/(64 G) + 2 (G - 1)
+    + 8 chunk periods, and 1 when nothing beats the plain call's T/64."""
+    seg = lambda B, H, T, Dk=128, Dv=128, opts=4, sms=148, C=64, dt=1: \
+        L.deltanet_seq_segments_sm(B, H, T, Dk, Dv, C, dt, opts, sms)
+    assert seg(1, 16, 4096) == 2        # as many heads as two segments allow
+    assert seg(1, 2, 4096) == 4
+    assert seg(1, 3, 3000, 128, 64) == 4
+    assert seg(2, 2, 2200, 64, 64) == 4
+    assert seg(1, 1, 9100) == 7         # odd counts when T's divisors call for them
+    assert seg(1, 1, 32768) == 16
+    assert seg(1, 8, 65536) == 4
+    assert seg(1, 4, 65536) == 8
+    assert seg(1, 32, 65536) == 1       # the plain chain already fills the SMs
+    assert seg(4, 16, 1024) == 1
+    assert seg(1, 1, 1000) == 1         # too short for two 8-chunk segments to pay
+    # fewer SMs: both chains of every segment must fit one wave
+    assert seg(1, 8, 65536, sms=64) == 2
+    assert seg(1, 8, 65536, sms=63) == 1
+    # only bf16, C = 64, and no option besides the pre-step
+    assert seg(1, 2, 4096, opts=5) == 4
+    assert seg(1, 2, 4096, opts=0) == 1
+    assert seg(1, 2, 4096, opts=6) == 1
+    assert seg(1, 2, 4096, opts=7) == 1
+    assert seg(1, 2, 4096, dt=0) == 1
+    assert seg(1, 2, 4096, C=128) == 1
+    assert seg(1, 2, 4096, Dk=96) == 1
+    assert seg(1, 2, 4096, sms=0) == 1
