@@ -15,10 +15,11 @@
 //   1. K (rows past T zero) -> shared memory; beta, log-alpha prefix g.
 //   2. G = K K^T by tcgen05 (bf16 operands from the swizzled K tile, float32
 //      accumulator in TMEM), read back row by row into A, masked and scaled.
-//   3. C/16 diagonal 16x16 inverses (one column per lane, right-looking
-//      substitution so only one multiply-add per step is on the dependency
-//      chain), then the blocks below the diagonal from the 2 x 2 block
-//      inverse [[L11, 0], [L21, L22]]^-1 = [[T1, 0], [-T2 L21 T1, T2]] applied
+//   3. C/16 diagonal 16x16 inverses (two per warp, one per half-warp; one
+//      column per lane, right-looking substitution so only one multiply-add
+//      per step is on the dependency chain), then the blocks below the
+//      diagonal from the 2 x 2 block inverse
+//      [[L11, 0], [L21, L22]]^-1 = [[T1, 0], [-T2 L21 T1, T2]] applied
 //      recursively (64 x 64 halves of 32 x 32 halves), with tf32 WMMA products
 //      spread over all warps: four dependent levels at C = 64, six at C = 128.
 //   4. Tb, Tbg -> global (row-major bf16 C x C tiles).
@@ -253,11 +254,12 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
   tc_fence_before();
   __syncthreads();
 
-  // 3. T = (I + A)^-1.  Diagonal 16x16 blocks D_w: warp w, lanes 0-15 own
-  //    column j; right-looking, so only one multiply-add per step is on the
-  //    dependency chain.
-  if (lane < 16) {
-    const int o = 16 * warp, j = lane;
+  // 3. T = (I + A)^-1.  Diagonal 16x16 blocks D_b: block 2w + (lane / 16) on
+  //    warp w, lane j % 16 owning column j % 16 (half the warps issue this phase,
+  //    which leaves the SM's issue slots to the other resident CTAs);
+  //    right-looking, so only one multiply-add per step is on the dependency chain.
+  if (warp < kC / 32) {  // two diagonal blocks per warp, one per half-warp
+    const int o = 16 * (2 * warp + (lane >> 4)), j = lane & 15;
     float col[16], acc[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
 #pragma unroll
       for (int i = m + 1; i < 16; ++i) acc[i] = fmaf(Am[(o + i) * kApad + o + m], col[m], acc[i]);
     }
-    __syncwarp(0x0000FFFFu);  // every lane has read its block of A before T may overwrite it
+    __syncwarp();  // every lane has read its block of A before T may overwrite it
 #pragma unroll
     for (int i = 0; i < 16; ++i) Tm[(o + i) * kApad + o + j] = col[i];
   }
@@ -320,7 +322,7 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
         mac(acc, At(a + 1, a), Tt(a, a));
         put(At(a, a + 1), acc, false);
       }
-      __syncthreads();
+      __syncwarp();  // level 2 reads back only this warp's level-1 tile
       if (wl < 2) {  // level 2: T10 = -D1 S01, T32 = -D3 S23
         const int a = b0 + 2 * wl;
         wmma::fill_fragment(acc, 0.f);
