@@ -252,7 +252,10 @@ __global__ void __launch_bounds__(2 * C, C == 64 ? 8 : 2)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  // At C = 64 warp w extracted rows 32 w .. + 31 of A, exactly the rows of the
+  // two diagonal blocks it solves below; at C = 128 other warps wrote half of them.
+  if constexpr (kC == 64) __syncwarp();
+  else __syncthreads();
 
   // 3. T = (I + A)^-1.  Diagonal 16x16 blocks D_b: block 2w + (lane / 16) on
   //    warp w, lane j % 16 owning column j % 16 (half the warps issue this phase,
