@@ -11,7 +11,6 @@
 //   combine: Sin[1] = Send[0], Sin[g+1] = A[g] Sin[g] + Send[g], S_out = A[G-1] Sin[G-1] + Send[G-1];
 //   correct: O_g = O'_g + R_g Sin[g] for g >= 1 (the outputs are linear in the entry state).
 #include <cuda_bf16.h>
-#include <mma.h>
 
 #include <algorithm>
 #include <climits>
@@ -21,8 +20,6 @@
 
 namespace dn {
 namespace {
-
-using namespace nvcuda;
 
 // 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros and reads nothing.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
