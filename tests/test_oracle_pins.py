@@ -505,3 +505,52 @@ def test_gradient_of_a_single_write(oracle_mod):
     np.testing.assert_allclose(g["dq"][0, 0, 0], 0.5 * vdo * k[0, 0, 0])
     Gt = np.outer(q[0, 0, 0], dO[0, 0, 0]) + dS[0, 0]
     np.testing.assert_allclose(g["dS0"][0, 0], Gt - 0.5 * np.outer(k[0, 0, 0], k[0, 0, 0] @ Gt))
+
+
+# -- the affine chunk transition behind the sequence split ------------------------
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_segments_joined_by_their_affine_maps_give_the_whole_sequence(oracle_mod, gated):
+    """The transition over any run of tokens is affine in the entry state ("GPT-2
+    から Kimi K3 まで", section "DeltaNet (Parallelizing linear transformers with
+    delta rule)": a product of generalised Householder factors, each decayed by
+    its gate, plus the writes).  So, on the oracle alone: run each segment from a
+    zero state (outputs O', end state S_end) and its homogeneous chain (v = 0
+    from S0 = I: outputs R, end state A = the product of its transitions); then
+    S_in of the next segment = A S_in + S_end and the segment's outputs are
+    O' + R S_in.  Joined over unequal, ragged segments this must reproduce the
+    whole sequence from S0, outputs and final state."""
+    rng = np.random.default_rng(17 + gated)
+    B, H, T, Dk, Dv = 1, 2, 300, 8, 6
+    q = torch.from_numpy(_rand((B, H, T, Dk), rng))
+    k = torch.from_numpy(_unit_rows(_rand((B, H, T, Dk), rng)))
+    v = torch.from_numpy(_rand((B, H, T, Dv), rng))
+    beta = torch.from_numpy(rng.uniform(0.1, 1.0, (B, H, T)).astype(np.float32))
+    alpha = torch.from_numpy(rng.uniform(0.85, 1.0, (B, H, T)).astype(np.float32)) if gated else None
+    S0 = rng.standard_normal((B, H, Dk, Dv))
+    o_whole, S_whole = oracle_mod.deltanet(q, k, v, beta, alpha, S0)
+
+    eye = np.broadcast_to(np.eye(Dk), (B, H, Dk, Dk)).copy()
+    S_in = S0
+    o_join = np.zeros_like(o_whole)
+    for a, b in ((0, 110), (110, 171), (171, 300)):
+        sl = slice(a, b)
+        part = lambda x: None if x is None else x[:, :, sl].contiguous()
+        o_zero, S_end = oracle_mod.deltanet(part(q), part(k), part(v), part(beta), part(alpha))
+        zeros = torch.zeros(B, H, b - a, Dk)
+        R, A = oracle_mod.deltanet(part(q), part(k), zeros, part(beta), part(alpha), eye)
+        o_join[:, :, sl] = o_zero + R @ S_in
+        S_in = A @ S_in + S_end
+    scale = np.abs(o_whole).max()
+    assert np.abs(o_join - o_whole).max() <= 1e-11 * scale
+    assert np.abs(S_in - S_whole).max() <= 1e-11 * np.abs(S_whole).max()
+    # and the homogeneous chain's end state is the product of its transitions:
+    # entered with any state X it carries X to A X
+    X = rng.standard_normal((B, H, Dk, Dv))
+    _, S_X = oracle_mod.deltanet(q[:, :, :50].contiguous(), k[:, :, :50].contiguous(), torch.zeros(B, H, 50, Dv),
+                                 beta[:, :, :50].contiguous(), None if alpha is None else alpha[:, :, :50].contiguous(),
+                                 X)
+    _, A50 = oracle_mod.deltanet(q[:, :, :50].contiguous(), k[:, :, :50].contiguous(), torch.zeros(B, H, 50, Dk),
+                                 beta[:, :, :50].contiguous(), None if alpha is None else alpha[:, :, :50].contiguous(),
+                                 eye)
+    assert np.abs(S_X - A50 @ X).max() <= 1e-12 * np.abs(S_X).max()
