@@ -32,7 +32,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-constexpr int kCombCols = 16;  // Dv columns per combine CTA
 
 // tf32 tensor-core product D += A B on one 16 x 8 tile (mma.sync m16n8k8,
 // float32 accumulation).  Lane l holds A at rows l/4 (a0, a2) and l/4 + 8
@@ -55,7 +54,7 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
 }
 
-// One CTA per (b, h, 16-column slice of Dv), DK / 8 warps: the G - 1
+// One CTA per (b, h, NC-column slice of Dv; NC = 8 or 16), DK / 8 warps: the G - 1
 // sequential steps S <- A[g] S + Send[g], each product on the tensor cores as
 // three tf32 products of the split operands, accumulated in float32.  Warp w
 // takes rows 16 (w % (DK/16)) .. + 15 of the slice and one half of the k
@@ -63,22 +62,23 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
 // The state is kept already split (tf32 hi and lo words), A[g + 1] streams
 // into shared memory while step g computes, and each step's Send values are
 // loaded before its product and added after it.
-template <int DK>
+template <int DK, int NC>
 __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __restrict__ Send,
                                                               const float* __restrict__ A, float* __restrict__ Sin,
                                                               float* __restrict__ S_out, int G, int Dv) {
   constexpr int NT = 4 * DK;   // threads
   constexpr int RW = DK / 16;  // row groups (warps per k half)
   constexpr int AP = DK + 4;   // padded row of A: fragment reads hit 32 banks
-  constexpr int CS = 24;       // padded row of the 16-column state: likewise
+  constexpr int NTL = NC / 8;  // 8-column tiles of the slice
+  constexpr int CS = NC == 16 ? 24 : 8;  // (padded) row of the state slice: fragment reads hit 32 banks
   constexpr int KH = DK / 16;  // 8-wide k tiles per half
   extern __shared__ __align__(16) float seg_smem[];
   float* As = seg_smem;                                             // 2 x DK x AP
   uint32_t* ch = reinterpret_cast<uint32_t*>(As + 2 * DK * AP);     // DK x CS, state (tf32 hi)
   uint32_t* cl = ch + DK * CS;                                      // DK x CS, state (tf32 lo)
-  float* red = reinterpret_cast<float*>(cl + DK * CS);              // RW x 256, second-half sums
-  const int nsl = Dv / kCombCols;
-  const int bh = blockIdx.x / nsl, j0 = (blockIdx.x % nsl) * kCombCols;
+  float* red = reinterpret_cast<float*>(cl + DK * CS);              // RW x (NTL x 128), second-half sums
+  const int nsl = Dv / NC;
+  const int bh = blockIdx.x / nsl, j0 = (blockIdx.x % nsl) * NC;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rw = warp % RW, kh = warp / RW, r0 = 16 * rw;
   const int lr = lane / 4, lc = lane % 4;
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
     }
     cp_async_commit();
   };
-  // this lane's 8 values of a 16-column slice: rows r0 + lr + 8 h, columns 8 nt + 2 lc + {0, 1}
+  // this lane's values of the slice: rows r0 + lr + 8 h, columns 8 nt + 2 lc + {0, 1}
   auto elem = [&](int nt, int h) { return (size_t)(r0 + lr + 8 * h) * Dv + j0 + 8 * nt + 2 * lc; };
   auto put_state = [&](int nt, int h, float x0, float x1) {
     const int c = (r0 + lr + 8 * h) * CS + 8 * nt + 2 * lc;
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
   // Sin[1] = Send[0]
   if (kh == 0) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NTL; ++nt)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float2 x = *reinterpret_cast<const float2*>(Send + (size_t)bh * G * sblk + elem(nt, h));
@@ -115,10 +115,10 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
   }
   for (int g = 1; g < G; ++g) {
     const int buf = (g - 1) & 1;
-    float2 sg[2][2];
+    float2 sg[NTL][2];
     if (kh == 0) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NTL; ++nt)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
           sg[nt][h] = *reinterpret_cast<const float2*>(Send + ((size_t)bh * G + g) * sblk + elem(nt, h));
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
     __syncthreads();  // A[g] and the state are complete; red is free
     // independent accumulators (k-tile parity x column tile, the hi*hi
     // product apart from the two correction terms) keep eight mma chains in flight
-    float big[2][2][4] = {}, sml[2][2][4] = {};
+    float big[2][NTL][4] = {}, sml[2][NTL][4] = {};
     const float* Ab = As + buf * DK * AP + (r0 + lr) * AP + lc;
 #pragma unroll
     for (int j = 0; j < KH; ++j) {
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
       split_tf32(Ab[8 * kt + 4], ah[2], al[2]);
       split_tf32(Ab[8 * AP + 8 * kt + 4], ah[3], al[3]);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < NTL; ++nt) {
         const int b0 = (8 * kt + lc) * CS + 8 * nt + lr, b1 = b0 + 4 * CS;
         const uint32_t bhi[2] = {ch[b0], ch[b1]}, blo[2] = {cl[b0], cl[b1]};
         mma_1688_tf32(sml[j & 1][nt], al, bhi);
@@ -151,17 +151,17 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
         mma_1688_tf32(big[j & 1][nt], ah, bhi);
       }
     }
-    float acc[2][4];
+    float acc[NTL][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NTL; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         acc[nt][e] = (big[0][nt][e] + big[1][nt][e]) + (sml[0][nt][e] + sml[1][nt][e]);
     if (kh == 1) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NTL; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) red[rw * 256 + (4 * nt + e) * 32 + lane] = acc[nt][e];
+        for (int e = 0; e < 4; ++e) red[rw * NTL * 128 + (4 * nt + e) * 32 + lane] = acc[nt][e];
     }
     __syncthreads();  // every warp has read the state and As[buf]; red holds the second halves
     if (kh == 0) {
@@ -169,11 +169,12 @@ __global__ void __launch_bounds__(4 * DK) seg_combine_kernel(const float* __rest
       float* dst =
           g + 1 < G ? Sin + ((size_t)bh * G + g + 1) * sblk : (S_out ? S_out + (size_t)bh * sblk : nullptr);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NTL; ++nt)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float x0 = acc[nt][2 * h] + red[rw * 256 + (4 * nt + 2 * h) * 32 + lane] + sg[nt][h].x;
-          const float x1 = acc[nt][2 * h + 1] + red[rw * 256 + (4 * nt + 2 * h + 1) * 32 + lane] + sg[nt][h].y;
+          const float x0 = acc[nt][2 * h] + red[rw * NTL * 128 + (4 * nt + 2 * h) * 32 + lane] + sg[nt][h].x;
+          const float x1 =
+              acc[nt][2 * h + 1] + red[rw * NTL * 128 + (4 * nt + 2 * h + 1) * 32 + lane] + sg[nt][h].y;
           put_state(nt, h, x0, x1);
           if (dst) *reinterpret_cast<float2*>(dst + elem(nt, h)) = make_float2(x0, x1);
         }
@@ -305,14 +306,15 @@ __global__ void __launch_bounds__(DV) seg_correct_kernel(__nv_bfloat16* __restri
   }
 }
 
-template <int DK>
+template <int DK, int NC>
 cudaError_t combine_t(const float* Send, const float* A, float* Sin, float* S_out, int BH, int G, int Dv,
                       cudaStream_t st) {
-  const size_t smem = (size_t)(2 * DK * (DK + 4) + 2 * DK * 24 + (DK / 16) * 256) * sizeof(float);
-  auto kern = seg_combine_kernel<DK>;
+  constexpr int CS = NC == 16 ? 24 : 8;
+  const size_t smem = (size_t)(2 * DK * (DK + 4) + 2 * DK * CS + (DK / 16) * (NC / 8) * 128) * sizeof(float);
+  auto kern = seg_combine_kernel<DK, NC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(BH * (Dv / kCombCols)), 4 * DK, smem, st>>>(Send, A, Sin, S_out, G, Dv);
+  kern<<<(unsigned)(BH * (Dv / NC)), 4 * DK, smem, st>>>(Send, A, Sin, S_out, G, Dv);
   return cudaGetLastError();
 }
 
@@ -350,9 +352,16 @@ cudaError_t correct_t(void* o, const void* R, const float* Sin, int BH, int G, i
 
 cudaError_t launch_seg_combine(const float* Send, const float* A, float* Sin, float* S_out, int BH, int G,
                                int Dk, int Dv, cudaStream_t st) {
-  if (G < 2 || Dv % kCombCols != 0) return cudaErrorInvalidValue;
-  if (Dk == 128) return combine_t<128>(Send, A, Sin, S_out, BH, G, Dv, st);
-  if (Dk == 64) return combine_t<64>(Send, A, Sin, S_out, BH, G, Dv, st);
+  if (G < 2 || Dv % 16 != 0) return cudaErrorInvalidValue;
+  // The steps are sequential, so every CTA of one call should be resident at
+  // once: 8-column slices (twice the CTAs, half the work per step) while they fit one wave.
+  const bool narrow = (long long)BH * (Dv / 8) <= sm_count_dev();
+  if (Dk == 128)
+    return narrow ? combine_t<128, 8>(Send, A, Sin, S_out, BH, G, Dv, st)
+                  : combine_t<128, 16>(Send, A, Sin, S_out, BH, G, Dv, st);
+  if (Dk == 64)
+    return narrow ? combine_t<64, 8>(Send, A, Sin, S_out, BH, G, Dv, st)
+                  : combine_t<64, 16>(Send, A, Sin, S_out, BH, G, Dv, st);
   return cudaErrorNotSupported;
 }
 
