@@ -21,6 +21,7 @@
 //              tcgen05.mma of the CTA, in a fixed order that keeps the state
 //              chain fed:
 //                [Q;W]S (c), W/Uh (c+1), K^T U (c), PU (c), QK^T (c+1)
+//              (gated: W (c+1) before K^T U (c), Uh (c+1) after it)
 //              W/Uh (c+1) runs while the U epilogue of chunk c drains (Uh is
 //              double-buffered in TMEM); PU (c) and QK^T (c+1) run during the
 //              state update.  The single P tile is rewritten only after PU (c)
@@ -303,6 +304,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
+    // Gated: W (c) and Uh (c) issued apart (they share no operand), so that
+    // only W (c+1) sits in the pipe ahead of K^T U (c)
+    auto issue_w_only = [&](int c) {
+      const uint32_t st = stage(c);
+      constexpr uint32_t idw = idesc_bf16(128, DK, false, true);
+      const uint64_t dw = desc_k(st + L::TB_OFF), dk = desc_mn(st + L::K_OFF, L::KB_STRIDE);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16_ss_elect(tmem + TM_W, desc_step(dw, ks * 32), desc_step(dk, ks * 2048), idw, ks > 0);
+    };
+    auto issue_uh_only = [&](int c) {
+      const uint32_t st = stage(c);
+      constexpr uint32_t idu = idesc_bf16(128, DVS, false, true);
+      const uint64_t dt = desc_k(st + L::V_OFF), dv = desc_mn(st + L::V_OFF + vcol, kTile);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_bf16_ss_elect(tmem + ((c & 1) ? TM_UH1 : TM_UH0), desc_step(dt, ks * 32), desc_step(dv, ks * 2048), idu,
+                          ks > 0);
+    };
     // [Q S ; W S] (lanes 0-63 ; 64-127 of TM_QW[c & 1])
     auto issue_qw = [&](int c) {
       const uint32_t st = stage(c);
@@ -353,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar + B_FULL + 8 * ((c + 1) % NST), ((c + 1) / NST) & 1, wc));
         if (!ok) break;
         tc_fence_after();
-        issue_wu(c + 1);
+        if (GATED) issue_w_only(c + 1);
+        else issue_wu(c + 1);
         mma_commit_elect(bar + B_PMMA2);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar + B_UREADY, c & 1, wc));
@@ -361,6 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       issue_ds(c);
       mma_commit_elect(bar + B_CMMA4);
+      // gated: Uh (c+1) after K^T U (c); the U epilogue of chunk c+1 reads it after
+      // [Q;W]S (c+1), which the in-order pipe completes later still
+      if (GATED && c + 1 < nchunks) issue_uh_only(c + 1);
       // K^T U (c) is the last MMA that reads stage c.  Ungated the stage is
       // free now (its W / Q epilogues came before W_READY); gated the P rows
       // of chunk c still read its g rows, so it goes once they are done.
